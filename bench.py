@@ -1,0 +1,407 @@
+"""Benchmark of the partially synchronized row-parallel FC2 (7B shape) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl caat|reference]
+                    [--workload fc2-7b|fc2-1b|tiny] [--p 0.5] [--sweep]
+
+One step = one call of caat_rowpar_forward on one batch of synthetic input: the P partial
+GEMMs, the partial channel-reduce, the private scale, the residual add and the per-rank
+RMSNorm.  Default workload: T=8192 tokens, H=4096, K=11008 split over P=8 emulated ranks,
+p=0.5 with the first 2048 channels shared (the 7B-scale FC2).  Each step touches 1.34 GB,
+more than the 126 MB L2, so no flush is needed between steps.
+
+N > 1 (torchrun): every rank runs its own independent batch of the same workload on its own
+GPU (tokens are independent through the whole path: no data-path collective), so per-GPU
+work is fixed ("weak" scaling).  Timing: CUDA events around exactly K steps, barrier and
+synchronize on both sides, max over ranks.
+
+Prints ONE JSON line on rank 0.  --impl reference times the float64 CPU oracle (the only
+reference this method has) on a bounded row sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+WORKLOADS = {
+    # name: (T, K, H, P, default p, random S?)
+    "fc2-7b": (8192, 11008, 4096, 8, 0.5, False),
+    "fc2-1b": (4096, 5632, 2048, 4, 0.5, True),
+    "tiny": (256, 768, 768, 2, 0.5, False),
+}
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_desc(name, T, K, H, P, p, rand):
+    return (f"{name}: partially synced row-parallel FC2 + residual + RMSNorm, T={T} H={H} K={K} P={P} "
+            f"p={p} ({'seeded random' if rand else 'contiguous'} S)")
+
+
+# ---------------------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        time.sleep(0.3)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "samples": len(sm),
+                "power_w_max": max(power) if power else None, "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------------------
+# CPU baseline: the float64 oracle on a bounded row sample
+# ---------------------------------------------------------------------------------------
+def cpu_baseline(T, K, H, P, p, sync_idx, target_s=10.0, seed=0):
+    import numpy as np
+    from oracle import caat_oracle as O
+    from partial_activation_sync_caat_b200 import inputs as I
+
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = len(os.sched_getaffinity(0))
+    # a sample of token rows; weights at full size
+    n_rows = 16
+    d = I.make_rowpar_inputs(min(T, 2048), K, H, P, seed=seed)
+    flops_per_row = 2.0 * K * H
+    t_total, rows_done = 0.0, 0
+    while True:
+        rows = np.arange(min(n_rows, d["X"].shape[1]))
+        t0 = time.perf_counter()
+        O.rowpar_rows(d["X"], d["W"], d["R"], d["gamma"], P, p, rows, sync_idx)
+        dt = time.perf_counter() - t0
+        t_total += dt
+        rows_done += len(rows)
+        if t_total >= target_s or len(rows) >= d["X"].shape[1]:
+            break
+        n_rows = int(min(d["X"].shape[1], max(2 * n_rows, n_rows * (target_s - t_total) / max(dt, 1e-3))))
+    tflops = flops_per_row * rows_done / t_total / 1e12
+    return {"value": tflops, "unit": "TFLOP/s", "cores": int(threads), "kind": "oracle",
+            "sample": f"{rows_done} token rows (all {P} ranks, full H={H}, K={K}) of the workload, "
+                      f"{t_total:.1f} s of float64 NumPy on the host",
+            "tokens_per_s": rows_done / t_total}
+
+
+# ---------------------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------------------
+def run_caat(args):
+    import torch
+    import torch.distributed as dist
+    from partial_activation_sync_caat_b200 import build as B
+    from partial_activation_sync_caat_b200 import caat as C
+    from partial_activation_sync_caat_b200 import inputs as I
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    if rank == 0:
+        B.build()
+    if world > 1:
+        dist.barrier()
+    C.lib()
+
+    T, K, H, P, p_def, rand = WORKLOADS[args.workload]
+    p = args.p if args.p is not None else p_def
+    ns = int((H * p) // 1)
+    sync_idx = I.random_sync_idx(H, ns, seed=0) if rand else None
+    d = I.make_rowpar_inputs(T, K, H, P, seed=1000 + rank, device="cuda")
+    out = torch.empty_like(d["R"])
+    ws = C.alloc_workspace(C.caat_workspace_size(T, K, H, P), "cuda")
+    stream = torch.cuda.current_stream()
+    flops = 2.0 * T * K * H
+    timing = C.Timing(capacity=args.steps + 8)
+
+    def step(tm=None):
+        C.caat_rowpar_forward(d["X"], d["W"], d["R"], d["gamma"], sync_idx, P, p, out, workspace=ws,
+                              stream=stream, timing=tm)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if C.caat_get_device_status() != 0:
+        raise SystemExit("device status set during warm-up")
+
+    sampler = ClockSampler(local) if rank == 0 else None
+    if sampler:
+        sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step(timing)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    per_kernel = timing.read()
+    k1 = [r[0] for r in per_kernel if len(r) >= 1]
+    k2 = [r[1] for r in per_kernel if len(r) >= 2]
+    status = C.caat_get_device_status()
+
+    # optional p sweep (same shapes, fewer steps), rank 0 only
+    sweep = None
+    if args.sweep and rank == 0:
+        sweep = {}
+        for ps in (0.0, 0.25, 0.5, 0.75, 1.0):
+            idx_s = I.random_sync_idx(H, int((H * ps) // 1), seed=0) if rand else None
+            for _ in range(2):
+                C.caat_rowpar_forward(d["X"], d["W"], d["R"], d["gamma"], idx_s, P, ps, out, workspace=ws)
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            n = max(3, args.steps // 2)
+            a.record()
+            for _ in range(n):
+                C.caat_rowpar_forward(d["X"], d["W"], d["R"], d["gamma"], idx_s, P, ps, out, workspace=ws)
+            b.record()
+            torch.cuda.synchronize()
+            t_ms = a.elapsed_time(b) / n
+            sweep[str(ps)] = {"ms_per_step": round(t_ms, 4), "tflops": round(flops / t_ms / 1e9, 1)}
+
+    # end to end through the host-buffer entry point (pinned host tensors, copies timed)
+    e2e = None
+    if not args.no_e2e:
+        hX, hW, hR, hg = (d[k].cpu().pin_memory() for k in ("X", "W", "R", "gamma"))
+        hout = torch.empty(hR.shape, dtype=torch.bfloat16).pin_memory()
+        wsh = C.alloc_workspace(C.caat_workspace_size(T, K, H, P, C.CAAT_VARIANT_ROWPAR_HOST), "cuda")
+        for _ in range(2):
+            C.caat_rowpar_forward_host(hX, hW, hR, hg, sync_idx, P, p, hout, wsh, stream=stream)
+        torch.cuda.synchronize()
+        n_e2e = max(3, min(args.steps, 10))
+        if world > 1:
+            dist.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n_e2e):
+            C.caat_rowpar_forward_host(hX, hW, hR, hg, sync_idx, P, p, hout, wsh, stream=stream)
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = a.elapsed_time(b) / n_e2e
+        if world > 1:
+            t = torch.tensor([e_ms], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        h2d = sum(x.numel() * 2 for x in (hX, hW, hR, hg))
+        d2h = hout.numel() * 2
+        e2e = {"value": round(world * flops / e_ms / 1e9, 2), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms, 3),
+               "api": "caat_rowpar_forward_host (pinned host buffers; H2D of X, W, residual, gamma and "
+                      "D2H of out inside the timed region)"}
+        del wsh
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks, peak_src = load_peaks()
+    ms_step = ms / args.steps
+    value = world * flops / ms_step / 1e9  # TFLOP/s, whole job
+    k1_ms = statistics.mean(k1) if k1 else float("nan")
+    k2_ms = statistics.mean(k2) if k2 else float("nan")
+    k1_tflops = flops / k1_ms / 1e9
+    norm_bytes = 2.0 * P * T * H * 2
+    k2_gbs = norm_bytes / k2_ms / 1e6
+    alg_bytes = 2.0 * (P * T * (K // P) + P * H * (K // P) + 2 * P * T * H + H)
+    result = {
+        "metric": "TFLOP/s & tokens/s of partially-synced row-parallel FC2 (7B shape), % bf16 peak",
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) activations and residual, N(0,0.02) weights, gamma=1)",
+        "config": {"workload": workload_desc(args.workload, T, K, H, P, p, rand), "T": T, "H": H, "K": K,
+                   "P": P, "p": p, "parallelism": f"{world} independent GPU(s), P={P} emulated TP ranks each",
+                   "l2": "inputs larger than L2 (%.2f GB touched per step); no flush" % (alg_bytes / 1e9)},
+        "tokens_per_s": round(world * T / (ms_step / 1e3), 1),
+        "pct_bf16_peak": {"measured_burst": round(100 * value / world / peaks["bf16_tflops"], 1),
+                          "datasheet_2250": round(100 * value / world / 2250.0, 1)},
+        "roofline": {"kernel": "rowpar_gemm_kernel (tcgen05 GEMM + partial channel-reduce + residual)",
+                     "bound": "tensor", "achieved": round(k1_tflops, 1), "peak": peaks["bf16_tflops"],
+                     "peak_source": f"{peak_src} bf16 burst", "unit": "TFLOP/s",
+                     "frac": round(k1_tflops / peaks["bf16_tflops"], 3),
+                     "frac_vs_sustained": round(k1_tflops / peaks["bf16_tflops_sustained"], 3),
+                     "traffic": None, "launch_ms": round(k1_ms, 4),
+                     "algorithmic": "2*T*K*H flops per launch"},
+        "norm_kernel": {"kernel": "rownorm_kernel", "bound": "hbm", "achieved": round(k2_gbs, 1),
+                        "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(k2_gbs / peaks["hbm_gbs"], 3),
+                        "launch_ms": round(k2_ms, 4), "algorithmic": "2*P*T*H*2 bytes (read h, write out)"},
+        "gpu_launches": 2 * args.steps,
+        "device_status": status,
+        "clocks": clocks,
+    }
+    if sweep is not None:
+        result["p_sweep"] = sweep
+    if e2e is not None:
+        result["e2e"] = e2e
+    if not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(T, K, H, P, p, sync_idx, target_s=args.cpu_seconds)
+    print(json.dumps(result))
+
+
+# ---------------------------------------------------------------------------------------
+# reference arm: the float64 oracle on the host cores
+# ---------------------------------------------------------------------------------------
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    import numpy as np
+    from oracle import caat_oracle as O
+    from partial_activation_sync_caat_b200 import inputs as I
+
+    T, K, H, P, p_def, rand = WORKLOADS[args.workload]
+    p = args.p if args.p is not None else p_def
+    sync_idx = I.random_sync_idx(H, O.n_sync(H, p), seed=0) if rand else None
+    rows_per_step = args.ref_rows
+    d = I.make_rowpar_inputs(rows_per_step, K, H, P, seed=0)
+    rows = np.arange(rows_per_step)
+    for _ in range(args.warmup):
+        O.rowpar_rows(d["X"], d["W"], d["R"], d["gamma"], P, p, rows, sync_idx)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        O.rowpar_rows(d["X"], d["W"], d["R"], d["gamma"], P, p, rows, sync_idx)
+    dt = (time.perf_counter() - t0) / args.steps
+    flops = 2.0 * rows_per_step * K * H
+    value = flops / dt / 1e12
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = len(os.sched_getaffinity(0))
+    sample = f"{rows_per_step} token rows per step (all {P} ranks, full H and K) of the workload"
+    print(json.dumps({
+        "impl": "reference",
+        "metric": "TFLOP/s & tokens/s of partially-synced row-parallel FC2 (7B shape), % bf16 peak",
+        "value": round(value, 5), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_desc(args.workload, T, K, H, P, p, rand), "T": T, "H": H, "K": K,
+                   "P": P, "p": p, "parallelism": "host cores (float64 NumPy oracle)"},
+        "tokens_per_s": round(rows_per_step / dt, 2),
+        "cpu_baseline": {"value": round(value, 5), "unit": "TFLOP/s", "cores": int(threads), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 5), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["caat", "reference"], default="caat")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="fc2-7b")
+    ap.add_argument("--p", type=float, default=None)
+    ap.add_argument("--sweep", action="store_true", help="also time p in {0,.25,.5,.75,1}")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--ref-rows", type=int, default=64)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_caat(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,213 @@
+/*
+ * caat.h - C ABI of the B200 (sm_100a) library for the partially synchronized
+ * row-parallel linear layer of CAAT-Net.
+ *
+ * Source of every operation: "Tensor-Parallelism with Partially Synchronized Activations"
+ * (Lamprecht, Karnieli, Hanani, Giladi, Soudry; arXiv 2506.19645).
+ *
+ *   - P tensor-parallel ranks are emulated side by side in one GPU's memory, as the paper's
+ *     "logical devices" (§3.2): the partial channel-reduce becomes an on-chip sum.
+ *   - Partial products: Zt_m = X_m W_m^T over rank m's K/P slice (§3.1 Eq. 4-5, App. A.2
+ *     Eq. 21-22; W_m is the row-parallel block B~_m, stored transposed).
+ *   - Partial channel-reduce (App. A.2 Eq. 22; §3.1 Eq. 8): for the shared channels
+ *     c in S, |S| = floor(H p), every rank gets sum_m Zt_m[:, c]; the private channels keep
+ *     the rank's own Zt_m[:, c], optionally times private_scale (§4 Eq. 14-15: sqrt(P)).
+ *   - Residual add and norm (§4 Eq. 9, App. B Eq. 25): h_m = Z_m + R_m, then RMSNorm per
+ *     rank and token, out_m = h_m / sqrt(mean_c h_m^2 + eps) * gamma (gamma shared by the
+ *     ranks, since norm parameters are synchronized, §4).
+ *   - MLP block (§3.1 Eq. 6 with sigma = SwiGLU): Y_m = silu(X_m A_gate,m^T) * (X_m A_up,m^T),
+ *     then the layer above with X := Y.
+ *
+ * Conventions for every call below
+ *   - bf16 tensors are raw bfloat16 bit patterns (caat_bf16), row-major, last dim contiguous.
+ *   - Device pointers are owned by the caller, must be 16-byte aligned and stay valid until
+ *     the work queued on `stream` has finished.  The library never allocates device memory
+ *     and never synchronizes the stream in a forward call.
+ *   - Every forward call validates all arguments on the host first; an invalid call queues
+ *     no work and returns an error code.  No call throws across the ABI.
+ *   - Work is queued asynchronously on `stream` (a cudaStream_t; NULL = legacy default).
+ *   - Device-side waits are bounded: a wait that runs out (about 1 s) records
+ *     CAAT_ERR_TIMEOUT in a device status word, which caat_get_device_status() reads.
+ */
+#ifndef CAAT_H_
+#define CAAT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(CAAT_BUILD) && defined(__GNUC__)
+#define CAAT_API __attribute__((visibility("default")))
+#else
+#define CAAT_API
+#endif
+
+typedef uint16_t caat_bf16;                   /* bfloat16 bit pattern */
+typedef struct CUstream_st* caat_stream_t;    /* identical to cudaStream_t */
+typedef struct caat_timing caat_timing;       /* opaque per-kernel event recorder */
+
+typedef enum caat_status {
+  CAAT_OK = 0,
+  CAAT_ERR_INVALID_ARG = 1,   /* a pointer, size or value is invalid (nothing queued) */
+  CAAT_ERR_UNSUPPORTED = 2,   /* valid, but outside what the kernels handle (alignment,
+                                 divisibility, limits) or no sm_100 device */
+  CAAT_ERR_CUDA = 3,          /* a CUDA runtime call failed */
+  CAAT_ERR_TIMEOUT = 4,       /* a bounded device-side wait ran out (read from the device) */
+  CAAT_ERR_WORKSPACE = 5      /* workspace NULL, misaligned or smaller than required */
+} caat_status;
+
+/* Limits of this build. */
+#define CAAT_MAX_H 65536      /* hidden size H */
+#define CAAT_MAX_P 64         /* emulated tensor-parallel ranks */
+#define CAAT_DECODE_MAX_T 64  /* T <= this uses the decode (weight-streaming) path */
+
+/* Workspace variants for caat_workspace_size(). */
+#define CAAT_VARIANT_ROWPAR 0 /* caat_rowpar_forward[_ex]; K = FFN dim */
+#define CAAT_VARIANT_MLP 1    /* caat_mlp_forward[_ex]; K = F */
+#define CAAT_VARIANT_ROWPAR_HOST 2 /* caat_rowpar_forward_host; K = FFN dim */
+
+/* Flags of caat_rowpar_args.flags / caat_mlp_args.flags. */
+#define CAAT_FLAG_FORCE_GEMM_PATH 0x1u   /* use the tensor-core GEMM path even for small T */
+#define CAAT_FLAG_FORCE_DECODE_PATH 0x2u /* use the weight-streaming path even for large T */
+#define CAAT_FLAG_TEST_STALL 0x100u      /* test hook: the GEMM kernel's MMA warp never signals
+                                            its accumulator, so every consumer wait runs out
+                                            and the call reports CAAT_ERR_TIMEOUT through
+                                            caat_get_device_status().  Nothing faults. */
+
+/*
+ * caat_rowpar_forward - the partially synchronized row-parallel layer, residual add and
+ * per-rank RMSNorm (App. A.2 Eq. 22, §4 Eq. 9).
+ *
+ *   X         device, bf16 [P, T, K/P]   rank m's input slice X_m
+ *   W         device, bf16 [P, H, K/P]   rank m's weight block (B~_m transposed, K contiguous)
+ *   residual  device, bf16 [P, T, H]     per-rank residual R_m (App. B)
+ *   gamma     device, bf16 [H]           RMSNorm weight, shared by the ranks
+ *   sync_idx  HOST, int32, NULL or floor(H p) strictly increasing channels in [0, H).
+ *             NULL selects the first floor(H p) channels (§3).  Read before return.
+ *   P, p      ranks (1..CAAT_MAX_P) and sync factor p in [0, 1]; n_s = floor(H p) in double.
+ *   out       device, bf16 [P, T, H]     normalized output; may alias `residual`.
+ *   T, K, H   tokens (>= 0), FFN dim (K % P == 0, (K/P) % 8 == 0), hidden (H % 8 == 0).
+ *   workspace device scratch of caat_workspace_size(T, K, H, P, CAAT_VARIANT_ROWPAR) bytes,
+ *             256-byte aligned; its contents need not be initialized and are clobbered.
+ * eps = 1e-5 and private_scale = 1 (use caat_rowpar_forward_ex for other values).
+ * Returns CAAT_OK once the work is queued.
+ */
+CAAT_API caat_status caat_rowpar_forward(const caat_bf16* X, const caat_bf16* W, const caat_bf16* residual,
+                                const caat_bf16* gamma, const int32_t* sync_idx, int P, double p,
+                                caat_bf16* out, int64_t T, int64_t K, int64_t H,
+                                void* workspace, size_t ws_bytes, caat_stream_t stream);
+
+/* Extended arguments of the row-parallel layer (same meaning as above, plus): */
+typedef struct caat_rowpar_args {
+  const caat_bf16* X;
+  const caat_bf16* W;
+  const caat_bf16* residual;
+  const caat_bf16* gamma;
+  const int32_t* sync_idx;     /* host */
+  caat_bf16* out;
+  caat_bf16* h_out;            /* optional (NULL): device bf16 [P, T, H] receives the pre-norm
+                                  residual stream h = Z + R; may alias `residual` */
+  void* workspace;
+  size_t ws_bytes;
+  caat_stream_t stream;
+  caat_timing* timing;         /* optional (NULL): records CUDA events around each kernel */
+  int64_t T, K, H;
+  double p;
+  float eps;                   /* RMSNorm epsilon, >= 0, inside the square root */
+  float private_scale;         /* multiplies private channels before the residual add */
+  int32_t P;
+  uint32_t flags;              /* CAAT_FLAG_* */
+} caat_rowpar_args;
+
+CAAT_API caat_status caat_rowpar_forward_ex(const caat_rowpar_args* args);
+
+/*
+ * caat_rowpar_forward_host - the same layer for callers whose tensors live in HOST memory.
+ * args->X, W, residual, gamma, out (and h_out if not NULL) are host pointers (pinned memory
+ * for asynchronous copies; pageable memory also works, with synchronous staging).
+ * args->workspace is a device buffer of caat_workspace_size(T, K, H, P,
+ * CAAT_VARIANT_ROWPAR_HOST) bytes that receives device copies of the inputs and outputs.
+ * The call queues on args->stream: host-to-device copies of X, W, residual and gamma, the
+ * kernels of caat_rowpar_forward_ex, and device-to-host copies of out (and h_out).  The
+ * host buffers must stay valid until the stream reaches that point.
+ */
+CAAT_API caat_status caat_rowpar_forward_host(const caat_rowpar_args* args);
+
+/*
+ * caat_mlp_forward - the MLP block per rank: column-parallel FC1 with SwiGLU (§3.1 Eq. 6),
+ * then the partially synchronized FC2 (App. A.2 Eq. 22), residual add and RMSNorm (Eq. 9).
+ *
+ *   X         device, bf16 [P, T, H]        per-rank block input X_m
+ *   A         device, bf16 [P, 2F/P, H]     rank m's FC1 rows: F/P gate rows, then F/P up rows
+ *   W2        device, bf16 [P, H, F/P]      rank m's FC2 block
+ *   residual, gamma, sync_idx, P, p, out    as for caat_rowpar_forward
+ *   T, H, F   F % P == 0, (F/P) % 8 == 0, H % 8 == 0
+ *   workspace caat_workspace_size(T, F, H, P, CAAT_VARIANT_MLP) bytes (holds Y [P,T,F/P]).
+ */
+CAAT_API caat_status caat_mlp_forward(const caat_bf16* X, const caat_bf16* A, const caat_bf16* W2,
+                             const caat_bf16* residual, const caat_bf16* gamma,
+                             const int32_t* sync_idx, int P, double p, caat_bf16* out,
+                             int64_t T, int64_t H, int64_t F,
+                             void* workspace, size_t ws_bytes, caat_stream_t stream);
+
+typedef struct caat_mlp_args {
+  const caat_bf16* X;
+  const caat_bf16* A;
+  const caat_bf16* W2;
+  const caat_bf16* residual;
+  const caat_bf16* gamma;
+  const int32_t* sync_idx;     /* host */
+  caat_bf16* out;
+  caat_bf16* h_out;            /* optional pre-norm residual stream, as in caat_rowpar_args */
+  void* workspace;
+  size_t ws_bytes;
+  caat_stream_t stream;
+  caat_timing* timing;
+  int64_t T, H, F;
+  double p;
+  float eps;
+  float private_scale;
+  int32_t P;
+  uint32_t flags;
+} caat_mlp_args;
+
+CAAT_API caat_status caat_mlp_forward_ex(const caat_mlp_args* args);
+
+/* Bytes of device workspace a forward call of this shape needs (0 for invalid shapes is
+ * never returned: invalid shapes give SIZE_MAX).  variant: CAAT_VARIANT_*; for the MLP
+ * variant K is F. */
+CAAT_API size_t caat_workspace_size(int64_t T, int64_t K, int64_t H, int P, int variant);
+
+/*
+ * caat_sync_mask - host-only sync-set bookkeeping (App. A.2 Eq. 22; §3): n_s = floor(H p)
+ * in double, S = first n_s channels (sync_idx NULL) or the given list, validated exactly as
+ * the forward calls validate it.  mask_out (host, H bytes, may be NULL) receives 1 for
+ * shared and 0 for private channels; n_sync_out (may be NULL) receives n_s.  No GPU needed.
+ */
+CAAT_API caat_status caat_sync_mask(int64_t H, double p, const int32_t* sync_idx, uint8_t* mask_out,
+                           int64_t* n_sync_out);
+
+/* Synchronizes `stream`, returns the device status word recorded by bounded waits since the
+ * last call (0 = none; low byte = caat_status, upper bits = where) and clears it. */
+CAAT_API caat_status caat_get_device_status(caat_stream_t stream, int32_t* status_out);
+
+/* Event recorder for per-kernel device timing (outside the hot path: create once).
+ * Each forward call given a recorder appends one record: events before the first kernel and
+ * after each kernel it launches.  caat_timing_read synchronizes on the last event and
+ * returns, for record i and kernel j, ms[i * max_kernels + j]. */
+CAAT_API caat_status caat_timing_create(int capacity, caat_timing** out);
+CAAT_API caat_status caat_timing_destroy(caat_timing* t);
+CAAT_API caat_status caat_timing_reset(caat_timing* t);
+CAAT_API caat_status caat_timing_read(caat_timing* t, float* ms, int max_records, int max_kernels,
+                             int* n_records, int* n_kernels);
+
+CAAT_API const char* caat_status_string(caat_status s);
+CAAT_API const char* caat_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CAAT_H_ */

@@ -1,0 +1,525 @@
+// caat_api.cu - host side of the C ABI declared in include/caat.h: argument validation,
+// sync-set bookkeeping, tensor-map construction, kernel launches, timing and status.
+//
+// Source of the operations: "Tensor-Parallelism with Partially Synchronized Activations"
+// (App. A.2 Eq. 22; §3 shared channels = first floor(h p); §3.1 Eq. 6 and 8; §4 Eq. 9 and
+// 14-15).  The device code lives in the *.cuh files included below.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "caat.h"
+#include "ptx.cuh"
+#include "rowpar_gemm.cuh"
+#include "rownorm.cuh"
+
+namespace {
+
+using caat::RowparParams;
+
+constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;  // bounded device waits: 2 s
+
+// ---------------------------------------------------------------------------------------
+// Device info and one-time kernel attributes (per device)
+// ---------------------------------------------------------------------------------------
+struct DeviceInfo {
+  bool init = false;
+  bool supported = false;
+  int sm_count = 0;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[64];
+
+caat_status device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return CAAT_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return CAAT_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.init) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return CAAT_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return CAAT_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return CAAT_ERR_CUDA;
+    d.sm_count = sms;
+    d.supported = (major == 10 && minor == 0);
+    if (d.supported) {
+      if (cudaFuncSetAttribute(caat::rowpar_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               caat::K1_SMEM_BYTES) != cudaSuccess)
+        return CAAT_ERR_CUDA;
+    }
+    d.init = true;
+  }
+  if (!d.supported) return CAAT_ERR_UNSUPPORTED;
+  *out = &d;
+  return CAAT_OK;
+}
+
+uint64_t timeout_ns() {
+  static uint64_t v = [] {
+    const char* e = std::getenv("CAAT_TIMEOUT_MS");
+    if (e && *e) {
+      const double ms = std::atof(e);
+      if (ms > 0) return static_cast<uint64_t>(ms * 1e6);
+    }
+    return kDefaultTimeoutNs;
+  }();
+  return v;
+}
+
+// ---------------------------------------------------------------------------------------
+// Tensor maps (driver entry point fetched through the runtime; no link to libcuda)
+// ---------------------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<EncodeTiledFn>(nullptr);
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// 3-D bf16 tensor [d2][d1][d0] (d0 contiguous), box {b0, b1, 1}, 128-byte swizzle.
+caat_status make_map_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0,
+                        uint32_t b1) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return CAAT_ERR_CUDA;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  const cuuint32_t box[3] = {b0, b1, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? CAAT_OK : CAAT_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------------------
+// Validation and sync-set bookkeeping
+// ---------------------------------------------------------------------------------------
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+caat_status check_shapes(int64_t T, int64_t K, int64_t H, int P, double p) {
+  if (P < 1 || P > CAAT_MAX_P) return CAAT_ERR_INVALID_ARG;
+  if (T < 0 || K <= 0 || H <= 0) return CAAT_ERR_INVALID_ARG;
+  if (!(p >= 0.0 && p <= 1.0)) return CAAT_ERR_INVALID_ARG;
+  if (K % P != 0) return CAAT_ERR_UNSUPPORTED;
+  const int64_t Kp = K / P;
+  if (Kp % 8 != 0 || Kp > (int64_t(1) << 30)) return CAAT_ERR_UNSUPPORTED;
+  if (H % 8 != 0 || H > CAAT_MAX_H) return CAAT_ERR_UNSUPPORTED;
+  if (T > (int64_t(1) << 30)) return CAAT_ERR_UNSUPPORTED;
+  return CAAT_OK;
+}
+
+int64_t n_sync_of(int64_t H, double p) {
+  return static_cast<int64_t>(std::floor(static_cast<double>(H) * p));
+}
+
+// Fills mask (H entries, 1 = shared) from (H, p, sync_idx); validates sync_idx.
+caat_status build_mask(int64_t H, double p, const int32_t* sync_idx, std::vector<uint8_t>& mask, int64_t* ns_out) {
+  if (H <= 0 || !(p >= 0.0 && p <= 1.0)) return CAAT_ERR_INVALID_ARG;
+  const int64_t ns = n_sync_of(H, p);
+  mask.assign(static_cast<size_t>(H), 0);
+  if (sync_idx == nullptr) {
+    for (int64_t c = 0; c < ns; ++c) mask[c] = 1;
+  } else {
+    int64_t prev = -1;
+    for (int64_t i = 0; i < ns; ++i) {
+      const int64_t c = sync_idx[i];
+      if (c < 0 || c >= H || c <= prev) return CAAT_ERR_INVALID_ARG;
+      mask[c] = 1;
+      prev = c;
+    }
+  }
+  if (ns_out) *ns_out = ns;
+  return CAAT_OK;
+}
+
+constexpr size_t kCounterBytes = 256;
+
+size_t rowpar_workspace(int64_t T, int64_t K, int64_t H, int P) {
+  (void)T;
+  (void)K;
+  (void)H;
+  (void)P;
+  return kCounterBytes;
+}
+
+size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
+
+// Device staging layout of caat_rowpar_forward_host: [rowpar workspace | X | W | R | gamma |
+// out | h], each region 256-byte aligned.
+struct HostLayout {
+  size_t ws, x, w, r, g, o, h, total;
+};
+
+HostLayout host_layout(int64_t T, int64_t K, int64_t H, int P) {
+  HostLayout L;
+  const size_t Kp = static_cast<size_t>(K / P);
+  L.ws = 0;
+  L.x = align256(rowpar_workspace(T, K, H, P));
+  L.w = L.x + align256(size_t(P) * T * Kp * 2);
+  L.r = L.w + align256(size_t(P) * H * Kp * 2);
+  L.g = L.r + align256(size_t(P) * T * H * 2);
+  L.o = L.g + align256(size_t(H) * 2);
+  L.h = L.o + align256(size_t(P) * T * H * 2);
+  L.total = L.h + align256(size_t(P) * T * H * 2);
+  return L;
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------------------
+// Timing recorder
+// ---------------------------------------------------------------------------------------
+struct caat_timing {
+  int capacity = 0;
+  int max_kernels = 4;
+  int n = 0;
+  std::vector<cudaEvent_t> ev;
+  std::vector<int> nk;
+};
+
+namespace {
+
+struct Recorder {
+  caat_timing* t = nullptr;
+  int rec = -1;
+  int k = 0;
+  void begin(caat_timing* tm, cudaStream_t s) {
+    t = tm;
+    if (!t || t->n >= t->capacity) {
+      t = nullptr;
+      return;
+    }
+    rec = t->n++;
+    k = 0;
+    cudaEventRecord(t->ev[rec * (t->max_kernels + 1)], s);
+  }
+  void after_kernel(cudaStream_t s) {
+    if (!t || k >= t->max_kernels) return;
+    ++k;
+    cudaEventRecord(t->ev[rec * (t->max_kernels + 1) + k], s);
+    t->nk[rec] = k;
+  }
+};
+
+// ---------------------------------------------------------------------------------------
+// The row-parallel layer: GEMM + partial channel-reduce + residual (K1), RMSNorm (K2)
+// ---------------------------------------------------------------------------------------
+caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>& mask, const DeviceInfo* dev,
+                          unsigned int* counter) {
+  const int P = a->P;
+  const int64_t T = a->T, H = a->H, Kp = a->K / P;
+  cudaStream_t st = a->stream;
+  __nv_bfloat16* hdst = reinterpret_cast<__nv_bfloat16*>(a->h_out ? a->h_out : a->out);
+
+  static thread_local RowparParams prm;  // ~10 KiB: keep it off the stack
+  std::memset(&prm, 0, sizeof(prm));
+  prm.R = reinterpret_cast<const __nv_bfloat16*>(a->residual);
+  prm.Hout = hdst;
+  prm.counter = counter;
+  prm.T = static_cast<int>(T);
+  prm.H = static_cast<int>(H);
+  prm.Kp = static_cast<int>(Kp);
+  prm.P = P;
+  prm.n_mblk = static_cast<int>((T + caat::K1_BM - 1) / caat::K1_BM);
+  prm.kblk_per_rank = static_cast<int>((Kp + caat::K1_BK - 1) / caat::K1_BK);
+  const int64_t tail = Kp - int64_t(prm.kblk_per_rank - 1) * caat::K1_BK;
+  prm.last_k16 = static_cast<int>((tail + 15) / 16);
+  prm.private_scale = a->private_scale;
+  prm.timeout_ns = timeout_ns();
+  prm.flags = a->flags;
+  const int nblk = static_cast<int>((H + caat::K1_BN - 1) / caat::K1_BN);
+  for (int nb = 0; nb < nblk; ++nb) {
+    const int64_t c0 = int64_t(nb) * caat::K1_BN;
+    const int64_t c1 = std::min<int64_t>(H, c0 + caat::K1_BN);
+    int64_t cnt = 0;
+    for (int64_t c = c0; c < c1; ++c) cnt += mask[c];
+    const uint8_t cls = cnt == 0 ? 0 : (cnt == c1 - c0 ? 1 : 2);
+    prm.ncls[nb] = cls;
+    if (cls != 0) prm.slist[prm.nS++] = static_cast<uint16_t>(nb);
+    if (cls != 1) prm.plist[prm.nPriv++] = static_cast<uint16_t>(nb);
+  }
+  for (int64_t c = 0; c < H; ++c)
+    if (mask[c]) prm.mask_bits[c >> 5] |= 1u << (c & 31);
+  const int64_t units = int64_t(prm.n_mblk) * (prm.nS + int64_t(P) * prm.nPriv);
+  if (units > INT32_MAX / 2) return CAAT_ERR_UNSUPPORTED;
+  prm.n_units = static_cast<int>(units);
+
+  CUtensorMap tmX, tmW;
+  caat_status s = make_map_3d(&tmX, a->X, Kp, T, P, caat::K1_BK, caat::K1_BM);
+  if (s != CAAT_OK) return s;
+  s = make_map_3d(&tmW, a->W, Kp, H, P, caat::K1_BK, caat::K1_BN);
+  if (s != CAAT_OK) return s;
+
+  Recorder rec;
+  rec.begin(a->timing, st);
+  if (cudaMemsetAsync(counter, 0, sizeof(unsigned int), st) != cudaSuccess) return CAAT_ERR_CUDA;
+  const int grid = static_cast<int>(std::min<int64_t>(dev->sm_count, units));
+  caat::rowpar_gemm_kernel<<<grid, caat::K1_THREADS, caat::K1_SMEM_BYTES, st>>>(tmX, tmW, prm);
+  if (cudaGetLastError() != cudaSuccess) return CAAT_ERR_CUDA;
+  rec.after_kernel(st);
+
+  const int64_t rows = int64_t(P) * T;
+  const int64_t warps_per_block = caat::K2_THREADS / 32;
+  const int64_t blocks = std::min<int64_t>((rows + warps_per_block - 1) / warps_per_block, int64_t(dev->sm_count) * 16);
+  const __nv_bfloat16* g = reinterpret_cast<const __nv_bfloat16*>(a->gamma);
+  __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(a->out);
+  if (H <= 1024)
+    caat::rownorm_kernel<4><<<blocks, caat::K2_THREADS, 0, st>>>(hdst, o, g, rows, static_cast<int>(H), a->eps);
+  else if (H <= 2048)
+    caat::rownorm_kernel<8><<<blocks, caat::K2_THREADS, 0, st>>>(hdst, o, g, rows, static_cast<int>(H), a->eps);
+  else
+    caat::rownorm_kernel<16><<<blocks, caat::K2_THREADS, 0, st>>>(hdst, o, g, rows, static_cast<int>(H), a->eps);
+  if (cudaGetLastError() != cudaSuccess) return CAAT_ERR_CUDA;
+  rec.after_kernel(st);
+  return CAAT_OK;
+}
+
+caat_status validate_rowpar(const caat_rowpar_args* a, std::vector<uint8_t>& mask) {
+  if (!a) return CAAT_ERR_INVALID_ARG;
+  caat_status s = check_shapes(a->T, a->K, a->H, a->P, a->p);
+  if (s != CAAT_OK) return s;
+  if (!(a->eps >= 0.f) || !std::isfinite(a->eps) || !std::isfinite(a->private_scale)) return CAAT_ERR_INVALID_ARG;
+  s = build_mask(a->H, a->p, a->sync_idx, mask, nullptr);
+  if (s != CAAT_OK) return s;
+  if (a->T == 0) return CAAT_OK;
+  if (!a->X || !a->W || !a->residual || !a->gamma || !a->out) return CAAT_ERR_INVALID_ARG;
+  if (!aligned16(a->X) || !aligned16(a->W) || !aligned16(a->residual) || !aligned16(a->gamma) ||
+      !aligned16(a->out) || (a->h_out && !aligned16(a->h_out)))
+    return CAAT_ERR_UNSUPPORTED;
+  const size_t need = rowpar_workspace(a->T, a->K, a->H, a->P);
+  if (need > 0) {
+    if (!a->workspace || a->ws_bytes < need || (reinterpret_cast<uintptr_t>(a->workspace) & 255u))
+      return CAAT_ERR_WORKSPACE;
+  }
+  return CAAT_OK;
+}
+
+}  // namespace
+
+// =======================================================================================
+// C ABI
+// =======================================================================================
+extern "C" {
+
+const char* caat_status_string(caat_status s) {
+  switch (s) {
+    case CAAT_OK: return "CAAT_OK";
+    case CAAT_ERR_INVALID_ARG: return "CAAT_ERR_INVALID_ARG";
+    case CAAT_ERR_UNSUPPORTED: return "CAAT_ERR_UNSUPPORTED";
+    case CAAT_ERR_CUDA: return "CAAT_ERR_CUDA";
+    case CAAT_ERR_TIMEOUT: return "CAAT_ERR_TIMEOUT";
+    case CAAT_ERR_WORKSPACE: return "CAAT_ERR_WORKSPACE";
+  }
+  return "CAAT_ERR_UNKNOWN";
+}
+
+const char* caat_version(void) { return "caat-b200 0.1.0 (sm_100a)"; }
+
+caat_status caat_sync_mask(int64_t H, double p, const int32_t* sync_idx, uint8_t* mask_out, int64_t* n_sync_out) {
+  if (H <= 0 || H > CAAT_MAX_H) return CAAT_ERR_INVALID_ARG;
+  std::vector<uint8_t> mask;
+  int64_t ns = 0;
+  const caat_status s = build_mask(H, p, sync_idx, mask, &ns);
+  if (s != CAAT_OK) return s;
+  if (mask_out) std::memcpy(mask_out, mask.data(), static_cast<size_t>(H));
+  if (n_sync_out) *n_sync_out = ns;
+  return CAAT_OK;
+}
+
+size_t caat_workspace_size(int64_t T, int64_t K, int64_t H, int P, int variant) {
+  if (check_shapes(T, K, H, P, 0.0) != CAAT_OK) return SIZE_MAX;
+  if (variant == CAAT_VARIANT_ROWPAR) return rowpar_workspace(T, K, H, P);
+  if (variant == CAAT_VARIANT_ROWPAR_HOST) return host_layout(T, K, H, P).total;
+  return SIZE_MAX;
+}
+
+caat_status caat_rowpar_forward_ex(const caat_rowpar_args* a) {
+  std::vector<uint8_t> mask;
+  caat_status s = validate_rowpar(a, mask);
+  if (s != CAAT_OK) return s;
+  if (a->T == 0) return CAAT_OK;
+  DeviceInfo* dev = nullptr;
+  s = device_info(&dev);
+  if (s != CAAT_OK) return s;
+  return launch_rowpar(a, mask, dev, static_cast<unsigned int*>(a->workspace));
+}
+
+caat_status caat_rowpar_forward_host(const caat_rowpar_args* a) {
+  if (!a) return CAAT_ERR_INVALID_ARG;
+  caat_status s = check_shapes(a->T, a->K, a->H, a->P, a->p);
+  if (s != CAAT_OK) return s;
+  if (a->T == 0) return CAAT_OK;
+  if (!a->X || !a->W || !a->residual || !a->gamma || !a->out) return CAAT_ERR_INVALID_ARG;
+  const HostLayout L = host_layout(a->T, a->K, a->H, a->P);
+  if (!a->workspace || a->ws_bytes < L.total || (reinterpret_cast<uintptr_t>(a->workspace) & 255u))
+    return CAAT_ERR_WORKSPACE;
+  uint8_t* base = static_cast<uint8_t*>(a->workspace);
+  caat_rowpar_args d = *a;
+  d.X = reinterpret_cast<const caat_bf16*>(base + L.x);
+  d.W = reinterpret_cast<const caat_bf16*>(base + L.w);
+  d.residual = reinterpret_cast<const caat_bf16*>(base + L.r);
+  d.gamma = reinterpret_cast<const caat_bf16*>(base + L.g);
+  d.out = reinterpret_cast<caat_bf16*>(base + L.o);
+  d.h_out = a->h_out ? reinterpret_cast<caat_bf16*>(base + L.h) : nullptr;
+  d.workspace = base;
+  d.ws_bytes = L.x;
+  std::vector<uint8_t> mask;
+  s = validate_rowpar(&d, mask);
+  if (s != CAAT_OK) return s;
+  DeviceInfo* dev = nullptr;
+  s = device_info(&dev);
+  if (s != CAAT_OK) return s;
+  const size_t Kp = static_cast<size_t>(a->K / a->P);
+  const size_t nx = size_t(a->P) * a->T * Kp * 2, nw = size_t(a->P) * a->H * Kp * 2;
+  const size_t nr = size_t(a->P) * a->T * a->H * 2, ng = size_t(a->H) * 2;
+  cudaStream_t st = a->stream;
+  if (cudaMemcpyAsync(base + L.x, a->X, nx, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(base + L.w, a->W, nw, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(base + L.r, a->residual, nr, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(base + L.g, a->gamma, ng, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return CAAT_ERR_CUDA;
+  s = launch_rowpar(&d, mask, dev, static_cast<unsigned int*>(d.workspace));
+  if (s != CAAT_OK) return s;
+  if (cudaMemcpyAsync(a->out, base + L.o, nr, cudaMemcpyDeviceToHost, st) != cudaSuccess) return CAAT_ERR_CUDA;
+  if (a->h_out && cudaMemcpyAsync(a->h_out, base + L.h, nr, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return CAAT_ERR_CUDA;
+  return CAAT_OK;
+}
+
+caat_status caat_rowpar_forward(const caat_bf16* X, const caat_bf16* W, const caat_bf16* residual,
+                                const caat_bf16* gamma, const int32_t* sync_idx, int P, double p, caat_bf16* out,
+                                int64_t T, int64_t K, int64_t H, void* workspace, size_t ws_bytes,
+                                caat_stream_t stream) {
+  caat_rowpar_args a;
+  std::memset(&a, 0, sizeof(a));
+  a.X = X;
+  a.W = W;
+  a.residual = residual;
+  a.gamma = gamma;
+  a.sync_idx = sync_idx;
+  a.out = out;
+  a.workspace = workspace;
+  a.ws_bytes = ws_bytes;
+  a.stream = stream;
+  a.T = T;
+  a.K = K;
+  a.H = H;
+  a.p = p;
+  a.eps = 1e-5f;
+  a.private_scale = 1.0f;
+  a.P = P;
+  return caat_rowpar_forward_ex(&a);
+}
+
+caat_status caat_mlp_forward_ex(const caat_mlp_args* a) {
+  if (!a) return CAAT_ERR_INVALID_ARG;
+  return CAAT_ERR_UNSUPPORTED;
+}
+
+caat_status caat_mlp_forward(const caat_bf16* X, const caat_bf16* A, const caat_bf16* W2, const caat_bf16* residual,
+                             const caat_bf16* gamma, const int32_t* sync_idx, int P, double p, caat_bf16* out,
+                             int64_t T, int64_t H, int64_t F, void* workspace, size_t ws_bytes,
+                             caat_stream_t stream) {
+  caat_mlp_args a;
+  std::memset(&a, 0, sizeof(a));
+  a.X = X;
+  a.A = A;
+  a.W2 = W2;
+  a.residual = residual;
+  a.gamma = gamma;
+  a.sync_idx = sync_idx;
+  a.out = out;
+  a.workspace = workspace;
+  a.ws_bytes = ws_bytes;
+  a.stream = stream;
+  a.T = T;
+  a.H = H;
+  a.F = F;
+  a.p = p;
+  a.eps = 1e-5f;
+  a.private_scale = 1.0f;
+  a.P = P;
+  return caat_mlp_forward_ex(&a);
+}
+
+caat_status caat_get_device_status(caat_stream_t stream, int32_t* status_out) {
+  if (!status_out) return CAAT_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return CAAT_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, caat::g_status_word, sizeof(int)) != cudaSuccess) return CAAT_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(caat::g_status_word, &zero, sizeof(int)) != cudaSuccess) return CAAT_ERR_CUDA;
+  *status_out = v;
+  return (v & 0xFF) == 0 ? CAAT_OK : static_cast<caat_status>(v & 0xFF);
+}
+
+caat_status caat_timing_create(int capacity, caat_timing** out) {
+  if (capacity <= 0 || capacity > (1 << 20) || !out) return CAAT_ERR_INVALID_ARG;
+  caat_timing* t = new caat_timing();
+  t->capacity = capacity;
+  t->ev.resize(static_cast<size_t>(capacity) * (t->max_kernels + 1), nullptr);
+  t->nk.assign(static_cast<size_t>(capacity), 0);
+  for (auto& e : t->ev) {
+    if (cudaEventCreate(&e) != cudaSuccess) {
+      caat_timing_destroy(t);
+      return CAAT_ERR_CUDA;
+    }
+  }
+  *out = t;
+  return CAAT_OK;
+}
+
+caat_status caat_timing_destroy(caat_timing* t) {
+  if (!t) return CAAT_ERR_INVALID_ARG;
+  for (auto& e : t->ev)
+    if (e) cudaEventDestroy(e);
+  delete t;
+  return CAAT_OK;
+}
+
+caat_status caat_timing_reset(caat_timing* t) {
+  if (!t) return CAAT_ERR_INVALID_ARG;
+  t->n = 0;
+  std::fill(t->nk.begin(), t->nk.end(), 0);
+  return CAAT_OK;
+}
+
+caat_status caat_timing_read(caat_timing* t, float* ms, int max_records, int max_kernels, int* n_records,
+                             int* n_kernels) {
+  if (!t || !ms || max_records <= 0 || max_kernels <= 0) return CAAT_ERR_INVALID_ARG;
+  const int nr = std::min(t->n, max_records);
+  int nk_max = 0;
+  for (int r = 0; r < nr; ++r) {
+    const int nk = t->nk[r];
+    nk_max = std::max(nk_max, nk);
+    if (nk == 0) continue;
+    cudaEvent_t* e = &t->ev[static_cast<size_t>(r) * (t->max_kernels + 1)];
+    if (cudaEventSynchronize(e[nk]) != cudaSuccess) return CAAT_ERR_CUDA;
+    for (int k = 0; k < std::min(nk, max_kernels); ++k) {
+      float v = 0.f;
+      if (cudaEventElapsedTime(&v, e[k], e[k + 1]) != cudaSuccess) return CAAT_ERR_CUDA;
+      ms[r * max_kernels + k] = v;
+    }
+  }
+  if (n_records) *n_records = nr;
+  if (n_kernels) *n_kernels = nk_max;
+  return CAAT_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,149 @@
+"""GPU parity of the row-parallel layer (tcgen05 GEMM + partial channel-reduce epilogue +
+RMSNorm kernels, called through the C ABI) against the float64 oracle."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import caat_oracle as O
+from partial_activation_sync_caat_b200 import caat as C
+from partial_activation_sync_caat_b200 import inputs as I
+
+from gpu_util import assert_h_close, assert_out_close, ensure_built, run_rowpar, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    ensure_built()
+
+
+def _compare(d, P, p, idx=None, *, eps=1e-5, scale=1.0, what=""):
+    out, h = run_rowpar(d, P, p, idx, eps=eps, private_scale=scale)
+    ref = O.rowpar_forward(d["X"], d["W"], d["R"], d["gamma"], P, p, idx, eps=eps,
+                           private_scale=scale, return_all=True)
+    assert_h_close(h, ref["h"], what + " h")
+    return assert_out_close(out, ref["out"], what + " out")
+
+
+# ------------------------------------------------------------------ tiny sanity workload
+def test_tiny_config_full():
+    """T=256, K=H=768, P=2, p=0.5 (S = first 384), X,W ~ N(0,0.02), R ~ N(0,1), gamma=1."""
+    d = I.make_rowpar_inputs(256, 768, 768, 2, seed=0, x_std=0.02, w_std=0.02, r_std=1.0)
+    _compare(d, 2, 0.5, what="tiny")
+
+
+def test_tiny_config_zero_residual_random_gamma():
+    """Same shape with R = 0 and gamma ~ U(0.5,1.5): the output is the normalized GEMM."""
+    d = I.make_rowpar_inputs(256, 768, 768, 2, seed=1, x_std=0.02, w_std=0.02, r_std=0.0, gamma="uniform")
+    _compare(d, 2, 0.5, what="tiny R=0")
+
+
+# ------------------------------------------------------------------ p sweep, ragged multi-tile
+@pytest.mark.parametrize("p", [0.0, 0.25, 0.5, 0.75, 1.0])
+def test_p_sweep_ragged(p):
+    """T=300 (3 row blocks, ragged), H=776 (4 column blocks, 8-wide tail), K/P=200 (4 k-blocks,
+    8-wide tail), P=4."""
+    d = I.make_rowpar_inputs(300, 800, 776, 4, seed=2, x_std=1.0, w_std=0.05, r_std=1.0, gamma="uniform")
+    _compare(d, 4, p, what=f"p={p}")
+
+
+@pytest.mark.parametrize("p", [0.7, 0.703125, 0.333])
+def test_unaligned_shared_boundary(p):
+    """n_s not a multiple of the tile width (537, 540, 255 of 768): mixed column blocks."""
+    d = I.make_rowpar_inputs(200, 768, 768, 2, seed=3, x_std=1.0, w_std=0.05, r_std=1.0)
+    _compare(d, 2, p, what=f"p={p}")
+
+
+def test_random_sync_idx_small():
+    d = I.make_rowpar_inputs(260, 1024, 1024, 4, seed=4, x_std=1.0, w_std=0.05, r_std=0.5)
+    idx = I.random_sync_idx(1024, O.n_sync(1024, 0.5), seed=0)
+    _compare(d, 4, 0.5, idx, what="random S")
+
+
+def test_private_scale_sqrt_p_and_eps():
+    d = I.make_rowpar_inputs(192, 512, 512, 4, seed=5, x_std=1.0, w_std=0.05, r_std=1.0)
+    _compare(d, 4, 0.5, scale=math.sqrt(4), eps=1e-3, what="scale")
+
+
+@pytest.mark.parametrize("T", [1, 8, 64, 127, 129])
+def test_small_token_counts(T):
+    d = I.make_rowpar_inputs(T, 1024, 512, 8, seed=6, x_std=1.0, w_std=0.05, r_std=1.0)
+    _compare(d, 8, 0.5, what=f"T={T}")
+
+
+def test_single_rank():
+    d = I.make_rowpar_inputs(150, 256, 264, 1, seed=7, x_std=1.0, w_std=0.05, r_std=1.0)
+    for p in (0.0, 0.5, 1.0):
+        _compare(d, 1, p, what=f"P=1 p={p}")
+
+
+# ------------------------------------------------------------------ bit-exact bookkeeping
+def _integer_inputs(P, T, H, Kp):
+    X = torch.zeros(P, T, Kp, dtype=torch.bfloat16)
+    W = torch.zeros(P, H, Kp, dtype=torch.bfloat16)
+    a = torch.tensor([1.0 + (t % 4) for t in range(T)])
+    for m in range(P):
+        X[m, :, 3] = a
+        W[m, :, 3] = float(2 ** m)
+    return {"X": X, "W": W, "R": torch.zeros(P, T, H, dtype=torch.bfloat16),
+            "gamma": torch.ones(H, dtype=torch.bfloat16)}
+
+
+@pytest.mark.parametrize("P,p,random_idx", [(4, 0.5, False), (4, 0.3, True), (4, 0.0, False),
+                                            (4, 1.0, False), (2, 0.7, False), (3, 0.5, True)])
+def test_integer_construction_bit_exact(P, p, random_idx):
+    """partial_m[t, c] = 2^m a(t): every shared channel must read exactly (2^P - 1) a(t), every
+    private channel of rank m exactly 2^m a(t) (exact in fp32 and bf16)."""
+    T, H, Kp = 130, 520, 16
+    d = _integer_inputs(P, T, H, Kp)
+    idx = I.random_sync_idx(H, O.n_sync(H, p), seed=P) if random_idx else None
+    _, h = run_rowpar(d, P, p, idx)
+    mask, ns = C.caat_sync_mask(H, p, idx)
+    mask = mask.astype(bool)
+    np.testing.assert_array_equal(mask, O.sync_mask(H, p, idx))
+    a = np.array([1.0 + (t % 4) for t in range(T)])
+    hv = h.double().numpy()
+    for m in range(P):
+        want = np.where(mask[None, :], (2 ** P - 1) * a[:, None], (2 ** m) * a[:, None])
+        np.testing.assert_array_equal(hv[m], want)
+
+
+# ------------------------------------------------------------------ aliasing, determinism
+def test_out_aliases_residual():
+    d = I.make_rowpar_inputs(140, 512, 512, 2, seed=8, x_std=1.0, w_std=0.05, r_std=1.0)
+    ref = O.rowpar_forward(d["X"], d["W"], d["R"], d["gamma"], 2, 0.5)
+    out, _ = run_rowpar(d, 2, 0.5, out_alias_residual=True)
+    assert_out_close(out, ref, "in-place")
+
+
+def test_deterministic():
+    d = I.make_rowpar_inputs(300, 1024, 768, 4, seed=9, x_std=1.0, w_std=0.05, r_std=1.0)
+    o1, h1 = run_rowpar(d, 4, 0.5)
+    o2, h2 = run_rowpar(d, 4, 0.5)
+    assert torch.equal(o1, o2) and torch.equal(h1, h2)
+
+
+def test_empty_tokens():
+    g = to_dev(I.make_rowpar_inputs(0, 256, 256, 2, seed=0))
+    out = torch.empty_like(g["R"])
+    C.caat_rowpar_forward(g["X"], g["W"], g["R"], g["gamma"], None, 2, 0.5, out)
+    torch.cuda.synchronize()
+
+
+# ------------------------------------------------------------------ bounded waits
+def test_stall_reports_timeout_and_context_survives():
+    """The test hook makes the MMA warp withhold its accumulator signal: every consumer wait
+    must run out (bounded), the status word must read CAAT_ERR_TIMEOUT, and the next call
+    must work normally."""
+    d = I.make_rowpar_inputs(256, 512, 512, 2, seed=10, x_std=1.0, w_std=0.05, r_std=1.0)
+    g = to_dev(d)
+    out = torch.empty_like(g["R"])
+    C.caat_rowpar_forward(g["X"], g["W"], g["R"], g["gamma"], None, 2, 0.5, out,
+                          flags=C.CAAT_FLAG_TEST_STALL)
+    st = C.caat_get_device_status()
+    assert st & 0xFF == C.CAAT_ERR_TIMEOUT
+    assert C.caat_get_device_status() == 0     # cleared by the read
+    _compare(d, 2, 0.5, what="after timeout")
