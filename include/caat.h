@@ -137,6 +137,28 @@ CAAT_API caat_status caat_rowpar_forward_ex(const caat_rowpar_args* args);
 CAAT_API caat_status caat_rowpar_forward_host(const caat_rowpar_args* args);
 
 /*
+ * caat_rowpar_forward_noalloc - the same layer for callers that cannot allocate device memory
+ * at all: code running where cudaMalloc is unavailable or forbidden (a host process whose
+ * allocator is owned by someone else, an embedding that may not grow its memory footprint,
+ * a hot loop that must never enter the allocator).  No counterpart in the paper: it is a
+ * deployment convenience of this library.
+ *
+ * Arguments as caat_rowpar_forward_ex, except that args->workspace and args->ws_bytes are
+ * ignored.  The scratch the kernels need (the work-unit counter of the GEMM kernel) lives in
+ * a fixed device array inside the library, CAAT_NOALLOC_SCRATCH_BYTES bytes per GPU, held by
+ * every GPU that loads the library until the process exits.  A call whose scratch need
+ * exceeds that size returns CAAT_ERR_WORKSPACE and queues nothing.
+ *   - Calls no cudaMalloc, cudaFree or other allocating routine.
+ *   - The first call on a device looks up the array's device address (once per device, with
+ *     that device current); make that first call before any stream capture.
+ *   - Every call shares the one array and clears the part that must start at zero; calls
+ *     whose work overlaps on the GPU (other streams, other host threads) race on it and must
+ *     be serialized by the caller.
+ */
+#define CAAT_NOALLOC_SCRATCH_BYTES 1048576
+CAAT_API caat_status caat_rowpar_forward_noalloc(const caat_rowpar_args* args);
+
+/*
  * caat_mlp_forward - the MLP block per rank: column-parallel FC1 with SwiGLU (§3.1 Eq. 6),
  * then the partially synchronized FC2 (App. A.2 Eq. 22), residual add and RMSNorm (Eq. 9).
  *

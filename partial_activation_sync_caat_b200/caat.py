@@ -31,9 +31,12 @@ CAAT_FLAG_FORCE_GEMM_PATH = 0x1
 CAAT_FLAG_FORCE_DECODE_PATH = 0x2
 CAAT_FLAG_TEST_STALL = 0x100
 
+CAAT_NOALLOC_SCRATCH_BYTES = 1048576
+
 # Every symbol include/caat.h declares (checked by the ABI tests).
 EXPORTS = [
-    "caat_rowpar_forward", "caat_rowpar_forward_ex", "caat_rowpar_forward_host", "caat_mlp_forward", "caat_mlp_forward_ex",
+    "caat_rowpar_forward", "caat_rowpar_forward_ex", "caat_rowpar_forward_host",
+    "caat_rowpar_forward_noalloc", "caat_mlp_forward", "caat_mlp_forward_ex",
     "caat_workspace_size", "caat_sync_mask", "caat_get_device_status", "caat_timing_create",
     "caat_timing_destroy", "caat_timing_reset", "caat_timing_read", "caat_status_string",
     "caat_version",
@@ -89,6 +92,8 @@ def lib() -> ctypes.CDLL:
     L.caat_rowpar_forward_ex.restype = ctypes.c_int
     L.caat_rowpar_forward_host.argtypes = [ctypes.POINTER(RowparArgs)]
     L.caat_rowpar_forward_host.restype = ctypes.c_int
+    L.caat_rowpar_forward_noalloc.argtypes = [ctypes.POINTER(RowparArgs)]
+    L.caat_rowpar_forward_noalloc.restype = ctypes.c_int
     L.caat_mlp_forward.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.c_int, dbl, vp, i64, i64, i64, vp, sz, vp]
     L.caat_mlp_forward.restype = ctypes.c_int
     L.caat_mlp_forward_ex.argtypes = [ctypes.POINTER(MlpArgs)]
@@ -266,6 +271,39 @@ def caat_rowpar_forward_host(X, W, residual, gamma, sync_idx, P: int, p: float, 
     a.P = P
     a.flags = int(flags)
     _check(lib().caat_rowpar_forward_host(ctypes.byref(a)), "caat_rowpar_forward_host")
+    return out
+
+
+def caat_rowpar_forward_noalloc(X, W, residual, gamma, sync_idx, P: int, p: float, out, *, h_out=None,
+                                eps: float = 1e-5, private_scale: float = 1.0, flags: int = 0,
+                                stream=None, timing=None):
+    """The layer without any device allocation, for callers that cannot allocate device memory:
+    the library's built-in scratch array (CAAT_NOALLOC_SCRATCH_BYTES per GPU) replaces the
+    workspace.  Calls that overlap on the GPU share that array and race; serialize them."""
+    P = int(P)
+    T = int(X.shape[1])
+    K = int(X.shape[2]) * P
+    H = int(W.shape[1])
+    arr, idx_ptr = _sync_idx_host(sync_idx)
+    a = RowparArgs()
+    a.X = _bf16_dev(X, "X")
+    a.W = _bf16_dev(W, "W")
+    a.residual = _bf16_dev(residual, "residual")
+    a.gamma = _bf16_dev(gamma, "gamma")
+    a.sync_idx = idx_ptr
+    a.out = _bf16_dev(out, "out")
+    a.h_out = _bf16_dev(h_out, "h_out") if h_out is not None else None
+    a.workspace = None
+    a.ws_bytes = 0
+    a.stream = _stream_ptr(stream)
+    a.timing = timing.handle if timing is not None else None
+    a.T, a.K, a.H = T, K, H
+    a.p = float(p)
+    a.eps = float(eps)
+    a.private_scale = float(private_scale)
+    a.P = P
+    a.flags = int(flags)
+    _check(lib().caat_rowpar_forward_noalloc(ctypes.byref(a)), "caat_rowpar_forward_noalloc")
     return out
 
 

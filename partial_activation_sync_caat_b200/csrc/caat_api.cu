@@ -402,6 +402,67 @@ caat_status caat_rowpar_forward_host(const caat_rowpar_args* a) {
   return CAAT_OK;
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------------------------------
+// Entry point without any device allocation: the scratch is a fixed device array.
+// ---------------------------------------------------------------------------------------
+namespace {
+
+// Scratch of caat_rowpar_forward_noalloc (the work-unit counter of the GEMM kernel), shared
+// by every call of that entry point on a device.  In host code `g_noalloc_scratch` is only a
+// host-side stand-in for the symbol: the kernels get its device address, looked up once per
+// device with cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[CAAT_NOALLOC_SCRATCH_BYTES];
+
+void* g_noalloc_ptr[64];
+bool g_noalloc_ready[64];
+
+caat_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return CAAT_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return CAAT_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_noalloc_ready[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return CAAT_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+    g_noalloc_ready[dev] = true;
+  }
+  *out = g_noalloc_ptr[dev];
+  return CAAT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+caat_status caat_rowpar_forward_noalloc(const caat_rowpar_args* a) {
+  if (!a) return CAAT_ERR_INVALID_ARG;
+  // Per-thread host buffer for the sync mask: after the first call of a thread it is reused
+  // without growing (its capacity only increases for a larger H).
+  static thread_local std::vector<uint8_t> mask;
+  caat_rowpar_args d = *a;
+  d.workspace = nullptr;
+  d.ws_bytes = 0;
+  caat_status s = check_shapes(d.T, d.K, d.H, d.P, d.p);
+  if (s != CAAT_OK) return s;
+  if (d.T == 0) return validate_rowpar(&d, mask);
+  if (rowpar_workspace(d.T, d.K, d.H, d.P) > CAAT_NOALLOC_SCRATCH_BYTES) return CAAT_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  s = noalloc_scratch(&scratch);
+  if (s != CAAT_OK) return s;
+  d.workspace = scratch;
+  d.ws_bytes = CAAT_NOALLOC_SCRATCH_BYTES;
+  s = validate_rowpar(&d, mask);
+  if (s != CAAT_OK) return s;
+  DeviceInfo* dev = nullptr;
+  s = device_info(&dev);
+  if (s != CAAT_OK) return s;
+  // launch_rowpar zeroes the counter (cudaMemsetAsync on the stream) before the GEMM kernel.
+  return launch_rowpar(&d, mask, dev, static_cast<unsigned int*>(scratch));
+}
+
 caat_status caat_rowpar_forward(const caat_bf16* X, const caat_bf16* W, const caat_bf16* residual,
                                 const caat_bf16* gamma, const int32_t* sync_idx, int P, double p, caat_bf16* out,
                                 int64_t T, int64_t K, int64_t H, void* workspace, size_t ws_bytes,
