@@ -181,6 +181,8 @@ def run_caat(args):
     C.lib()
 
     T, K, H, P, p_def, rand = WORKLOADS[args.workload]
+    if args.tokens:
+        T = args.tokens
     p = args.p if args.p is not None else p_def
     ns = int((H * p) // 1)
     sync_idx = I.random_sync_idx(H, ns, seed=0) if rand else None
@@ -389,6 +391,7 @@ def main():
     ap.add_argument("--impl", choices=["caat", "reference"], default="caat")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="fc2-7b")
     ap.add_argument("--p", type=float, default=None)
+    ap.add_argument("--tokens", type=int, default=None, help="override T (profiling a smaller case)")
     ap.add_argument("--sweep", action="store_true", help="also time p in {0,.25,.5,.75,1}")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
