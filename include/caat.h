@@ -72,6 +72,8 @@ typedef enum caat_status {
 /* Flags of caat_rowpar_args.flags / caat_mlp_args.flags. */
 #define CAAT_FLAG_FORCE_GEMM_PATH 0x1u   /* use the tensor-core GEMM path even for small T */
 #define CAAT_FLAG_FORCE_DECODE_PATH 0x2u /* use the weight-streaming path even for large T */
+#define CAAT_FLAG_SINGLE_CTA 0x4u        /* use the single-CTA GEMM kernel (128-token tiles)
+                                            instead of the CTA-pair kernel (256-token tiles) */
 #define CAAT_FLAG_TEST_STALL 0x100u      /* test hook: the GEMM kernel's MMA warp never signals
                                             its accumulator, so every consumer wait runs out
                                             and the call reports CAAT_ERR_TIMEOUT through

@@ -16,6 +16,7 @@
 #include "caat.h"
 #include "ptx.cuh"
 #include "rowpar_gemm.cuh"
+#include "rowpar_gemm2.cuh"
 #include "rownorm.cuh"
 
 namespace {
@@ -31,6 +32,7 @@ struct DeviceInfo {
   bool init = false;
   bool supported = false;
   int sm_count = 0;
+  int max_pairs = 0;  // co-resident 2-CTA clusters of the pair GEMM kernel
 };
 
 std::mutex g_mu;
@@ -53,6 +55,26 @@ caat_status device_info(DeviceInfo** out) {
       if (cudaFuncSetAttribute(caat::rowpar_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                caat::K1_SMEM_BYTES) != cudaSuccess)
         return CAAT_ERR_CUDA;
+      if (cudaFuncSetAttribute(caat::rowpar_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               caat::K2P_SMEM_BYTES) != cudaSuccess)
+        return CAAT_ERR_CUDA;
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
+      cfg.blockDim = dim3(caat::K1_THREADS, 1, 1);
+      cfg.dynamicSmemBytes = caat::K2P_SMEM_BYTES;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int clusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&clusters, caat::rowpar_gemm_pair_kernel, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        clusters = 0;
+      }
+      d.max_pairs = clusters;
     }
     d.init = true;
   }
@@ -260,17 +282,41 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
   if (units > INT32_MAX / 2) return CAAT_ERR_UNSUPPORTED;
   prm.n_units = static_cast<int>(units);
 
+  // The CTA-pair kernel (256-token tiles) for all but the smallest token counts.
+  const bool pair = !(a->flags & CAAT_FLAG_SINGLE_CTA) && dev->max_pairs > 0 && T > caat::K1_BM;
+  if (pair) {
+    prm.n_mblk = static_cast<int>((T + 2 * caat::K2P_BM - 1) / (2 * caat::K2P_BM));
+    const int64_t pu = int64_t(prm.n_mblk) * (prm.nS + int64_t(P) * prm.nPriv);
+    prm.n_units = static_cast<int>(pu);
+  }
   CUtensorMap tmX, tmW;
   caat_status s = make_map_3d(&tmX, a->X, Kp, T, P, caat::K1_BK, caat::K1_BM);
   if (s != CAAT_OK) return s;
-  s = make_map_3d(&tmW, a->W, Kp, H, P, caat::K1_BK, caat::K1_BN);
+  s = make_map_3d(&tmW, a->W, Kp, H, P, caat::K1_BK, pair ? caat::K2P_BN / 2 : caat::K1_BN);
   if (s != CAAT_OK) return s;
 
   Recorder rec;
   rec.begin(a->timing, st);
   if (cudaMemsetAsync(counter, 0, sizeof(unsigned int), st) != cudaSuccess) return CAAT_ERR_CUDA;
-  const int grid = static_cast<int>(std::min<int64_t>(dev->sm_count, units));
-  caat::rowpar_gemm_kernel<<<grid, caat::K1_THREADS, caat::K1_SMEM_BYTES, st>>>(tmX, tmW, prm);
+  if (pair) {
+    const int pairs = static_cast<int>(std::min<int64_t>(dev->max_pairs, prm.n_units));
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * pairs, 1, 1);
+    cfg.blockDim = dim3(caat::K1_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = caat::K2P_SMEM_BYTES;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, caat::rowpar_gemm_pair_kernel, tmX, tmW, prm) != cudaSuccess) return CAAT_ERR_CUDA;
+  } else {
+    const int grid = static_cast<int>(std::min<int64_t>(dev->sm_count, units));
+    caat::rowpar_gemm_kernel<<<grid, caat::K1_THREADS, caat::K1_SMEM_BYTES, st>>>(tmX, tmW, prm);
+  }
   if (cudaGetLastError() != cudaSuccess) return CAAT_ERR_CUDA;
   rec.after_kernel(st);
 

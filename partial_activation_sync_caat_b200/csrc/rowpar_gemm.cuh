@@ -23,7 +23,8 @@
 //   warp 1      TMEM allocator and single-thread tcgen05.mma issuer (M=128, N=256, K=16),
 //               accumulating into one of two 256-column TMEM buffers (double-buffered so
 //               the epilogue of one unit overlaps the mainloop of the next).
-//   warps 2-5   epilogue: tcgen05.ld 32 lanes x 32 columns, residual add, bf16 stores.
+//   warps 2-5   epilogue: residual loads issued ahead (a whole row segment, or one chunk for
+//               up to 8 ranks), tcgen05.ld 32 lanes x 32 columns, residual add, bf16 stores.
 // Every wait is bounded (about 1 s): on expiry the device status word is set and all
 // roles leave their loops; in-flight TMA loads and MMAs are waited for before exit.
 #pragma once
@@ -90,54 +91,100 @@ __device__ __forceinline__ K1Unit k1_decode(int u, const RowparParams& prm) {
   return un;
 }
 
-// Epilogue of one accumulator pass for one rank: 32 rows (one per lane) x up to 256 cols.
-// mode 0: store every column; mode 1: only shared columns; mode 2: only private columns.
-__device__ __forceinline__ void k1_epilogue_pass(uint32_t tmem_row_base, const RowparParams& prm, int row,
-                                                 int rank, int n0, float scale, int mode) {
+// Converts 8 accumulator values (+ residual) to bf16 and stores them for one 16-byte piece.
+// want: bit e set = column e of the piece is written (mixed column blocks), 0xFF = all.
+__device__ __forceinline__ void k1_store_piece(__nv_bfloat16* dst, const uint32_t* v8, uint4 r, float scale,
+                                               uint32_t want) {
+  const uint32_t rw[4] = {r.x, r.y, r.z, r.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float a0 = __uint_as_float(v8[2 * e]) * scale + bf16lo(rw[e]);
+    const float a1 = __uint_as_float(v8[2 * e + 1]) * scale + bf16hi(rw[e]);
+    o[e] = pack_bf16x2(a0, a1);
+  }
+  if (want == 0xFFu) {
+    st_v4(dst, make_uint4(o[0], o[1], o[2], o[3]));
+  } else if (want != 0u) {
+    unsigned short* d16 = reinterpret_cast<unsigned short*>(dst);
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      if (want & (1u << e)) d16[e] = static_cast<unsigned short>((o[e >> 1] >> (16 * (e & 1))) & 0xFFFFu);
+  }
+}
+
+// Epilogue of a private unit (one rank): 32 rows (one per lane) x up to 256 columns.  All 32
+// residual pieces of the row segment are loaded up front (memory-level parallelism), then
+// the accumulator is read from TMEM 32 columns at a time.
+__device__ __forceinline__ void k1_epilogue_private(uint32_t trow, const RowparParams& prm, int row, int rank,
+                                                    int n0, bool mixed) {
   const bool row_ok = row < prm.T;
   const size_t rowoff = (static_cast<size_t>(rank) * prm.T + (row_ok ? row : 0)) * prm.H;
-  const __nv_bfloat16* Rp = prm.R + rowoff;
-  __nv_bfloat16* Op = prm.Hout + rowoff;
+  const __nv_bfloat16* Rp = prm.R + rowoff + n0;
+  __nv_bfloat16* Op = prm.Hout + rowoff + n0;
+  const int ncols = min(K1_BN, prm.H - n0);
+  uint4 rv[K1_BN / 8];
+#pragma unroll
+  for (int j = 0; j < K1_BN / 8; ++j) {
+    rv[j] = make_uint4(0, 0, 0, 0);
+    if (row_ok && 8 * j < ncols) rv[j] = ld_nc_v4(Rp + 8 * j);
+  }
+  const float scale = prm.private_scale;
+#pragma unroll
+  for (int c = 0; c < K1_BN / 32; ++c) {
+    if (32 * c >= ncols) break;  // warp-uniform
+    uint32_t v[32];
+    __syncwarp();
+    tmem_ld_32x32b_x32(trow + 32 * c, v);
+    tmem_wait_ld();
+    const uint32_t want = mixed ? ~prm.mask_bits[(n0 + 32 * c) >> 5] : 0xFFFFFFFFu;
+    if (row_ok) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (32 * c + 8 * k < ncols)
+          k1_store_piece(Op + 32 * c + 8 * k, v + 8 * k, rv[4 * c + k], scale, (want >> (8 * k)) & 0xFFu);
+    }
+  }
+}
+
+// Epilogue of a shared unit: the one accumulator (the cross-rank sum) serves every rank.  Per
+// 32-column chunk: one TMEM read, then the residual pieces of up to 8 ranks loaded together,
+// then one store per rank.
+__device__ __forceinline__ void k1_epilogue_shared(uint32_t trow, const RowparParams& prm, int row, int n0,
+                                                   bool mixed) {
+  constexpr int RG = 8;  // ranks per residual group
+  const bool row_ok = row < prm.T;
+  const size_t rstride = static_cast<size_t>(prm.T) * prm.H;
+  const size_t base = static_cast<size_t>(row_ok ? row : 0) * prm.H + n0;
   const int ncols = min(K1_BN, prm.H - n0);
 #pragma unroll 1
   for (int c = 0; c < K1_BN / 32; ++c) {
-    const int col = n0 + c * 32;
-    if (c * 32 >= ncols) break;  // warp-uniform
-    uint4 rv[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      rv[k] = make_uint4(0, 0, 0, 0);
-      if (row_ok && col + 8 * k < prm.H) rv[k] = ld_nc_v4(Rp + col + 8 * k);
-    }
+    if (32 * c >= ncols) break;  // warp-uniform
     uint32_t v[32];
     __syncwarp();
-    tmem_ld_32x32b_x32(tmem_row_base + c * 32, v);
-    tmem_wait_ld();
-    uint32_t want = 0xFFFFFFFFu;
-    if (mode != 0) {
-      const uint32_t bits = prm.mask_bits[col >> 5];
-      want = (mode == 1) ? bits : ~bits;
-    }
+    tmem_ld_32x32b_x32(trow + 32 * c, v);
+    const uint32_t want = mixed ? prm.mask_bits[(n0 + 32 * c) >> 5] : 0xFFFFFFFFu;
+#pragma unroll 1
+    for (int r0 = 0; r0 < prm.P; r0 += RG) {
+      uint4 rv[RG][4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      if (!row_ok || col + 8 * k >= prm.H) continue;
-      const uint32_t rw[4] = {rv[k].x, rv[k].y, rv[k].z, rv[k].w};
-      uint32_t o[4];
+      for (int rr = 0; rr < RG; ++rr)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float a0 = __uint_as_float(v[8 * k + 2 * e]) * scale + bf16lo(rw[e]);
-        const float a1 = __uint_as_float(v[8 * k + 2 * e + 1]) * scale + bf16hi(rw[e]);
-        o[e] = pack_bf16x2(a0, a1);
-      }
-      const uint32_t byte = (want >> (8 * k)) & 0xFFu;
-      __nv_bfloat16* dst = Op + col + 8 * k;
-      if (byte == 0xFFu) {
-        st_v4(dst, make_uint4(o[0], o[1], o[2], o[3]));
-      } else if (byte != 0u) {
-        unsigned short* d16 = reinterpret_cast<unsigned short*>(dst);
+        for (int k = 0; k < 4; ++k) {
+          rv[rr][k] = make_uint4(0, 0, 0, 0);
+          if (row_ok && r0 + rr < prm.P && 32 * c + 8 * k < ncols)
+            rv[rr][k] = ld_nc_v4(prm.R + (r0 + rr) * rstride + base + 32 * c + 8 * k);
+        }
+      if (r0 == 0) tmem_wait_ld();
+      if (row_ok) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-          if (byte & (1u << e)) d16[e] = static_cast<unsigned short>((o[e >> 1] >> (16 * (e & 1))) & 0xFFFFu);
+        for (int rr = 0; rr < RG; ++rr) {
+          if (r0 + rr >= prm.P) break;
+          __nv_bfloat16* Op = prm.Hout + (r0 + rr) * rstride + base + 32 * c;
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            if (32 * c + 8 * k < ncols) k1_store_piece(Op + 8 * k, v + 8 * k, rv[rr][k], 1.0f, (want >> (8 * k)) & 0xFFu);
+        }
       }
     }
   }
@@ -306,9 +353,9 @@ __global__ void __launch_bounds__(K1_THREADS, 1)
       const int n0 = un.n * K1_BN;
       const bool mixed = prm.ncls[un.n] == 2;
       if (un.rank < 0) {
-        for (int r = 0; r < prm.P; ++r) k1_epilogue_pass(trow, prm, row, r, n0, 1.0f, mixed ? 1 : 0);
+        k1_epilogue_shared(trow, prm, row, n0, mixed);
       } else {
-        k1_epilogue_pass(trow, prm, row, un.rank, n0, prm.private_scale, mixed ? 2 : 0);
+        k1_epilogue_private(trow, prm, row, un.rank, n0, mixed);
       }
       tc_fence_before();
       __syncwarp();

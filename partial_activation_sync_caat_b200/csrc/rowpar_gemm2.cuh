@@ -1,0 +1,230 @@
+// rowpar_gemm2.cuh - the partially synchronized row-parallel GEMM on CTA pairs.
+//
+// Same computation and work decomposition as rowpar_gemm.cuh ("Tensor-Parallelism with
+// Partially Synchronized Activations", App. A.2 Eq. 22 with the §4 residual add), but each
+// tile is 256 tokens x 256 channels computed by a pair of CTAs (a 2-CTA cluster on one TPC)
+// with tcgen05.mma.cta_group::2:
+//   * CTA c of the pair loads X rows [256 m + 128 c, +128) and W rows [256 n + 128 c, +128)
+//     (half of A and half of B) into its own shared memory; the leader CTA (c = 0) issues
+//     one M=256, N=256, K=16 MMA that reads both halves and leaves in each CTA's TMEM the
+//     128 x 256 accumulator of that CTA's tokens.  Per SM this halves the W bytes each k
+//     block costs, so a 32 KiB stage holds the same MMA work a 48 KiB stage did, and 6
+//     stages fit in shared memory.
+//   * Both CTAs' TMA loads signal the leader's full barrier (cta_group::2 form, no
+//     multicast); the leader's MMA commits arrive on both CTAs' empty / TMEM-full barriers
+//     (multicast commit); both CTAs' epilogues release the accumulator on the leader's
+//     TMEM-empty barrier.
+//   * Dynamic scheduling: the leader's producer draws a unit from the global counter and
+//     writes it into both CTAs' broadcast ring.
+// Every wait is bounded; on expiry the device status word is set, all roles leave their
+// loops, copies in flight are given time to land, and both CTAs meet at a final cluster
+// barrier before TMEM is freed.
+#pragma once
+
+#include "ptx.cuh"
+#include "rowpar_gemm.cuh"
+
+namespace caat {
+
+constexpr int K2P_BM = 128;                     // rows per CTA (pair tile: 256)
+constexpr int K2P_BN = 256;                     // channels per pair tile (per CTA B half: 128)
+constexpr int K2P_BK = 64;
+constexpr int K2P_STAGES = 6;
+constexpr int K2P_A_BYTES = K2P_BM * K2P_BK * 2;        // 16 KiB
+constexpr int K2P_B_BYTES = (K2P_BN / 2) * K2P_BK * 2;  // 16 KiB
+constexpr int K2P_STAGE_BYTES = K2P_A_BYTES + K2P_B_BYTES;
+constexpr int K2P_SMEM_BYTES = 1024 + K2P_STAGES * K2P_STAGE_BYTES + 512;
+constexpr uint64_t K2P_DRAIN_NS = 1000000;      // error path only: let copies in flight land
+
+__global__ void __launch_bounds__(K1_THREADS, 1)
+    rowpar_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                            const __grid_constant__ RowparParams prm) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + K2P_STAGES * K2P_A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + K2P_STAGES * K2P_STAGE_BYTES);
+  uint64_t* full = bars;                    // [STAGES]  used in the leader
+  uint64_t* empty = full + K2P_STAGES;      // [STAGES]  both CTAs (multicast commit)
+  uint64_t* tfull = empty + K2P_STAGES;     // [2]       both CTAs (multicast commit)
+  uint64_t* tempty = tfull + 2;             // [2]       leader: 4 local + 4 peer warps
+  uint64_t* sfull = tempty + 2;             // [SCHED]   both CTAs (leader producer arrives)
+  uint64_t* sempty = sfull + K1_SCHED;      // [SCHED]   leader: 5 local + 5 peer arrivals
+  uint64_t* mma_done = sempty + K1_SCHED;   // [1]       leader
+  int* sched_unit = reinterpret_cast<int*>(mma_done + 1);  // [SCHED] both CTAs
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sched_unit + K1_SCHED);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t cta = cluster_ctarank();   // 0 = leader, 1 = peer
+  const bool leader = cta == 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < K2P_STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 8);
+    }
+    for (int s = 0; s < K1_SCHED; ++s) {
+      mbar_init(&sfull[s], 1);
+      mbar_init(&sempty[s], 10);
+    }
+    mbar_init(mma_done, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmW);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_holder, K1_TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();  // barriers of both CTAs initialized, TMEM allocated, before any remote access
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const uint64_t tmo = prm.timeout_ns;
+  const uint32_t peer = cta ^ 1u;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producers
+    if (lane == 0) {
+      const uint64_t pol_x = policy_evict_normal();
+      const uint64_t pol_w = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true, issued = false;
+      for (int i = 0; ok; ++i) {
+        const int slot = i % K1_SCHED;
+        const uint32_t sph = (i / K1_SCHED) & 1;
+        int u;
+        if (leader) {
+          if (!mbar_wait_cluster(&sempty[slot], sph ^ 1, tmo, 21)) { ok = false; break; }
+          u = static_cast<int>(atomicAdd(prm.counter, 1u));
+          sched_unit[slot] = u;
+          st_shared_cluster_u32(mapa_shared(smem_u32(&sched_unit[slot]), peer), static_cast<uint32_t>(u));
+          mbar_arrive(&sfull[slot]);
+          mbar_arrive_cluster(mapa_shared(smem_u32(&sfull[slot]), peer));
+        } else {
+          if (!mbar_wait_cluster(&sfull[slot], sph, tmo, 22)) { ok = false; break; }
+          u = sched_unit[slot];
+          mbar_arrive_cluster(mapa_shared(smem_u32(&sempty[slot]), 0));
+        }
+        if (u >= prm.n_units) break;
+        const K1Unit un = k1_decode(u, prm);
+        const int r0 = un.rank < 0 ? 0 : un.rank;
+        const int r1 = un.rank < 0 ? prm.P : un.rank + 1;
+        const int xrow = un.m * (2 * K2P_BM) + static_cast<int>(cta) * K2P_BM;
+        const int wrow = un.n * K2P_BN + static_cast<int>(cta) * (K2P_BN / 2);
+        for (int r = r0; r < r1 && ok; ++r) {
+          for (int kb = 0; kb < prm.kblk_per_rank; ++kb) {
+            if (!mbar_wait(&empty[stage], phase ^ 1, tmo, 23)) { ok = false; break; }
+            const uint32_t fbar = mapa_shared(smem_u32(&full[stage]), 0);
+            if (leader) mbar_arrive_expect_tx(&full[stage], 2 * K2P_STAGE_BYTES);
+            tma_load_3d_pair(sA + stage * K2P_A_BYTES, &tmX, fbar, kb * K2P_BK, xrow, r, pol_x);
+            tma_load_3d_pair(sB + stage * K2P_B_BYTES, &tmW, fbar, kb * K2P_BK, wrow, r, pol_w);
+            issued = true;
+            if (++stage == K2P_STAGES) { stage = 0; phase ^= 1; }
+          }
+        }
+      }
+      if (!ok && issued) spin_ns(K2P_DRAIN_NS);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer (leader)
+    if (leader && lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(2 * K2P_BM, K2P_BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      bool ok = true;
+      for (int i = 0; ok; ++i) {
+        const int slot = i % K1_SCHED;
+        const uint32_t sph = (i / K1_SCHED) & 1;
+        if (!mbar_wait(&sfull[slot], sph, tmo, 24)) { ok = false; break; }
+        const int u = sched_unit[slot];
+        mbar_arrive(&sempty[slot]);
+        if (u >= prm.n_units) break;
+        const K1Unit un = k1_decode(u, prm);
+        const int buf = local & 1;
+        const uint32_t bph = (local >> 1) & 1;
+        if (!mbar_wait_cluster(&tempty[buf], bph ^ 1, tmo, 25)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t dt = tmem_base + static_cast<uint32_t>(buf * K2P_BN);
+        const int nkb = (un.rank < 0 ? prm.P : 1) * prm.kblk_per_rank;
+        int kb_in_rank = 0;
+        for (int j = 0; j < nkb; ++j) {
+          if (!mbar_wait(&full[stage], phase, tmo, 26)) { ok = false; break; }
+          tc_fence_after();
+          const int nk16 = (kb_in_rank == prm.kblk_per_rank - 1) ? prm.last_k16 : (K2P_BK / 16);
+          const uint32_t a_addr = smem_u32(sA + stage * K2P_A_BYTES);
+          const uint32_t b_addr = smem_u32(sB + stage * K2P_B_BYTES);
+          for (int kk = 0; kk < nk16; ++kk) {
+            umma_bf16_pair(dt, sw128_kmajor_desc(a_addr + kk * 32), sw128_kmajor_desc(b_addr + kk * 32), idesc,
+                           (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit_pair_mc(&empty[stage], 0x3);
+          if (++stage == K2P_STAGES) { stage = 0; phase ^= 1; }
+          if (++kb_in_rank == prm.kblk_per_rank) kb_in_rank = 0;
+        }
+        if (!ok) break;
+        if (!(prm.flags & K1_FLAG_TEST_STALL)) umma_commit_pair_mc(&tfull[buf], 0x3);
+        ++local;
+      }
+      umma_commit_pair(mma_done);
+      mbar_wait(mma_done, 0, tmo, 27);
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue warps
+    const int q = warp & 3;
+    const uint32_t tempty_leader[2] = {mapa_shared(smem_u32(&tempty[0]), 0), mapa_shared(smem_u32(&tempty[1]), 0)};
+    int local = 0;
+    for (int i = 0;; ++i) {
+      const int slot = i % K1_SCHED;
+      const uint32_t sph = (i / K1_SCHED) & 1;
+      int u = 0;
+      int ok = 1;
+      if (lane == 0) {
+        ok = mbar_wait_cluster(&sfull[slot], sph, tmo, 28) ? 1 : 0;
+        if (ok) {
+          u = sched_unit[slot];
+          if (leader) mbar_arrive(&sempty[slot]);
+          else mbar_arrive_cluster(mapa_shared(smem_u32(&sempty[slot]), 0));
+        }
+      }
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      u = __shfl_sync(0xFFFFFFFFu, u, 0);
+      if (!ok || u >= prm.n_units) break;
+      const K1Unit un = k1_decode(u, prm);
+      const int buf = local & 1;
+      const uint32_t bph = (local >> 1) & 1;
+      if (lane == 0) ok = mbar_wait(&tfull[buf], bph, tmo, 29) ? 1 : 0;
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t trow = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * K2P_BN);
+      const int row = un.m * (2 * K2P_BM) + static_cast<int>(cta) * K2P_BM + q * 32 + lane;
+      const int n0 = un.n * K2P_BN;
+      const bool mixed = prm.ncls[un.n] == 2;
+      if (un.rank < 0) {
+        k1_epilogue_shared(trow, prm, row, n0, mixed);
+      } else {
+        k1_epilogue_private(trow, prm, row, un.rank, n0, mixed);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty_leader[buf]);
+      ++local;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // neither CTA leaves while the other may still touch its shared memory
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem_base, K1_TMEM_COLS);
+}
+
+}  // namespace caat

@@ -20,8 +20,8 @@ def _built():
     ensure_built()
 
 
-def _compare(d, P, p, idx=None, *, eps=1e-5, scale=1.0, what=""):
-    out, h = run_rowpar(d, P, p, idx, eps=eps, private_scale=scale)
+def _compare(d, P, p, idx=None, *, eps=1e-5, scale=1.0, what="", flags=0):
+    out, h = run_rowpar(d, P, p, idx, eps=eps, private_scale=scale, flags=flags)
     ref = O.rowpar_forward(d["X"], d["W"], d["R"], d["gamma"], P, p, idx, eps=eps,
                            private_scale=scale, return_all=True)
     assert_h_close(h, ref["h"], what + " h")
@@ -80,6 +80,19 @@ def test_single_rank():
         _compare(d, 1, p, what=f"P=1 p={p}")
 
 
+@pytest.mark.parametrize("p", [0.0, 0.5, 0.7, 1.0])
+def test_single_cta_kernel(p):
+    """The single-CTA GEMM kernel (128-token tiles), forced for a shape the pair kernel would take."""
+    d = I.make_rowpar_inputs(300, 800, 776, 4, seed=12, x_std=1.0, w_std=0.05, r_std=1.0)
+    _compare(d, 4, p, flags=C.CAAT_FLAG_SINGLE_CTA, what=f"single-CTA p={p}")
+
+
+def test_single_cta_random_sync_idx():
+    d = I.make_rowpar_inputs(260, 1024, 1024, 4, seed=13, x_std=1.0, w_std=0.05, r_std=0.5)
+    idx = I.random_sync_idx(1024, O.n_sync(1024, 0.5), seed=3)
+    _compare(d, 4, 0.5, idx, flags=C.CAAT_FLAG_SINGLE_CTA, what="single-CTA random S")
+
+
 # ------------------------------------------------------------------ bit-exact bookkeeping
 def _integer_inputs(P, T, H, Kp):
     X = torch.zeros(P, T, Kp, dtype=torch.bfloat16)
@@ -134,7 +147,8 @@ def test_empty_tokens():
 
 
 # ------------------------------------------------------------------ bounded waits
-def test_stall_reports_timeout_and_context_survives():
+@pytest.mark.parametrize("flags", [0, C.CAAT_FLAG_SINGLE_CTA])
+def test_stall_reports_timeout_and_context_survives(flags):
     """The test hook makes the MMA warp withhold its accumulator signal: every consumer wait
     must run out (bounded), the status word must read CAAT_ERR_TIMEOUT, and the next call
     must work normally."""
@@ -142,7 +156,7 @@ def test_stall_reports_timeout_and_context_survives():
     g = to_dev(d)
     out = torch.empty_like(g["R"])
     C.caat_rowpar_forward(g["X"], g["W"], g["R"], g["gamma"], None, 2, 0.5, out,
-                          flags=C.CAAT_FLAG_TEST_STALL)
+                          flags=C.CAAT_FLAG_TEST_STALL | flags)
     st = C.caat_get_device_status()
     assert st & 0xFF == C.CAAT_ERR_TIMEOUT
     assert C.caat_get_device_status() == 0     # cleared by the read
