@@ -195,7 +195,7 @@ def run_caat(args):
 
     def step(tm=None):
         C.caat_rowpar_forward(d["X"], d["W"], d["R"], d["gamma"], sync_idx, P, p, out, workspace=ws,
-                              stream=stream, timing=tm)
+                              stream=stream, timing=tm, flags=args.flags)
 
     for _ in range(args.warmup):
         step()
@@ -226,6 +226,7 @@ def run_caat(args):
     per_kernel = timing.read()
     k1 = [r[0] for r in per_kernel if len(r) >= 1]
     k2 = [r[1] for r in per_kernel if len(r) >= 2]
+    n_kernels = max((len(r) for r in per_kernel), default=1)
     status = C.caat_get_device_status()
 
     # optional p sweep (same shapes, fewer steps), rank 0 only
@@ -235,13 +236,15 @@ def run_caat(args):
         for ps in (0.0, 0.25, 0.5, 0.75, 1.0):
             idx_s = I.random_sync_idx(H, int((H * ps) // 1), seed=0) if rand else None
             for _ in range(2):
-                C.caat_rowpar_forward(d["X"], d["W"], d["R"], d["gamma"], idx_s, P, ps, out, workspace=ws)
+                C.caat_rowpar_forward(d["X"], d["W"], d["R"], d["gamma"], idx_s, P, ps, out, workspace=ws,
+                                      flags=args.flags)
             torch.cuda.synchronize()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             n = max(3, args.steps // 2)
             a.record()
             for _ in range(n):
-                C.caat_rowpar_forward(d["X"], d["W"], d["R"], d["gamma"], idx_s, P, ps, out, workspace=ws)
+                C.caat_rowpar_forward(d["X"], d["W"], d["R"], d["gamma"], idx_s, P, ps, out, workspace=ws,
+                                      flags=args.flags)
             b.record()
             torch.cuda.synchronize()
             t_ms = a.elapsed_time(b) / n
@@ -288,10 +291,10 @@ def run_caat(args):
     ms_step = ms / args.steps
     value = world * flops / ms_step / 1e9  # TFLOP/s, whole job
     k1_ms = statistics.mean(k1) if k1 else float("nan")
-    k2_ms = statistics.mean(k2) if k2 else float("nan")
+    k2_ms = statistics.mean(k2) if k2 else None
     k1_tflops = flops / k1_ms / 1e9
     norm_bytes = 2.0 * P * T * H * 2
-    k2_gbs = norm_bytes / k2_ms / 1e6
+    k2_gbs = norm_bytes / k2_ms / 1e6 if k2_ms else None
     alg_bytes = 2.0 * (P * T * (K // P) + P * H * (K // P) + 2 * P * T * H + H)
     result = {
         "metric": "TFLOP/s & tokens/s of partially-synced row-parallel FC2 (7B shape), % bf16 peak",
@@ -312,20 +315,24 @@ def run_caat(args):
         "tokens_per_s": round(world * T / (ms_step / 1e3), 1),
         "pct_bf16_peak": {"measured_burst": round(100 * value / world / peaks["bf16_tflops"], 1),
                           "datasheet_2250": round(100 * value / world / 2250.0, 1)},
-        "roofline": {"kernel": "rowpar_gemm_kernel (tcgen05 GEMM + partial channel-reduce + residual)",
+        "roofline": {"kernel": "rowpar_gemm_pair_kernel (tcgen05 cta_group::2 GEMM + partial channel-reduce "
+                               "+ residual" + (")" if k2_ms else " + fused RMSNorm)"),
                      "bound": "tensor", "achieved": round(k1_tflops, 1), "peak": peaks["bf16_tflops"],
                      "peak_source": f"{peak_src} bf16 burst", "unit": "TFLOP/s",
                      "frac": round(k1_tflops / peaks["bf16_tflops"], 3),
                      "frac_vs_sustained": round(k1_tflops / peaks["bf16_tflops_sustained"], 3),
                      "traffic": None, "launch_ms": round(k1_ms, 4),
                      "algorithmic": "2*T*K*H flops per launch"},
-        "norm_kernel": {"kernel": "rownorm_kernel", "bound": "hbm", "achieved": round(k2_gbs, 1),
-                        "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(k2_gbs / peaks["hbm_gbs"], 3),
-                        "launch_ms": round(k2_ms, 4), "algorithmic": "2*P*T*H*2 bytes (read h, write out)"},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": n_kernels * args.steps,
         "device_status": status,
         "clocks": clocks,
     }
+    if k2_ms:
+        result["norm_kernel"] = {"kernel": "rownorm_kernel", "bound": "hbm", "achieved": round(k2_gbs, 1),
+                                 "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(k2_gbs / peaks["hbm_gbs"], 3),
+                                 "launch_ms": round(k2_ms, 4), "algorithmic": "2*P*T*H*2 bytes (read h, write out)"}
+    if args.flags:
+        result["config"]["flags"] = hex(args.flags)
     if sweep is not None:
         result["p_sweep"] = sweep
     if e2e is not None:
@@ -392,6 +399,7 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="fc2-7b")
     ap.add_argument("--p", type=float, default=None)
     ap.add_argument("--tokens", type=int, default=None, help="override T (profiling a smaller case)")
+    ap.add_argument("--flags", type=lambda x: int(x, 0), default=0, help="CAAT_FLAG_* bits (tuning variants)")
     ap.add_argument("--sweep", action="store_true", help="also time p in {0,.25,.5,.75,1}")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -72,6 +72,12 @@ typedef enum caat_status {
 /* Flags of caat_rowpar_args.flags / caat_mlp_args.flags. */
 #define CAAT_FLAG_FORCE_GEMM_PATH 0x1u   /* use the tensor-core GEMM path even for small T */
 #define CAAT_FLAG_FORCE_DECODE_PATH 0x2u /* use the weight-streaming path even for large T */
+#define CAAT_FLAG_FUSED_NORM 0x8u        /* run the RMSNorm inside the GEMM kernel (normalizer
+                                            warps fed by row-block completion counters) instead
+                                            of as a separate row kernel after it */
+#define CAAT_FLAG_ORDER_ROWBLOCK 0x10u   /* schedule the GEMM tiles row block by row block
+                                            (default: shared-channel tiles first, then the
+                                            private tiles rank by rank) */
 #define CAAT_FLAG_SINGLE_CTA 0x4u        /* use the single-CTA GEMM kernel (128-token tiles)
                                             instead of the CTA-pair kernel (256-token tiles) */
 #define CAAT_FLAG_TEST_STALL 0x100u      /* test hook: the GEMM kernel's MMA warp never signals
@@ -92,8 +98,10 @@ typedef enum caat_status {
  *   P, p      ranks (1..CAAT_MAX_P) and sync factor p in [0, 1]; n_s = floor(H p) in double.
  *   out       device, bf16 [P, T, H]     normalized output; may alias `residual`.
  *   T, K, H   tokens (>= 0), FFN dim (K % P == 0, (K/P) % 8 == 0), hidden (H % 8 == 0).
- *   workspace device scratch of caat_workspace_size(T, K, H, P, CAAT_VARIANT_ROWPAR) bytes,
- *             256-byte aligned; its contents need not be initialized and are clobbered.
+ *   workspace device scratch of caat_workspace_size(T, K, H, P, CAAT_VARIANT_ROWPAR) bytes
+ *             (about 32 (2 ceil(H/256)) P T bytes: row-block counters and per-row partial
+ *             sums of squares of the fused RMSNorm), 256-byte aligned; its contents need not
+ *             be initialized and are clobbered.
  * eps = 1e-5 and private_scale = 1 (use caat_rowpar_forward_ex for other values).
  * Returns CAAT_OK once the work is queued.
  */

@@ -52,10 +52,13 @@ caat_status device_info(DeviceInfo** out) {
     d.sm_count = sms;
     d.supported = (major == 10 && minor == 0);
     if (d.supported) {
-      if (cudaFuncSetAttribute(caat::rowpar_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               caat::K1_SMEM_BYTES) != cudaSuccess)
-        return CAAT_ERR_CUDA;
-      if (cudaFuncSetAttribute(caat::rowpar_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      if (cudaFuncSetAttribute(caat::rowpar_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               caat::K1_SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(caat::rowpar_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               caat::K1_SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(caat::rowpar_gemm_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               caat::K2P_SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(caat::rowpar_gemm_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                caat::K2P_SMEM_BYTES) != cudaSuccess)
         return CAAT_ERR_CUDA;
       cudaLaunchConfig_t cfg = {};
@@ -65,12 +68,12 @@ caat_status device_info(DeviceInfo** out) {
       attr[0].val.clusterDim.y = 1;
       attr[0].val.clusterDim.z = 1;
       cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
-      cfg.blockDim = dim3(caat::K1_THREADS, 1, 1);
+      cfg.blockDim = dim3(caat::K1Threads<true>::value, 1, 1);
       cfg.dynamicSmemBytes = caat::K2P_SMEM_BYTES;
       cfg.attrs = attr;
       cfg.numAttrs = 1;
       int clusters = 0;
-      if (cudaOccupancyMaxActiveClusters(&clusters, caat::rowpar_gemm_pair_kernel, &cfg) != cudaSuccess) {
+      if (cudaOccupancyMaxActiveClusters(&clusters, caat::rowpar_gemm_pair_kernel<true>, &cfg) != cudaSuccess) {
         cudaGetLastError();
         clusters = 0;
       }
@@ -172,15 +175,35 @@ caat_status build_mask(int64_t H, double p, const int32_t* sync_idx, std::vector
 
 constexpr size_t kCounterBytes = 256;
 
-size_t rowpar_workspace(int64_t T, int64_t K, int64_t H, int P) {
-  (void)T;
-  (void)K;
-  (void)H;
-  (void)P;
-  return kCounterBytes;
+size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
+
+// Workspace of the row-parallel layer: [counters (256 B) | rb_count[n_rb] | job_slots[n_rb] |
+// ss_part[P][T_pad][nslots_max] floats].  The counter region (first `zeroed` bytes) is cleared
+// on the stream before every launch; ss_part needs no clearing (every slot of every valid row
+// is written once).  Sized for the larger of the two GEMM kernels' row blocking.
+struct RowparWs {
+  size_t rb_count, job_slots, ss_part, zeroed, total;
+  int64_t T_pad, n_rb, nslots_max;
+};
+
+RowparWs rowpar_ws_layout(int64_t T, int64_t H, int P, bool fused) {
+  RowparWs L{};
+  L.T_pad = (T + 255) / 256 * 256;
+  L.n_rb = (L.T_pad / 128) * P;
+  L.nslots_max = 2 * ((H + 255) / 256);
+  L.rb_count = kCounterBytes;
+  L.job_slots = L.rb_count + size_t(L.n_rb) * 4;
+  L.zeroed = L.job_slots + size_t(L.n_rb) * 4;
+  L.ss_part = align256(L.zeroed);
+  L.total = fused ? L.ss_part + align256(size_t(P) * L.T_pad * L.nslots_max * 4) : kCounterBytes;
+  if (!fused) L.zeroed = kCounterBytes;
+  return L;
 }
 
-size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
+size_t rowpar_workspace(int64_t T, int64_t K, int64_t H, int P, bool fused = true) {
+  (void)K;
+  return rowpar_ws_layout(T, H, P, fused).total;
+}
 
 // Device staging layout of caat_rowpar_forward_host: [rowpar workspace | X | W | R | gamma |
 // out | h], each region 256-byte aligned.
@@ -251,9 +274,22 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
 
   static thread_local RowparParams prm;  // ~10 KiB: keep it off the stack
   std::memset(&prm, 0, sizeof(prm));
+  const bool fused = (a->flags & CAAT_FLAG_FUSED_NORM) != 0;
+  const RowparWs wl = rowpar_ws_layout(T, H, P, fused);
+  uint8_t* wsb = reinterpret_cast<uint8_t*>(counter);
   prm.R = reinterpret_cast<const __nv_bfloat16*>(a->residual);
   prm.Hout = hdst;
+  prm.Out = reinterpret_cast<__nv_bfloat16*>(a->out);
+  prm.gamma = reinterpret_cast<const __nv_bfloat16*>(a->gamma);
   prm.counter = counter;
+  prm.piece_claim = counter + 1;
+  prm.job_pub = counter + 2;
+  prm.rb_count = reinterpret_cast<unsigned int*>(wsb + wl.rb_count);
+  prm.job_slots = reinterpret_cast<unsigned int*>(wsb + wl.job_slots);
+  prm.ss_part = reinterpret_cast<float*>(wsb + wl.ss_part);
+  prm.fuse_norm = fused ? 1 : 0;
+  prm.order = (a->flags & CAAT_FLAG_ORDER_ROWBLOCK) ? 1 : 0;
+  prm.eps = a->eps;
   prm.T = static_cast<int>(T);
   prm.H = static_cast<int>(H);
   prm.Kp = static_cast<int>(Kp);
@@ -281,6 +317,9 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
   const int64_t units = int64_t(prm.n_mblk) * (prm.nS + int64_t(P) * prm.nPriv);
   if (units > INT32_MAX / 2) return CAAT_ERR_UNSUPPORTED;
   prm.n_units = static_cast<int>(units);
+  prm.nslots = prm.nS + prm.nPriv;
+  prm.T_pad = static_cast<int>(int64_t(prm.n_mblk) * caat::K1_BM);
+  prm.n_rb = prm.n_mblk * P;
 
   // The CTA-pair kernel (256-token tiles) for all but the smallest token counts.
   const bool pair = !(a->flags & CAAT_FLAG_SINGLE_CTA) && dev->max_pairs > 0 && T > caat::K1_BM;
@@ -288,16 +327,23 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
     prm.n_mblk = static_cast<int>((T + 2 * caat::K2P_BM - 1) / (2 * caat::K2P_BM));
     const int64_t pu = int64_t(prm.n_mblk) * (prm.nS + int64_t(P) * prm.nPriv);
     prm.n_units = static_cast<int>(pu);
+    prm.T_pad = prm.n_mblk * 2 * caat::K2P_BM;
+    prm.n_rb = 2 * prm.n_mblk * P;
   }
-  CUtensorMap tmX, tmW;
+  CUtensorMap tmX, tmW, tmR, tmH;
   caat_status s = make_map_3d(&tmX, a->X, Kp, T, P, caat::K1_BK, caat::K1_BM);
   if (s != CAAT_OK) return s;
   s = make_map_3d(&tmW, a->W, Kp, H, P, caat::K1_BK, pair ? caat::K2P_BN / 2 : caat::K1_BN);
   if (s != CAAT_OK) return s;
+  // residual in / pre-norm h out of the TMA epilogue: 32-row x 64-column boxes
+  s = make_map_3d(&tmR, a->residual, H, T, P, 64, 32);
+  if (s != CAAT_OK) return s;
+  s = make_map_3d(&tmH, hdst, H, T, P, 64, 32);
+  if (s != CAAT_OK) return s;
 
   Recorder rec;
   rec.begin(a->timing, st);
-  if (cudaMemsetAsync(counter, 0, sizeof(unsigned int), st) != cudaSuccess) return CAAT_ERR_CUDA;
+  if (cudaMemsetAsync(counter, 0, wl.zeroed, st) != cudaSuccess) return CAAT_ERR_CUDA;
   if (pair) {
     const int pairs = static_cast<int>(std::min<int64_t>(dev->max_pairs, prm.n_units));
     cudaLaunchConfig_t cfg = {};
@@ -307,30 +353,34 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.gridDim = dim3(2 * pairs, 1, 1);
-    cfg.blockDim = dim3(caat::K1_THREADS, 1, 1);
+    cfg.blockDim = dim3(fused ? caat::K1Threads<true>::value : caat::K1Threads<false>::value, 1, 1);
     cfg.dynamicSmemBytes = caat::K2P_SMEM_BYTES;
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, caat::rowpar_gemm_pair_kernel, tmX, tmW, prm) != cudaSuccess) return CAAT_ERR_CUDA;
+    const cudaError_t e =
+        fused ? cudaLaunchKernelEx(&cfg, caat::rowpar_gemm_pair_kernel<true>, tmX, tmW, tmR, tmH, prm)
+              : cudaLaunchKernelEx(&cfg, caat::rowpar_gemm_pair_kernel<false>, tmX, tmW, tmR, tmH, prm);
+    if (e != cudaSuccess) return CAAT_ERR_CUDA;
   } else {
     const int grid = static_cast<int>(std::min<int64_t>(dev->sm_count, units));
-    caat::rowpar_gemm_kernel<<<grid, caat::K1_THREADS, caat::K1_SMEM_BYTES, st>>>(tmX, tmW, prm);
+    if (fused)
+      caat::rowpar_gemm_kernel<true><<<grid, caat::K1Threads<true>::value, caat::K1_SMEM_BYTES, st>>>(tmX, tmW, tmR,
+                                                                                                     tmH, prm);
+    else
+      caat::rowpar_gemm_kernel<false><<<grid, caat::K1Threads<false>::value, caat::K1_SMEM_BYTES, st>>>(tmX, tmW, tmR,
+                                                                                                       tmH, prm);
   }
   if (cudaGetLastError() != cudaSuccess) return CAAT_ERR_CUDA;
   rec.after_kernel(st);
+  if (fused) return CAAT_OK;
 
   const int64_t rows = int64_t(P) * T;
   const int64_t warps_per_block = caat::K2_THREADS / 32;
-  const int64_t blocks = std::min<int64_t>((rows + warps_per_block - 1) / warps_per_block, int64_t(dev->sm_count) * 16);
+  const int64_t blocks = std::min<int64_t>((rows + warps_per_block - 1) / warps_per_block, int64_t(dev->sm_count) * 4);
   const __nv_bfloat16* g = reinterpret_cast<const __nv_bfloat16*>(a->gamma);
   __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(a->out);
-  if (H <= 1024)
-    caat::rownorm_kernel<4><<<blocks, caat::K2_THREADS, 0, st>>>(hdst, o, g, rows, static_cast<int>(H), a->eps);
-  else if (H <= 2048)
-    caat::rownorm_kernel<8><<<blocks, caat::K2_THREADS, 0, st>>>(hdst, o, g, rows, static_cast<int>(H), a->eps);
-  else
-    caat::rownorm_kernel<16><<<blocks, caat::K2_THREADS, 0, st>>>(hdst, o, g, rows, static_cast<int>(H), a->eps);
+  caat::rownorm_kernel<<<blocks, caat::K2_THREADS, 0, st>>>(hdst, o, g, rows, static_cast<int>(H), a->eps);
   if (cudaGetLastError() != cudaSuccess) return CAAT_ERR_CUDA;
   rec.after_kernel(st);
   return CAAT_OK;
@@ -348,7 +398,7 @@ caat_status validate_rowpar(const caat_rowpar_args* a, std::vector<uint8_t>& mas
   if (!aligned16(a->X) || !aligned16(a->W) || !aligned16(a->residual) || !aligned16(a->gamma) ||
       !aligned16(a->out) || (a->h_out && !aligned16(a->h_out)))
     return CAAT_ERR_UNSUPPORTED;
-  const size_t need = rowpar_workspace(a->T, a->K, a->H, a->P);
+  const size_t need = rowpar_workspace(a->T, a->K, a->H, a->P, (a->flags & CAAT_FLAG_FUSED_NORM) != 0);
   if (need > 0) {
     if (!a->workspace || a->ws_bytes < need || (reinterpret_cast<uintptr_t>(a->workspace) & 255u))
       return CAAT_ERR_WORKSPACE;
@@ -494,7 +544,13 @@ caat_status caat_rowpar_forward_noalloc(const caat_rowpar_args* a) {
   caat_status s = check_shapes(d.T, d.K, d.H, d.P, d.p);
   if (s != CAAT_OK) return s;
   if (d.T == 0) return validate_rowpar(&d, mask);
-  if (rowpar_workspace(d.T, d.K, d.H, d.P) > CAAT_NOALLOC_SCRATCH_BYTES) return CAAT_ERR_WORKSPACE;
+  // The fused RMSNorm needs scratch that grows with T; when it does not fit the built-in
+  // array, the norm runs as the separate row kernel, which needs only the unit counter.
+  if ((d.flags & CAAT_FLAG_FUSED_NORM) &&
+      rowpar_workspace(d.T, d.K, d.H, d.P, true) > CAAT_NOALLOC_SCRATCH_BYTES)
+    d.flags &= ~CAAT_FLAG_FUSED_NORM;
+  if (rowpar_workspace(d.T, d.K, d.H, d.P, (d.flags & CAAT_FLAG_FUSED_NORM) != 0) > CAAT_NOALLOC_SCRATCH_BYTES)
+    return CAAT_ERR_WORKSPACE;
   void* scratch = nullptr;
   s = noalloc_scratch(&scratch);
   if (s != CAAT_OK) return s;

@@ -16,13 +16,14 @@
 //     TMEM-empty barrier.
 //   * Dynamic scheduling: the leader's producer draws a unit from the global counter and
 //     writes it into both CTAs' broadcast ring.
-// Every wait is bounded; on expiry the device status word is set, all roles leave their
+// The RMSNorm is fused (rowpar_common.cuh): warps 6-9 of each CTA normalize completed row
+// blocks.  Every wait is bounded; on expiry the device status word is set, all roles leave their
 // loops, copies in flight are given time to land, and both CTAs meet at a final cluster
 // barrier before TMEM is freed.
 #pragma once
 
 #include "ptx.cuh"
-#include "rowpar_gemm.cuh"
+#include "rowpar_common.cuh"
 
 namespace caat {
 
@@ -33,17 +34,20 @@ constexpr int K2P_STAGES = 6;
 constexpr int K2P_A_BYTES = K2P_BM * K2P_BK * 2;        // 16 KiB
 constexpr int K2P_B_BYTES = (K2P_BN / 2) * K2P_BK * 2;  // 16 KiB
 constexpr int K2P_STAGE_BYTES = K2P_A_BYTES + K2P_B_BYTES;
-constexpr int K2P_SMEM_BYTES = 1024 + K2P_STAGES * K2P_STAGE_BYTES + 512;
+constexpr int K2P_SMEM_BYTES = 1024 + K2P_STAGES * K2P_STAGE_BYTES + K1_EPI_BYTES + 512;
 constexpr uint64_t K2P_DRAIN_NS = 1000000;      // error path only: let copies in flight land
 
-__global__ void __launch_bounds__(K1_THREADS, 1)
+template <bool kFused>
+__global__ void __launch_bounds__(K1Threads<kFused>::value, 1)
     rowpar_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                            const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmH,
                             const __grid_constant__ RowparParams prm) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sA = smem;
   uint8_t* sB = smem + K2P_STAGES * K2P_A_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + K2P_STAGES * K2P_STAGE_BYTES);
+  uint8_t* sEpi = smem + K2P_STAGES * K2P_STAGE_BYTES;  // [4 warps][K1_EPI_NBUF] boxes
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + K1_EPI_BYTES);
   uint64_t* full = bars;                    // [STAGES]  used in the leader
   uint64_t* empty = full + K2P_STAGES;      // [STAGES]  both CTAs (multicast commit)
   uint64_t* tfull = empty + K2P_STAGES;     // [2]       both CTAs (multicast commit)
@@ -51,7 +55,9 @@ __global__ void __launch_bounds__(K1_THREADS, 1)
   uint64_t* sfull = tempty + 2;             // [SCHED]   both CTAs (leader producer arrives)
   uint64_t* sempty = sfull + K1_SCHED;      // [SCHED]   leader: 5 local + 5 peer arrivals
   uint64_t* mma_done = sempty + K1_SCHED;   // [1]       leader
-  int* sched_unit = reinterpret_cast<int*>(mma_done + 1);  // [SCHED] both CTAs
+  uint64_t* sig = mma_done + 1;                   // [4] epilogue warps meet per tile
+  uint64_t* rbar = sig + 4;                        // [4 warps][K1_EPI_NBUF]
+  int* sched_unit = reinterpret_cast<int*>(rbar + 4 * K1_EPI_NBUF);  // [SCHED] both CTAs
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sched_unit + K1_SCHED);
 
   const int warp = threadIdx.x >> 5;
@@ -66,16 +72,20 @@ __global__ void __launch_bounds__(K1_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 8);
+      mbar_init(&tempty[b], 2 * K1Threads<kFused>::epi_warps);
     }
     for (int s = 0; s < K1_SCHED; ++s) {
       mbar_init(&sfull[s], 1);
-      mbar_init(&sempty[s], 10);
+      mbar_init(&sempty[s], 2 * (1 + K1Threads<kFused>::epi_warps));
     }
     mbar_init(mma_done, 1);
+    for (int b = 0; b < 4; ++b) mbar_init(&sig[b], K1Threads<kFused>::epi_warps);
+    for (int b = 0; b < 4 * K1_EPI_NBUF; ++b) mbar_init(&rbar[b], 1);
     fence_mbar_init();
     tma_prefetch_desc(&tmX);
     tma_prefetch_desc(&tmW);
+    tma_prefetch_desc(&tmR);
+    tma_prefetch_desc(&tmH);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_holder, K1_TMEM_COLS);
@@ -176,9 +186,16 @@ __global__ void __launch_bounds__(K1_THREADS, 1)
       umma_commit_pair(mma_done);
       mbar_wait(mma_done, 0, tmo, 27);
     }
+  } else if (kFused && warp >= K1_NORM_WARP0) {
+    // ---------------------------------------------------------------- normalizer warps
+    if constexpr (kFused) k1_normalizer(prm, lane);
   } else {
     // ---------------------------------------------------------------- epilogue warps
     const int q = warp & 3;
+    uint8_t* my_bufs = sEpi + (warp - 2) * K1_EPI_NBUF * K1_EPI_BOX_BYTES;
+    uint64_t* my_rbar = rbar + (warp - 2) * K1_EPI_NBUF;
+    uint32_t rphase = 0;
+    const uint64_t pol_r = policy_evict_first();
     const uint32_t tempty_leader[2] = {mapa_shared(smem_u32(&tempty[0]), 0), mapa_shared(smem_u32(&tempty[1]), 0)};
     int local = 0;
     for (int i = 0;; ++i) {
@@ -208,14 +225,19 @@ __global__ void __launch_bounds__(K1_THREADS, 1)
       const int row = un.m * (2 * K2P_BM) + static_cast<int>(cta) * K2P_BM + q * 32 + lane;
       const int n0 = un.n * K2P_BN;
       const bool mixed = prm.ncls[un.n] == 2;
-      if (un.rank < 0) {
-        k1_epilogue_shared(trow, prm, row, n0, mixed);
+      if (!kFused && !mixed) {
+        const int row0 = un.m * (2 * K2P_BM) + static_cast<int>(cta) * K2P_BM + q * 32;
+        if (!k1_epilogue_tma(trow, prm, &tmR, &tmH, row0, n0, un.rank, my_bufs, my_rbar, rphase, lane, pol_r))
+          break;
+      } else if (un.rank < 0) {
+        k1_epilogue_shared(trow, prm, row, n0, un.slot, mixed, 0, 8);
       } else {
-        k1_epilogue_private(trow, prm, row, un.rank, n0, mixed);
+        k1_epilogue_private(trow, prm, row, un.rank, n0, un.slot, mixed, 0, 2);
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty_leader[buf]);
+      k1_signal_tile(prm, sig, local, 2 * un.m + static_cast<int>(cta), un.rank);
       ++local;
     }
   }

@@ -93,6 +93,24 @@ def test_single_cta_random_sync_idx():
     _compare(d, 4, 0.5, idx, flags=C.CAAT_FLAG_SINGLE_CTA, what="single-CTA random S")
 
 
+@pytest.mark.parametrize("flags", [C.CAAT_FLAG_FUSED_NORM, C.CAAT_FLAG_ORDER_ROWBLOCK,
+                                   C.CAAT_FLAG_FUSED_NORM | C.CAAT_FLAG_SINGLE_CTA,
+                                   C.CAAT_FLAG_ORDER_ROWBLOCK | C.CAAT_FLAG_SINGLE_CTA])
+@pytest.mark.parametrize("p", [0.5, 0.7])
+def test_norm_and_order_variants(flags, p):
+    """The fused RMSNorm and the row-block-major tile order give the same result."""
+    d = I.make_rowpar_inputs(520, 1024, 1032, 4, seed=14, x_std=1.0, w_std=0.05, r_std=1.0, gamma="uniform")
+    _compare(d, 4, p, flags=flags, what=f"flags={flags:#x} p={p}")
+
+
+def test_without_h_out_normalizes_in_place():
+    d = I.make_rowpar_inputs(300, 800, 776, 4, seed=15, x_std=1.0, w_std=0.05, r_std=1.0, gamma="uniform")
+    ref = O.rowpar_forward(d["X"], d["W"], d["R"], d["gamma"], 4, 0.5)
+    for flags in (0, C.CAAT_FLAG_SINGLE_CTA, C.CAAT_FLAG_FUSED_NORM):
+        out, _ = run_rowpar(d, 4, 0.5, h_out=False, flags=flags)
+        assert_out_close(out, ref, f"no h_out flags={flags:#x}")
+
+
 # ------------------------------------------------------------------ bit-exact bookkeeping
 def _integer_inputs(P, T, H, Kp):
     X = torch.zeros(P, T, Kp, dtype=torch.bfloat16)
