@@ -86,6 +86,16 @@ caat_status device_info(DeviceInfo** out) {
   return CAAT_OK;
 }
 
+// Row blocks per group of the grouped tile order (tuning; CAAT_GROUP_M overrides).
+int group_m_setting() {
+  static int v = [] {
+    const char* e = std::getenv("CAAT_GROUP_M");
+    const int g = (e && *e) ? std::atoi(e) : 0;
+    return g > 0 ? g : 8;
+  }();
+  return v;
+}
+
 uint64_t timeout_ns() {
   static uint64_t v = [] {
     const char* e = std::getenv("CAAT_TIMEOUT_MS");
@@ -288,7 +298,10 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
   prm.job_slots = reinterpret_cast<unsigned int*>(wsb + wl.job_slots);
   prm.ss_part = reinterpret_cast<float*>(wsb + wl.ss_part);
   prm.fuse_norm = fused ? 1 : 0;
-  prm.order = (a->flags & CAAT_FLAG_ORDER_ROWBLOCK) ? 1 : 0;
+  // Tile order: the fused norm wants row blocks to complete throughout the kernel (grouped
+  // order); otherwise shared tiles first, then private tiles rank by rank.
+  prm.order = (a->flags & CAAT_FLAG_ORDER_ROWBLOCK) ? 1 : (fused ? 2 : 0);
+  prm.group_m = group_m_setting();
   prm.eps = a->eps;
   prm.T = static_cast<int>(T);
   prm.H = static_cast<int>(H);

@@ -64,7 +64,9 @@ struct RowparParams {
   int n_units;
   int fuse_norm;               // 1: normalizer warps produce `Out`; 0: h only
   int order;                   // unit order: 0 shared units first, then private rank-major;
-                               // 1 row-block-major (each row block's units together)
+                               // 1 row-block-major (each row block's units together);
+                               // 2 grouped: order 0 within groups of group_m row blocks
+  int group_m;                 // row blocks per group (order 2)
   int n_rb;                    // (128-row block, rank) pairs = n_m128 * P
   int T_pad;                   // n_m128 * 128
   int nslots;                  // nS + nPriv partial slots per row
@@ -85,6 +87,35 @@ struct K1Unit {
 
 __device__ __forceinline__ K1Unit k1_decode(int u, const RowparParams& prm) {
   K1Unit un;
+  if (prm.order == 2) {
+    // Grouped: for each group of group_m row blocks, its shared units (row block major),
+    // then its private units rank by rank.  Row blocks of a group complete together, while
+    // the next group's tiles are being computed.
+    const int G = prm.group_m;
+    const int per_m = prm.nS + prm.P * prm.nPriv;
+    const int full_groups = prm.n_mblk / G;
+    int g = u / (G * per_m);
+    if (g > full_groups) g = full_groups;
+    const int gm = g < full_groups ? G : prm.n_mblk - full_groups * G;
+    const int v = u - g * G * per_m;
+    if (v < prm.nS * gm) {
+      const int mi = v / prm.nS;
+      un.m = g * G + mi;
+      un.slot = v - mi * prm.nS;
+      un.n = prm.slist[un.slot];
+      un.rank = -1;
+    } else {
+      const int w = v - prm.nS * gm;
+      un.rank = w / (gm * prm.nPriv);
+      const int rem = w - un.rank * gm * prm.nPriv;
+      const int mi = rem / prm.nPriv;
+      un.m = g * G + mi;
+      const int pi = rem - mi * prm.nPriv;
+      un.n = prm.plist[pi];
+      un.slot = prm.nS + pi;
+    }
+    return un;
+  }
   if (prm.order == 1) {
     // Row-block-major: the nS shared units of row block m, then its private units rank by
     // rank, then row block m + 1.  A row block's h is complete soon after it is written, so
@@ -295,32 +326,32 @@ __device__ __forceinline__ void k1_epilogue_shared(uint32_t trow, const RowparPa
 // zero-filled on load and clipped on store by the tensor maps.  Items are pipelined over
 // K1_EPI_NBUF buffers.  Returns false if a wait ran out.
 __device__ __forceinline__ bool k1_epilogue_tma(uint32_t trow, const RowparParams& prm, const void* tmR,
-                                                const void* tmH, int row0, int n0, int rank, uint8_t* bufs,
+                                                const void* tmH, int row0, int n0, int rank, int slot, uint8_t* bufs,
                                                 uint64_t* rbar, uint32_t& phase, int lane, uint64_t pol_r) {
   const int nch = min(4, (prm.H - n0 + 63) / 64);
   const int nr = rank < 0 ? prm.P : 1;
-  const int n_items = nch * nr;
+  const int n_items = nch * nr;  // rank-major: item i = (rank i / nch, chunk i % nch)
   const float scale = rank < 0 ? 1.0f : prm.private_scale;
+  const int row = row0 + lane;
   const int npre = min(K1_EPI_NBUF, n_items);
   for (int i = 0; i < npre; ++i) {
-    const int c = i / nr, r = rank < 0 ? i - c * nr : rank;
+    const int ri = i / nch, c = i - ri * nch;
+    const int r = rank < 0 ? ri : rank;
     if (lane == 0) {
       mbar_arrive_expect_tx(&rbar[i], K1_EPI_BOX_BYTES);
       tma_load_3d(bufs + i * K1_EPI_BOX_BYTES, tmR, &rbar[i], n0 + 64 * c, row0, r, pol_r);
     }
   }
-  uint32_t v[64];
-  int cur_c = -1;
+  float ss = 0.f;
   for (int i = 0; i < n_items; ++i) {
-    const int c = i / nr, r = rank < 0 ? i - c * nr : rank;
+    const int ri = i / nch, c = i - ri * nch;
+    const int r = rank < 0 ? ri : rank;
     const int b = i % K1_EPI_NBUF;
-    if (c != cur_c) {
-      __syncwarp();
-      tmem_ld_32x32b_x32(trow + 64 * c, *reinterpret_cast<uint32_t(*)[32]>(v));
-      tmem_ld_32x32b_x32(trow + 64 * c + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
-      tmem_wait_ld();
-      cur_c = c;
-    }
+    uint32_t v[64];
+    __syncwarp();
+    tmem_ld_32x32b_x32(trow + 64 * c, *reinterpret_cast<uint32_t(*)[32]>(v));
+    tmem_ld_32x32b_x32(trow + 64 * c + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+    tmem_wait_ld();
     const bool ok = mbar_wait(&rbar[b], (phase >> b) & 1u, prm.timeout_ns, 32);
     phase ^= 1u << b;
     if (!__all_sync(0xFFFFFFFFu, ok)) return false;
@@ -332,9 +363,15 @@ __device__ __forceinline__ bool k1_epilogue_tma(uint32_t trow, const RowparParam
       const uint32_t rw[4] = {rr.x, rr.y, rr.z, rr.w};
       uint32_t o[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
+      for (int e = 0; e < 4; ++e) {
         o[e] = pack_bf16x2(__uint_as_float(v[8 * j + 2 * e]) * scale + bf16lo(rw[e]),
                            __uint_as_float(v[8 * j + 2 * e + 1]) * scale + bf16hi(rw[e]));
+        if (prm.fuse_norm && n0 + 64 * c + 8 * j < prm.H) {
+          const float lo = bf16lo(o[e]), hi = bf16hi(o[e]);
+          ss = fmaf(lo, lo, ss);
+          ss = fmaf(hi, hi, ss);
+        }
+      }
       *ptr = make_uint4(o[0], o[1], o[2], o[3]);
     }
     fence_proxy_async_smem();
@@ -343,18 +380,32 @@ __device__ __forceinline__ bool k1_epilogue_tma(uint32_t trow, const RowparParam
       tma_store_3d(tmH, bufs + b * K1_EPI_BOX_BYTES, n0 + 64 * c, row0, r);
       bulk_commit_group();
     }
+    if (prm.fuse_norm && c == nch - 1) {  // this rank's row segment is complete
+      if (row < prm.T) k1_put_partial(prm, r, row, slot, ss);
+      ss = 0.f;
+    }
     const int nx = i + K1_EPI_NBUF;
     if (nx < n_items) {
       if (lane == 0) {
         bulk_wait_group_read0();  // the store that read buffer b is done with it
-        const int c2 = nx / nr, r2 = rank < 0 ? nx - c2 * nr : rank;
+        const int r2i = nx / nch, c2 = nx - r2i * nch;
+        const int r2 = rank < 0 ? r2i : rank;
         mbar_arrive_expect_tx(&rbar[b], K1_EPI_BOX_BYTES);
         tma_load_3d(bufs + b * K1_EPI_BOX_BYTES, tmR, &rbar[b], n0 + 64 * c2, row0, r2, pol_r);
       }
       __syncwarp();
     }
   }
-  if (lane == 0) bulk_wait_group_read0();
+  if (lane == 0) {
+    if (prm.fuse_norm) {
+      // The normalizers of other CTAs read this tile's h: complete the stores and order
+      // them (async proxy) before the generic-proxy signal that follows.
+      bulk_wait_group0();
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+    } else {
+      bulk_wait_group_read0();
+    }
+  }
   __syncwarp();
   return true;
 }

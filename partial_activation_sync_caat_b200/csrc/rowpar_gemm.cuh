@@ -221,9 +221,10 @@ __global__ void __launch_bounds__(K1Threads<kFused>::value, 1)
       const int row = un.m * K1_BM + q * 32 + lane;
       const int n0 = un.n * K1_BN;
       const bool mixed = prm.ncls[un.n] == 2;
-      if (!kFused && !mixed) {
+      if (!mixed) {
         const int row0 = un.m * K1_BM + q * 32;
-        if (!k1_epilogue_tma(trow, prm, &tmR, &tmH, row0, n0, un.rank, my_bufs, my_rbar, rphase, lane, pol_r))
+        if (!k1_epilogue_tma(trow, prm, &tmR, &tmH, row0, n0, un.rank, un.slot, my_bufs, my_rbar, rphase, lane,
+                             pol_r))
           break;
       } else if (un.rank < 0) {
         k1_epilogue_shared(trow, prm, row, n0, un.slot, mixed, 0, 8);

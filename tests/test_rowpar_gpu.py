@@ -103,10 +103,18 @@ def test_norm_and_order_variants(flags, p):
     _compare(d, 4, p, flags=flags, what=f"flags={flags:#x} p={p}")
 
 
+@pytest.mark.parametrize("flags", [C.CAAT_FLAG_FUSED_NORM, C.CAAT_FLAG_FUSED_NORM | C.CAAT_FLAG_SINGLE_CTA])
+def test_fused_norm_several_row_block_groups(flags):
+    """T = 2304: more row blocks than one group of the grouped tile order (fused norm)."""
+    d = I.make_rowpar_inputs(2304, 512, 1032, 4, seed=16, x_std=1.0, w_std=0.05, r_std=1.0, gamma="uniform")
+    _compare(d, 4, 0.5, flags=flags, what=f"fused groups flags={flags:#x}")
+
+
 def test_without_h_out_normalizes_in_place():
     d = I.make_rowpar_inputs(300, 800, 776, 4, seed=15, x_std=1.0, w_std=0.05, r_std=1.0, gamma="uniform")
     ref = O.rowpar_forward(d["X"], d["W"], d["R"], d["gamma"], 4, 0.5)
-    for flags in (0, C.CAAT_FLAG_SINGLE_CTA, C.CAAT_FLAG_FUSED_NORM):
+    for flags in (0, C.CAAT_FLAG_SINGLE_CTA, C.CAAT_FLAG_FUSED_NORM,
+                  C.CAAT_FLAG_FUSED_NORM | C.CAAT_FLAG_SINGLE_CTA):
         out, _ = run_rowpar(d, 4, 0.5, h_out=False, flags=flags)
         assert_out_close(out, ref, f"no h_out flags={flags:#x}")
 
