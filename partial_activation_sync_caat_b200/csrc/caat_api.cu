@@ -17,6 +17,7 @@
 #include "ptx.cuh"
 #include "rowpar_gemm.cuh"
 #include "rowpar_gemm2.cuh"
+#include "fc1_swiglu.cuh"
 #include "rownorm.cuh"
 
 namespace {
@@ -59,7 +60,9 @@ caat_status device_info(DeviceInfo** out) {
           cudaFuncSetAttribute(caat::rowpar_gemm_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                caat::K2P_SMEM_BYTES) != cudaSuccess ||
           cudaFuncSetAttribute(caat::rowpar_gemm_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               caat::K2P_SMEM_BYTES) != cudaSuccess)
+                               caat::K2P_SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(caat::fc1_swiglu_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               caat::K3_SMEM_BYTES) != cudaSuccess)
         return CAAT_ERR_CUDA;
       cudaLaunchConfig_t cfg = {};
       cudaLaunchAttribute attr[1];
@@ -137,6 +140,21 @@ caat_status make_map_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_
   const cuuint32_t box[3] = {b0, b1, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? CAAT_OK : CAAT_ERR_CUDA;
+}
+
+// 4-D bf16 tensor [d3][d2][d1][d0] (d0 contiguous), box {b0, b1, 1, 1}, 128-byte swizzle.
+caat_status make_map_4d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t d3,
+                        uint32_t b0, uint32_t b1) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return CAAT_ERR_CUDA;
+  const cuuint64_t dims[4] = {d0, d1, d2, d3};
+  const cuuint64_t strides[3] = {d0 * 2, d0 * d1 * 2, d0 * d1 * d2 * 2};
+  const cuuint32_t box[4] = {b0, b1, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? CAAT_OK : CAAT_ERR_CUDA;
@@ -235,6 +253,19 @@ HostLayout host_layout(int64_t T, int64_t K, int64_t H, int P) {
   return L;
 }
 
+// Workspace of the MLP block: [FC1 unit counter (256 B) | row-parallel workspace | Y [P,T,F/P]].
+struct MlpWs {
+  size_t rowpar, y, total;
+};
+
+MlpWs mlp_ws_layout(int64_t T, int64_t H, int64_t F, int P, bool fused) {
+  MlpWs L{};
+  L.rowpar = kCounterBytes;
+  L.y = L.rowpar + align256(rowpar_workspace(T, F, H, P, fused));
+  L.total = L.y + align256(size_t(P) * T * (F / P) * 2);
+  return L;
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------------------------------
@@ -276,7 +307,7 @@ struct Recorder {
 // The row-parallel layer: GEMM + partial channel-reduce + residual (K1), RMSNorm (K2)
 // ---------------------------------------------------------------------------------------
 caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>& mask, const DeviceInfo* dev,
-                          unsigned int* counter) {
+                          unsigned int* counter, Recorder* outer = nullptr) {
   const int P = a->P;
   const int64_t T = a->T, H = a->H, Kp = a->K / P;
   cudaStream_t st = a->stream;
@@ -354,8 +385,9 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
   s = make_map_3d(&tmH, hdst, H, T, P, 64, 32);
   if (s != CAAT_OK) return s;
 
-  Recorder rec;
-  rec.begin(a->timing, st);
+  Recorder own;
+  Recorder& rec = outer ? *outer : own;
+  if (!outer) rec.begin(a->timing, st);
   if (cudaMemsetAsync(counter, 0, wl.zeroed, st) != cudaSuccess) return CAAT_ERR_CUDA;
   if (pair) {
     const int pairs = static_cast<int>(std::min<int64_t>(dev->max_pairs, prm.n_units));
@@ -455,6 +487,7 @@ size_t caat_workspace_size(int64_t T, int64_t K, int64_t H, int P, int variant) 
   if (check_shapes(T, K, H, P, 0.0) != CAAT_OK) return SIZE_MAX;
   if (variant == CAAT_VARIANT_ROWPAR) return rowpar_workspace(T, K, H, P);
   if (variant == CAAT_VARIANT_ROWPAR_HOST) return host_layout(T, K, H, P).total;
+  if (variant == CAAT_VARIANT_MLP) return mlp_ws_layout(T, H, K, P, true).total;
   return SIZE_MAX;
 }
 
@@ -605,7 +638,100 @@ caat_status caat_rowpar_forward(const caat_bf16* X, const caat_bf16* W, const ca
 
 caat_status caat_mlp_forward_ex(const caat_mlp_args* a) {
   if (!a) return CAAT_ERR_INVALID_ARG;
-  return CAAT_ERR_UNSUPPORTED;
+  caat_status s = check_shapes(a->T, a->F, a->H, a->P, a->p);
+  if (s != CAAT_OK) return s;
+  if (!(a->eps >= 0.f) || !std::isfinite(a->eps) || !std::isfinite(a->private_scale)) return CAAT_ERR_INVALID_ARG;
+  std::vector<uint8_t> mask;
+  s = build_mask(a->H, a->p, a->sync_idx, mask, nullptr);
+  if (s != CAAT_OK) return s;
+  if (a->T == 0) return CAAT_OK;
+  if (!a->X || !a->A || !a->W2 || !a->residual || !a->gamma || !a->out) return CAAT_ERR_INVALID_ARG;
+  if (!aligned16(a->X) || !aligned16(a->A) || !aligned16(a->W2) || !aligned16(a->residual) || !aligned16(a->gamma) ||
+      !aligned16(a->out) || (a->h_out && !aligned16(a->h_out)))
+    return CAAT_ERR_UNSUPPORTED;
+  const bool fused = (a->flags & CAAT_FLAG_FUSED_NORM) != 0;
+  const MlpWs L = mlp_ws_layout(a->T, a->H, a->F, a->P, fused);
+  if (!a->workspace || a->ws_bytes < L.total || (reinterpret_cast<uintptr_t>(a->workspace) & 255u))
+    return CAAT_ERR_WORKSPACE;
+  DeviceInfo* dev = nullptr;
+  s = device_info(&dev);
+  if (s != CAAT_OK) return s;
+  if (dev->max_pairs <= 0) return CAAT_ERR_UNSUPPORTED;
+
+  const int P = a->P;
+  const int64_t T = a->T, H = a->H, Fp = a->F / P;
+  uint8_t* ws = static_cast<uint8_t*>(a->workspace);
+  caat_bf16* Y = reinterpret_cast<caat_bf16*>(ws + L.y);
+  cudaStream_t st = a->stream;
+
+  // FC1 + SwiGLU: Y_m = silu(X_m A_gate,m^T) * (X_m A_up,m^T)
+  caat::Fc1Params fp{};
+  fp.counter = reinterpret_cast<unsigned int*>(ws);
+  fp.T = static_cast<int>(T);
+  fp.H = static_cast<int>(H);
+  fp.Fp = static_cast<int>(Fp);
+  fp.P = P;
+  fp.n_mblk = static_cast<int>((T + 2 * caat::K3_BM - 1) / (2 * caat::K3_BM));
+  fp.n_nblk = static_cast<int>((Fp + caat::K3_BN - 1) / caat::K3_BN);
+  fp.kblk = static_cast<int>((H + caat::K3_BK - 1) / caat::K3_BK);
+  const int64_t tail = H - int64_t(fp.kblk - 1) * caat::K3_BK;
+  fp.last_k16 = static_cast<int>((tail + 15) / 16);
+  const int64_t units = int64_t(P) * fp.n_mblk * fp.n_nblk;
+  if (units > INT32_MAX / 2) return CAAT_ERR_UNSUPPORTED;
+  fp.n_units = static_cast<int>(units);
+  fp.timeout_ns = timeout_ns();
+  fp.flags = a->flags;
+  CUtensorMap tmX, tmA, tmY;
+  s = make_map_3d(&tmX, a->X, H, T, P, caat::K3_BK, caat::K3_BM);
+  if (s != CAAT_OK) return s;
+  s = make_map_4d(&tmA, a->A, H, Fp, 2, P, caat::K3_BK, caat::K3_BN);
+  if (s != CAAT_OK) return s;
+  s = make_map_3d(&tmY, Y, Fp, T, P, 64, 32);
+  if (s != CAAT_OK) return s;
+
+  Recorder rec;
+  rec.begin(a->timing, st);
+  if (cudaMemsetAsync(ws, 0, kCounterBytes, st) != cudaSuccess) return CAAT_ERR_CUDA;
+  {
+    const int pairs = static_cast<int>(std::min<int64_t>(dev->max_pairs, units));
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * pairs, 1, 1);
+    cfg.blockDim = dim3(caat::K3_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = caat::K3_SMEM_BYTES;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, caat::fc1_swiglu_pair_kernel, tmX, tmA, tmY, fp) != cudaSuccess) return CAAT_ERR_CUDA;
+    if (cudaGetLastError() != cudaSuccess) return CAAT_ERR_CUDA;
+  }
+  rec.after_kernel(st);
+
+  // FC2: the partially synchronized row-parallel layer on Y
+  caat_rowpar_args r;
+  std::memset(&r, 0, sizeof(r));
+  r.X = Y;
+  r.W = a->W2;
+  r.residual = a->residual;
+  r.gamma = a->gamma;
+  r.out = a->out;
+  r.h_out = a->h_out;
+  r.workspace = ws + L.rowpar;
+  r.ws_bytes = L.y - L.rowpar;
+  r.stream = st;
+  r.T = T;
+  r.K = a->F;
+  r.H = H;
+  r.p = a->p;
+  r.eps = a->eps;
+  r.private_scale = a->private_scale;
+  r.P = P;
+  r.flags = a->flags;
+  return launch_rowpar(&r, mask, dev, reinterpret_cast<unsigned int*>(ws + L.rowpar), &rec);
 }
 
 caat_status caat_mlp_forward(const caat_bf16* X, const caat_bf16* A, const caat_bf16* W2, const caat_bf16* residual,
