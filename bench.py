@@ -33,13 +33,47 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 WORKLOADS = {
-    # name: (T, K, H, P, default p, random S?)
+    # name: (T, K, H, P, default p, random S?); for mlp-7b K is the FFN size F
     "fc2-7b": (8192, 11008, 4096, 8, 0.5, False),
     "fc2-1b": (4096, 5632, 2048, 4, 0.5, True),
     "tiny": (256, 768, 768, 2, 0.5, False),
+    "mlp-7b": (4096, 11008, 4096, 8, 0.5, False),
+    "decode-1": (1, 11008, 4096, 8, 0.5, False),
+    "decode-8": (8, 11008, 4096, 8, 0.5, False),
+    "decode-64": (64, 11008, 4096, 8, 0.5, False),
 }
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------------------------------
+# multi-rank helpers (weak scaling: every rank runs its own independent batch)
+# ---------------------------------------------------------------------------------------
+def rank_env():
+    """(world_size, rank, local_rank) from the torchrun environment (1, 0, 0 without it)."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def rank_seed(rank: int) -> int:
+    """Seed of a rank's synthetic batch: distinct per rank (independent problems)."""
+    return 1000 + rank
+
+
+def max_over_ranks(value: float, device: str = "cuda") -> float:
+    """The largest value over all ranks (device times: the job ends with its slowest rank)."""
+    import torch
+    import torch.distributed as dist
+    if not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_rank_step: float, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput: the work of all ranks divided by the (max-over-ranks) step time."""
+    return world * flops_per_rank_step / ms_per_step / 1e9
 
 
 def load_peaks():
@@ -164,9 +198,7 @@ def run_caat(args):
     from partial_activation_sync_caat_b200 import caat as C
     from partial_activation_sync_caat_b200 import inputs as I
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = rank_env()
     if world != args.gpus:
         raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
     torch.cuda.set_device(local)
@@ -186,16 +218,26 @@ def run_caat(args):
     p = args.p if args.p is not None else p_def
     ns = int((H * p) // 1)
     sync_idx = I.random_sync_idx(H, ns, seed=0) if rand else None
-    d = I.make_rowpar_inputs(T, K, H, P, seed=1000 + rank, device="cuda")
-    out = torch.empty_like(d["R"])
-    ws = C.alloc_workspace(C.caat_workspace_size(T, K, H, P), "cuda")
+    mlp = args.workload.startswith("mlp")
     stream = torch.cuda.current_stream()
-    flops = 2.0 * T * K * H
     timing = C.Timing(capacity=args.steps + 8)
+    if mlp:
+        d = I.make_mlp_inputs(T, H, K, P, seed=rank_seed(rank), device="cuda")
+        ws = C.alloc_workspace(C.caat_workspace_size(T, K, H, P, C.CAAT_VARIANT_MLP), "cuda")
+        flops = 2.0 * T * H * 2 * K + 2.0 * T * K * H
+    else:
+        d = I.make_rowpar_inputs(T, K, H, P, seed=rank_seed(rank), device="cuda")
+        ws = C.alloc_workspace(C.caat_workspace_size(T, K, H, P), "cuda")
+        flops = 2.0 * T * K * H
+    out = torch.empty_like(d["R"])
 
     def step(tm=None):
-        C.caat_rowpar_forward(d["X"], d["W"], d["R"], d["gamma"], sync_idx, P, p, out, workspace=ws,
-                              stream=stream, timing=tm, flags=args.flags)
+        if mlp:
+            C.caat_mlp_forward(d["X"], d["A"], d["W2"], d["R"], d["gamma"], sync_idx, P, p, out, workspace=ws,
+                               stream=stream, timing=tm, flags=args.flags)
+        else:
+            C.caat_rowpar_forward(d["X"], d["W"], d["R"], d["gamma"], sync_idx, P, p, out, workspace=ws,
+                                  stream=stream, timing=tm, flags=args.flags)
 
     for _ in range(args.warmup):
         step()
@@ -218,20 +260,19 @@ def run_caat(args):
     if world > 1:
         dist.barrier()
     clocks = sampler.stop() if sampler else None
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1))
     per_kernel = timing.read()
-    k1 = [r[0] for r in per_kernel if len(r) >= 1]
-    k2 = [r[1] for r in per_kernel if len(r) >= 2]
     n_kernels = max((len(r) for r in per_kernel), default=1)
+    kernel_ms = [statistics.mean(r[j] for r in per_kernel if len(r) > j) for j in range(n_kernels)]
+    # index of the row-parallel GEMM kernel in the per-call kernel list (FC1 comes first in the MLP)
+    kg = 1 if mlp else 0
+    k1 = [r[kg] for r in per_kernel if len(r) > kg]
+    k2 = [r[kg + 1] for r in per_kernel if len(r) > kg + 1]
     status = C.caat_get_device_status()
 
     # optional p sweep (same shapes, fewer steps), rank 0 only
     sweep = None
-    if args.sweep and rank == 0:
+    if args.sweep and rank == 0 and not mlp:
         sweep = {}
         for ps in (0.0, 0.25, 0.5, 0.75, 1.0):
             idx_s = I.random_sync_idx(H, int((H * ps) // 1), seed=0) if rand else None
@@ -252,7 +293,7 @@ def run_caat(args):
 
     # end to end through the host-buffer entry point (pinned host tensors, copies timed)
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not mlp:
         hX, hW, hR, hg = (d[k].cpu().pin_memory() for k in ("X", "W", "R", "gamma"))
         hout = torch.empty(hR.shape, dtype=torch.bfloat16).pin_memory()
         wsh = C.alloc_workspace(C.caat_workspace_size(T, K, H, P, C.CAAT_VARIANT_ROWPAR_HOST), "cuda")
@@ -268,14 +309,10 @@ def run_caat(args):
             C.caat_rowpar_forward_host(hX, hW, hR, hg, sync_idx, P, p, hout, wsh, stream=stream)
         b.record(stream)
         torch.cuda.synchronize()
-        e_ms = a.elapsed_time(b) / n_e2e
-        if world > 1:
-            t = torch.tensor([e_ms], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = max_over_ranks(a.elapsed_time(b) / n_e2e)
         h2d = sum(x.numel() * 2 for x in (hX, hW, hR, hg))
         d2h = hout.numel() * 2
-        e2e = {"value": round(world * flops / e_ms / 1e9, 2), "unit": "TFLOP/s",
+        e2e = {"value": round(whole_job_tflops(flops, world, e_ms), 2), "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms, 3),
                "api": "caat_rowpar_forward_host (pinned host buffers; H2D of X, W, residual, gamma and "
                       "D2H of out inside the timed region)"}
@@ -289,10 +326,11 @@ def run_caat(args):
 
     peaks, peak_src = load_peaks()
     ms_step = ms / args.steps
-    value = world * flops / ms_step / 1e9  # TFLOP/s, whole job
+    value = whole_job_tflops(flops, world, ms_step)
     k1_ms = statistics.mean(k1) if k1 else float("nan")
     k2_ms = statistics.mean(k2) if k2 else None
-    k1_tflops = flops / k1_ms / 1e9
+    fc2_flops = 2.0 * T * K * H
+    k1_tflops = fc2_flops / k1_ms / 1e9
     norm_bytes = 2.0 * P * T * H * 2
     k2_gbs = norm_bytes / k2_ms / 1e6 if k2_ms else None
     alg_bytes = 2.0 * (P * T * (K // P) + P * H * (K // P) + 2 * P * T * H + H)
@@ -327,6 +365,14 @@ def run_caat(args):
         "device_status": status,
         "clocks": clocks,
     }
+    result["kernels_ms"] = [round(x, 4) for x in kernel_ms]
+    if mlp:
+        result["metric"] = "TFLOP/s of the partially-synced MLP block (FC1+SwiGLU+FC2+residual+RMSNorm, 7B shape)"
+        result["fc1_kernel"] = {"kernel": "fc1_swiglu_pair_kernel", "launch_ms": round(kernel_ms[0], 4),
+                                "achieved_tflops": round(2.0 * T * H * 2 * K / kernel_ms[0] / 1e9, 1)}
+    if T <= 64:
+        result["decode"] = {"us_per_call": round(ms_step * 1e3, 2), "hbm_gbs": round(alg_bytes / ms_step / 1e6, 1),
+                            "frac_of_measured_hbm": round(alg_bytes / ms_step / 1e6 / peaks["hbm_gbs"], 3)}
     if k2_ms:
         result["norm_kernel"] = {"kernel": "rownorm_kernel", "bound": "hbm", "achieved": round(k2_gbs, 1),
                                  "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(k2_gbs / peaks["hbm_gbs"], 3),

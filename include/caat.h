@@ -62,7 +62,8 @@ typedef enum caat_status {
 /* Limits of this build. */
 #define CAAT_MAX_H 65536      /* hidden size H */
 #define CAAT_MAX_P 64         /* emulated tensor-parallel ranks */
-#define CAAT_DECODE_MAX_T 64  /* T <= this uses the decode (weight-streaming) path */
+#define CAAT_DECODE_MAX_T 64  /* 1 <= T <= this (with P <= 16, H <= 8192) uses the decode
+                                 (weight-streaming) path */
 
 /* Workspace variants for caat_workspace_size(). */
 #define CAAT_VARIANT_ROWPAR 0 /* caat_rowpar_forward[_ex]; K = FFN dim */

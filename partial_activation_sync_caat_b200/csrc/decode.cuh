@@ -1,0 +1,292 @@
+// decode.cuh - the partially synchronized row-parallel layer for decode-sized token counts
+// (T <= 64): the same result as rowpar_gemm*.cuh + rownorm.cuh, reorganized for a call
+// whose cost is streaming W once from HBM.
+//
+// "Tensor-Parallelism with Partially Synchronized Activations": partial products Zt_m =
+// X_m W_m^T (App. A.2 Eq. 22, first line), partial channel-reduce (Eq. 22, second line),
+// private scale (§4 Eq. 14-15), residual add and RMSNorm (§4 Eq. 9); §3.2 describes running
+// all tensor-parallel ranks on one device ("logical devices").
+//
+// K4a decode_partials_kernel: every (rank, 128-channel block, K split) is one unit; a
+//     persistent CTA streams W_m's 128 x (K/P)/splits slice with TMA and computes the swapped
+//     product D[c, t] = W_m[c,:] . X_m[t,:] with tcgen05.mma (M = 128 channels, N = T padded to
+//     a multiple of 16, fp32 in TMEM), then writes the fp32 partial Zp[split][m][t][c].  The
+//     tokens are the N side, so W (the only large operand) is read exactly once.
+// K4b decode_reduce_norm_kernel: one CTA per (rank m, token t) row.  It sums the K splits
+//     of rank m's partial, forms the shared channels' cross-rank sum (rank order 0..P-1,
+//     fp32), applies the private scale, adds the residual, stores h (bf16), reduces the sum
+//     of squares of the stored h over the CTA and rescales the row held in registers:
+//     out = h / sqrt(sum/H + eps) * gamma.
+#pragma once
+
+#include "ptx.cuh"
+#include "rowpar_common.cuh"
+
+namespace caat {
+
+constexpr int K4_BM = 128;                 // channels per unit
+constexpr int K4_BK = 64;
+constexpr int K4_STAGES = 8;
+constexpr int K4_MAXN = 64;                // max padded token count
+constexpr int K4_A_BYTES = K4_BM * K4_BK * 2;       // 16 KiB of W
+constexpr int K4_B_BYTES = K4_MAXN * K4_BK * 2;     // up to 8 KiB of X
+constexpr int K4_STAGE_BYTES = K4_A_BYTES + K4_B_BYTES;
+constexpr int K4_THREADS = 192;
+constexpr int K4_SMEM_BYTES = 1024 + K4_STAGES * K4_STAGE_BYTES + 256;
+constexpr int K4_TMEM_COLS = 128;          // two accumulators of up to 64 columns
+constexpr int K4_MAXP = 16;                // ranks supported by the reduce kernel
+constexpr int K4B_THREADS = 256;
+constexpr int K4B_VEC = 4;                 // 16-byte vectors per thread: H <= 8 * 256 * 4 = 8192
+
+struct DecodeParams {
+  float* Zp;                  // [splits][P][T][H] fp32 partials
+  const __nv_bfloat16* R;     // residual [P, T, H]
+  __nv_bfloat16* Hout;        // h [P, T, H]
+  __nv_bfloat16* Out;         // out [P, T, H]
+  const __nv_bfloat16* gamma;
+  int T, Tpad, H, Kp, P;
+  int n_cb;                   // ceil(H / 128)
+  int splits;                 // K splits
+  int kb_per_split;           // k-blocks (64) per split
+  int kblk;                   // ceil(Kp / 64)
+  int last_k16;               // 16-wide steps in the last k-block of a rank
+  int n_units;                // P * n_cb * splits
+  float private_scale, eps;
+  uint64_t timeout_ns;
+  uint32_t mask_bits[K1_MASK_WORDS];
+};
+
+__global__ void __launch_bounds__(K4_THREADS, 1)
+    decode_partials_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                           const __grid_constant__ DecodeParams prm) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + K4_STAGES * K4_A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + K4_STAGES * K4_STAGE_BYTES);
+  uint64_t* full = bars;
+  uint64_t* empty = full + K4_STAGES;
+  uint64_t* tfull = empty + K4_STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* mma_done = tempty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < K4_STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);
+    }
+    mbar_init(mma_done, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&tmW);
+    tma_prefetch_desc(&tmX);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, K4_TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const uint64_t tmo = prm.timeout_ns;
+  const int per_rank = prm.n_cb * prm.splits;
+  const uint32_t b_bytes = static_cast<uint32_t>(prm.Tpad) * K4_BK * 2;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_first();  // W is streamed once
+      const uint64_t pol_x = policy_evict_last();   // X is reused by every unit of its rank
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true, issued = false;
+      for (int u = blockIdx.x; u < prm.n_units && ok; u += gridDim.x) {
+        const int r = u / per_rank;
+        const int rem = u - r * per_rank;
+        const int cb = rem / prm.splits;
+        const int sp = rem - cb * prm.splits;
+        const int kb0 = sp * prm.kb_per_split;
+        const int kb1 = min(prm.kblk, kb0 + prm.kb_per_split);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, tmo, 61)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[stage], K4_A_BYTES + b_bytes);
+          tma_load_3d(sA + stage * K4_A_BYTES, &tmW, &full[stage], kb * K4_BK, cb * K4_BM, r, pol_w);
+          tma_load_3d(sB + stage * K4_B_BYTES, &tmX, &full[stage], kb * K4_BK, 0, r, pol_x);
+          issued = true;
+          if (++stage == K4_STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+      if (!ok && issued) spin_ns(1000000);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(K4_BM, prm.Tpad);
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < prm.n_units && ok; u += gridDim.x) {
+        const int rem = u % per_rank;
+        const int sp = rem % prm.splits;
+        const int kb0 = sp * prm.kb_per_split;
+        const int kb1 = min(prm.kblk, kb0 + prm.kb_per_split);
+        const int buf = local & 1;
+        const uint32_t bph = (local >> 1) & 1;
+        if (!mbar_wait(&tempty[buf], bph ^ 1, tmo, 62)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t dt = tmem_base + static_cast<uint32_t>(buf * K4_MAXN);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&full[stage], phase, tmo, 63)) { ok = false; break; }
+          tc_fence_after();
+          const int nk16 = (kb == prm.kblk - 1) ? prm.last_k16 : (K4_BK / 16);
+          const uint32_t a_addr = smem_u32(sA + stage * K4_A_BYTES);
+          const uint32_t b_addr = smem_u32(sB + stage * K4_B_BYTES);
+          for (int kk = 0; kk < nk16; ++kk)
+            umma_bf16(dt, sw128_kmajor_desc(a_addr + kk * 32), sw128_kmajor_desc(b_addr + kk * 32), idesc,
+                      (kb > kb0 || kk > 0) ? 1u : 0u);
+          umma_commit(&empty[stage]);
+          if (++stage == K4_STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[buf]);
+        ++local;
+      }
+      umma_commit(mma_done);
+      mbar_wait(mma_done, 0, tmo, 64);
+    }
+  } else {
+    const int q = warp & 3;
+    int local = 0;
+    for (int u = blockIdx.x; u < prm.n_units; u += gridDim.x) {
+      const int r = u / per_rank;
+      const int rem = u - r * per_rank;
+      const int cb = rem / prm.splits;
+      const int sp = rem - cb * prm.splits;
+      const int buf = local & 1;
+      const uint32_t bph = (local >> 1) & 1;
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait(&tfull[buf], bph, tmo, 65) ? 1 : 0;
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t trow = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * K4_MAXN);
+      uint32_t v[64];
+      __syncwarp();
+      tmem_ld_32x32b_x32(trow, *reinterpret_cast<uint32_t(*)[32]>(v));
+      if (prm.Tpad > 32) tmem_ld_32x32b_x32(trow + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[buf]);
+      const int c = cb * K4_BM + q * 32 + lane;
+      if (c < prm.H) {
+        float* zp = prm.Zp + ((static_cast<size_t>(sp) * prm.P + r) * prm.T) * prm.H + c;
+#pragma unroll
+        for (int t = 0; t < K4_MAXN; ++t)
+          if (t < prm.T) zp[static_cast<size_t>(t) * prm.H] = __uint_as_float(v[t]);
+      }
+      ++local;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, K4_TMEM_COLS);
+}
+
+// Sum of the K splits of rank r's partial for 8 channels starting at c.
+__device__ __forceinline__ void k4_load_z(const DecodeParams& prm, int r, int t, int c, float (&z)[8]) {
+#pragma unroll
+  for (int e = 0; e < 8; ++e) z[e] = 0.f;
+  for (int sp = 0; sp < prm.splits; ++sp) {
+    const float4* p = reinterpret_cast<const float4*>(
+        prm.Zp + ((static_cast<size_t>(sp) * prm.P + r) * prm.T + t) * prm.H + c);
+    const float4 a = __ldcg(p), b = __ldcg(p + 1);
+    z[0] += a.x; z[1] += a.y; z[2] += a.z; z[3] += a.w;
+    z[4] += b.x; z[5] += b.y; z[6] += b.z; z[7] += b.w;
+  }
+}
+
+// One CTA per (rank r, token t): the full row of h_r[t, :] (8 channels per thread and
+// vector slot, at most K4B_VEC slots held in registers), its sum of squares by a block
+// reduction, then the rescaled row.
+__global__ void __launch_bounds__(K4B_THREADS)
+    decode_reduce_norm_kernel(const __grid_constant__ DecodeParams prm) {
+  __shared__ float red[K4B_THREADS / 32];
+  __shared__ float s_rstd;
+  const int r = blockIdx.x % prm.P;
+  const int t = blockIdx.x / prm.P;
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int nvec = prm.H >> 3;
+  const size_t rowoff = (static_cast<size_t>(r) * prm.T + t) * prm.H;
+  uint4 hv[K4B_VEC];
+  float ss = 0.f;
+#pragma unroll
+  for (int k = 0; k < K4B_VEC; ++k) {
+    const int v = threadIdx.x + k * K4B_THREADS;
+    hv[k] = make_uint4(0, 0, 0, 0);
+    if (v >= nvec) continue;
+    const int c = 8 * v;
+    const uint32_t bits = (prm.mask_bits[c >> 5] >> (c & 31)) & 0xFFu;  // 8 channels, 8-aligned
+    float z[8], s[8];
+    if (bits != 0xFFu) k4_load_z(prm, r, t, c, z);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) s[e] = 0.f;
+    if (bits) {
+      for (int q = 0; q < prm.P; ++q) {  // cross-rank sum of the shared channels, ranks in order
+        float zq[8];
+        k4_load_z(prm, q, t, c, zq);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) s[e] += zq[e];
+      }
+    }
+    const uint4 rv = *reinterpret_cast<const uint4*>(prm.R + rowoff + c);
+    const uint32_t rw[4] = {rv.x, rv.y, rv.z, rv.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float z0 = ((bits >> (2 * e)) & 1u) ? s[2 * e] : prm.private_scale * z[2 * e];
+      const float z1 = ((bits >> (2 * e + 1)) & 1u) ? s[2 * e + 1] : prm.private_scale * z[2 * e + 1];
+      o[e] = pack_bf16x2(z0 + bf16lo(rw[e]), z1 + bf16hi(rw[e]));
+      const float lo = bf16lo(o[e]), hi = bf16hi(o[e]);
+      ss = fmaf(lo, lo, ss);
+      ss = fmaf(hi, hi, ss);
+    }
+    hv[k] = make_uint4(o[0], o[1], o[2], o[3]);
+    *reinterpret_cast<uint4*>(prm.Hout + rowoff + c) = hv[k];
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, off);
+  if (lane == 0) red[warp] = ss;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float v = 0.f;
+    for (int w = 0; w < K4B_THREADS / 32; ++w) v += red[w];
+    s_rstd = rsqrtf(v / static_cast<float>(prm.H) + prm.eps);
+  }
+  __syncthreads();
+  const float rs = s_rstd;
+  const uint4* g4 = reinterpret_cast<const uint4*>(prm.gamma);
+#pragma unroll
+  for (int k = 0; k < K4B_VEC; ++k) {
+    const int v = threadIdx.x + k * K4B_THREADS;
+    if (v >= nvec) continue;
+    const uint4 g = g4[v];
+    const uint32_t w[4] = {hv[k].x, hv[k].y, hv[k].z, hv[k].w};
+    const uint32_t gw[4] = {g.x, g.y, g.z, g.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      o[e] = pack_bf16x2(bf16lo(w[e]) * rs * bf16lo(gw[e]), bf16hi(w[e]) * rs * bf16hi(gw[e]));
+    *reinterpret_cast<uint4*>(prm.Out + rowoff + 8 * v) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+}  // namespace caat
