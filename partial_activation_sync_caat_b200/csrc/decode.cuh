@@ -13,8 +13,8 @@
 //     a multiple of 16, fp32 in TMEM), then writes the fp32 partial Zp[split][m][t][c].  The
 //     tokens are the N side, so W (the only large operand) is read exactly once.
 // K4b decode_reduce_norm_kernel: one CTA per (rank m, token t) row.  It sums the K splits
-//     of rank m's partial, forms the shared channels' cross-rank sum (rank order 0..P-1,
-//     fp32), applies the private scale, adds the residual, stores h (bf16), reduces the sum
+//     of rank m's partial, forms the shared channels' cross-rank sum (ranks and splits in
+//     order, fp32), applies the private scale, adds the residual, stores h (bf16), reduces the sum
 //     of squares of the stored h over the CTA and rescales the row held in registers:
 //     out = h / sqrt(sum/H + eps) * gamma.
 #pragma once
@@ -35,8 +35,8 @@ constexpr int K4_THREADS = 192;
 constexpr int K4_SMEM_BYTES = 1024 + K4_STAGES * K4_STAGE_BYTES + 256;
 constexpr int K4_TMEM_COLS = 128;          // two accumulators of up to 64 columns
 constexpr int K4_MAXP = 16;                // ranks supported by the reduce kernel
-constexpr int K4B_THREADS = 256;
-constexpr int K4B_VEC = 4;                 // 16-byte vectors per thread: H <= 8 * 256 * 4 = 8192
+constexpr int K4B_THREADS = 512;
+constexpr int K4B_VEC = 2;                 // 16-byte vectors per thread: H <= 8 * 512 * 2 = 8192
 
 struct DecodeParams {
   float* Zp;                  // [splits][P][T][H] fp32 partials
@@ -200,22 +200,50 @@ __global__ void __launch_bounds__(K4_THREADS, 1)
   if (warp == 1) tmem_dealloc(tmem_base, K4_TMEM_COLS);
 }
 
-// Sum of the K splits of rank r's partial for 8 channels starting at c.
-__device__ __forceinline__ void k4_load_z(const DecodeParams& prm, int r, int t, int c, float (&z)[8]) {
+// The partial sums a channel vector needs: own[8] = rank r's partial (all K splits) and, if
+// `shared`, s[8] = the cross-rank sum in rank order 0..P-1.  Loads go out in batches of 8
+// independent (rank, split) pairs so their latencies overlap.
+__device__ __forceinline__ void k4_gather(const DecodeParams& prm, int r, int t, int c, bool shared, float (&own)[8],
+                                          float (&s)[8]) {
 #pragma unroll
-  for (int e = 0; e < 8; ++e) z[e] = 0.f;
-  for (int sp = 0; sp < prm.splits; ++sp) {
-    const float4* p = reinterpret_cast<const float4*>(
-        prm.Zp + ((static_cast<size_t>(sp) * prm.P + r) * prm.T + t) * prm.H + c);
-    const float4 a = __ldcg(p), b = __ldcg(p + 1);
-    z[0] += a.x; z[1] += a.y; z[2] += a.z; z[3] += a.w;
-    z[4] += b.x; z[5] += b.y; z[6] += b.z; z[7] += b.w;
+  for (int e = 0; e < 8; ++e) {
+    own[e] = 0.f;
+    s[e] = 0.f;
+  }
+  const int q0 = shared ? 0 : r;
+  const int q1 = shared ? prm.P : r + 1;
+  const int n = (q1 - q0) * prm.splits;
+  for (int base = 0; base < n; base += 8) {
+    float4 a[8], b[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int idx = base + j;
+      a[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+      b[j] = a[j];
+      if (idx < n) {
+        const int q = q0 + idx / prm.splits;
+        const int sp = idx - (idx / prm.splits) * prm.splits;
+        const float4* p = reinterpret_cast<const float4*>(
+            prm.Zp + ((static_cast<size_t>(sp) * prm.P + q) * prm.T + t) * prm.H + c);
+        a[j] = __ldcg(p);
+        b[j] = __ldcg(p + 1);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int idx = base + j;
+      if (idx >= n) break;
+      const int q = q0 + idx / prm.splits;
+      const float v[8] = {a[j].x, a[j].y, a[j].z, a[j].w, b[j].x, b[j].y, b[j].z, b[j].w};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        s[e] += v[e];
+        if (q == r) own[e] += v[e];
+      }
+    }
   }
 }
 
-// One CTA per (rank r, token t): the full row of h_r[t, :] (8 channels per thread and
-// vector slot, at most K4B_VEC slots held in registers), its sum of squares by a block
-// reduction, then the rescaled row.
 __global__ void __launch_bounds__(K4B_THREADS)
     decode_reduce_norm_kernel(const __grid_constant__ DecodeParams prm) {
   __shared__ float red[K4B_THREADS / 32];
@@ -236,17 +264,7 @@ __global__ void __launch_bounds__(K4B_THREADS)
     const int c = 8 * v;
     const uint32_t bits = (prm.mask_bits[c >> 5] >> (c & 31)) & 0xFFu;  // 8 channels, 8-aligned
     float z[8], s[8];
-    if (bits != 0xFFu) k4_load_z(prm, r, t, c, z);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) s[e] = 0.f;
-    if (bits) {
-      for (int q = 0; q < prm.P; ++q) {  // cross-rank sum of the shared channels, ranks in order
-        float zq[8];
-        k4_load_z(prm, q, t, c, zq);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) s[e] += zq[e];
-      }
-    }
+    k4_gather(prm, r, t, c, bits != 0u, z, s);
     const uint4 rv = *reinterpret_cast<const uint4*>(prm.R + rowoff + c);
     const uint32_t rw[4] = {rv.x, rv.y, rv.z, rv.w};
     uint32_t o[4];
