@@ -141,9 +141,13 @@ CAAT_API caat_status caat_rowpar_forward_ex(const caat_rowpar_args* args);
  * for asynchronous copies; pageable memory also works, with synchronous staging).
  * args->workspace is a device buffer of caat_workspace_size(T, K, H, P,
  * CAAT_VARIANT_ROWPAR_HOST) bytes that receives device copies of the inputs and outputs.
- * The call queues on args->stream: host-to-device copies of X, W, residual and gamma, the
- * kernels of caat_rowpar_forward_ex, and device-to-host copies of out (and h_out).  The
- * host buffers must stay valid until the stream reaches that point.
+ * The call is pipelined over chunks of 1024 tokens (token rows are independent): W and gamma
+ * are copied once, then each chunk's X and residual rows are copied in, its kernels run on
+ * args->stream and its out (and h_out) rows are copied back, on two library-owned copy
+ * streams (created on the first call on a device) so that both copy directions overlap the
+ * kernels.  All of it is ordered after the work already queued on args->stream, and
+ * args->stream waits for the last copy back: the call is complete when args->stream reaches
+ * that point, and the host buffers must stay valid until then.
  */
 CAAT_API caat_status caat_rowpar_forward_host(const caat_rowpar_args* args);
 

@@ -250,24 +250,61 @@ size_t rowpar_workspace(int64_t T, int64_t K, int64_t H, int P, bool fused = tru
   return n;
 }
 
-// Device staging layout of caat_rowpar_forward_host: [rowpar workspace | X | W | R | gamma |
-// out | h], each region 256-byte aligned.
+// Device staging of caat_rowpar_forward_host.  Token rows are independent through the whole
+// path, so the call is pipelined over chunks of kHostChunk tokens: W and gamma are copied once,
+// then per chunk X and R are copied in, the kernels run and out (and h) are copied back, with
+// two chunk buffers so that copies in both directions overlap the kernels of other chunks.
+// Layout: [row-parallel workspace for one chunk | W | gamma | 2 x (X_c | R_c | O_c | H_c)].
+constexpr int64_t kHostChunk = 1024;
+
 struct HostLayout {
-  size_t ws, x, w, r, g, o, h, total;
+  int64_t Tc;
+  size_t ws, w, g, buf0, x, r, o, h, buf_bytes, total;
 };
 
 HostLayout host_layout(int64_t T, int64_t K, int64_t H, int P) {
-  HostLayout L;
+  HostLayout L{};
   const size_t Kp = static_cast<size_t>(K / P);
+  L.Tc = std::min<int64_t>(T, kHostChunk);
   L.ws = 0;
-  L.x = align256(rowpar_workspace(T, K, H, P));
-  L.w = L.x + align256(size_t(P) * T * Kp * 2);
-  L.r = L.w + align256(size_t(P) * H * Kp * 2);
-  L.g = L.r + align256(size_t(P) * T * H * 2);
-  L.o = L.g + align256(size_t(H) * 2);
-  L.h = L.o + align256(size_t(P) * T * H * 2);
-  L.total = L.h + align256(size_t(P) * T * H * 2);
+  L.w = align256(rowpar_workspace(L.Tc, K, H, P));
+  L.g = L.w + align256(size_t(P) * H * Kp * 2);
+  L.buf0 = L.g + align256(size_t(H) * 2);
+  L.x = 0;
+  L.r = align256(size_t(P) * L.Tc * Kp * 2);
+  L.o = L.r + align256(size_t(P) * L.Tc * H * 2);
+  L.h = L.o + align256(size_t(P) * L.Tc * H * 2);
+  L.buf_bytes = L.h + align256(size_t(P) * L.Tc * H * 2);
+  L.total = L.buf0 + 2 * L.buf_bytes;
   return L;
+}
+
+// Copy streams and events of the host-buffer pipeline (created once per device).
+struct HostPipe {
+  bool init = false;
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  cudaEvent_t ev_start = nullptr, ev_w = nullptr, ev_in[2] = {}, ev_comp[2] = {}, ev_out[2] = {};
+};
+HostPipe g_pipe[64];
+
+caat_status host_pipe(HostPipe** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return CAAT_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return CAAT_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_mu);
+  HostPipe& hp = g_pipe[dev];
+  if (!hp.init) {
+    if (cudaStreamCreateWithFlags(&hp.s_in, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&hp.s_out, cudaStreamNonBlocking) != cudaSuccess)
+      return CAAT_ERR_CUDA;
+    cudaEvent_t* evs[] = {&hp.ev_start, &hp.ev_w, &hp.ev_in[0], &hp.ev_in[1], &hp.ev_comp[0],
+                          &hp.ev_comp[1], &hp.ev_out[0], &hp.ev_out[1]};
+    for (cudaEvent_t* e : evs)
+      if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return CAAT_ERR_CUDA;
+    hp.init = true;
+  }
+  *out = &hp;
+  return CAAT_OK;
 }
 
 // Workspace of the MLP block: [FC1 unit counter (256 B) | row-parallel workspace | Y [P,T,F/P]].
@@ -578,41 +615,86 @@ caat_status caat_rowpar_forward_host(const caat_rowpar_args* a) {
   if (!a) return CAAT_ERR_INVALID_ARG;
   caat_status s = check_shapes(a->T, a->K, a->H, a->P, a->p);
   if (s != CAAT_OK) return s;
+  if (!(a->eps >= 0.f) || !std::isfinite(a->eps) || !std::isfinite(a->private_scale)) return CAAT_ERR_INVALID_ARG;
+  std::vector<uint8_t> mask;
+  s = build_mask(a->H, a->p, a->sync_idx, mask, nullptr);
+  if (s != CAAT_OK) return s;
   if (a->T == 0) return CAAT_OK;
   if (!a->X || !a->W || !a->residual || !a->gamma || !a->out) return CAAT_ERR_INVALID_ARG;
-  const HostLayout L = host_layout(a->T, a->K, a->H, a->P);
+  const int P = a->P;
+  const int64_t T = a->T, H = a->H, Kp = a->K / P;
+  const HostLayout L = host_layout(T, a->K, H, P);
   if (!a->workspace || a->ws_bytes < L.total || (reinterpret_cast<uintptr_t>(a->workspace) & 255u))
     return CAAT_ERR_WORKSPACE;
-  uint8_t* base = static_cast<uint8_t*>(a->workspace);
-  caat_rowpar_args d = *a;
-  d.X = reinterpret_cast<const caat_bf16*>(base + L.x);
-  d.W = reinterpret_cast<const caat_bf16*>(base + L.w);
-  d.residual = reinterpret_cast<const caat_bf16*>(base + L.r);
-  d.gamma = reinterpret_cast<const caat_bf16*>(base + L.g);
-  d.out = reinterpret_cast<caat_bf16*>(base + L.o);
-  d.h_out = a->h_out ? reinterpret_cast<caat_bf16*>(base + L.h) : nullptr;
-  d.workspace = base;
-  d.ws_bytes = L.x;
-  std::vector<uint8_t> mask;
-  s = validate_rowpar(&d, mask);
-  if (s != CAAT_OK) return s;
   DeviceInfo* dev = nullptr;
   s = device_info(&dev);
   if (s != CAAT_OK) return s;
-  const size_t Kp = static_cast<size_t>(a->K / a->P);
-  const size_t nx = size_t(a->P) * a->T * Kp * 2, nw = size_t(a->P) * a->H * Kp * 2;
-  const size_t nr = size_t(a->P) * a->T * a->H * 2, ng = size_t(a->H) * 2;
-  cudaStream_t st = a->stream;
-  if (cudaMemcpyAsync(base + L.x, a->X, nx, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-      cudaMemcpyAsync(base + L.w, a->W, nw, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-      cudaMemcpyAsync(base + L.r, a->residual, nr, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-      cudaMemcpyAsync(base + L.g, a->gamma, ng, cudaMemcpyHostToDevice, st) != cudaSuccess)
-    return CAAT_ERR_CUDA;
-  s = launch_rowpar(&d, mask, dev, static_cast<unsigned int*>(d.workspace));
+  HostPipe* hp = nullptr;
+  s = host_pipe(&hp);
   if (s != CAAT_OK) return s;
-  if (cudaMemcpyAsync(a->out, base + L.o, nr, cudaMemcpyDeviceToHost, st) != cudaSuccess) return CAAT_ERR_CUDA;
-  if (a->h_out && cudaMemcpyAsync(a->h_out, base + L.h, nr, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+  uint8_t* base = static_cast<uint8_t*>(a->workspace);
+  cudaStream_t st = a->stream;
+  const uint8_t* hX = reinterpret_cast<const uint8_t*>(a->X);
+  const uint8_t* hR = reinterpret_cast<const uint8_t*>(a->residual);
+  uint8_t* hO = reinterpret_cast<uint8_t*>(a->out);
+  uint8_t* hH = reinterpret_cast<uint8_t*>(a->h_out);
+
+  // Copies start after the work already queued on the caller's stream (which may still use
+  // this workspace).
+  if (cudaEventRecord(hp->ev_start, st) != cudaSuccess || cudaStreamWaitEvent(hp->s_in, hp->ev_start, 0) ||
+      cudaStreamWaitEvent(hp->s_out, hp->ev_start, 0))
     return CAAT_ERR_CUDA;
+  if (cudaMemcpyAsync(base + L.w, a->W, size_t(P) * H * Kp * 2, cudaMemcpyHostToDevice, hp->s_in) ||
+      cudaMemcpyAsync(base + L.g, a->gamma, size_t(H) * 2, cudaMemcpyHostToDevice, hp->s_in) ||
+      cudaEventRecord(hp->ev_w, hp->s_in) || cudaStreamWaitEvent(st, hp->ev_w, 0))
+    return CAAT_ERR_CUDA;
+
+  const int64_t nch = (T + L.Tc - 1) / L.Tc;
+  for (int64_t i = 0; i < nch; ++i) {
+    const int b = static_cast<int>(i & 1);
+    const int64_t t0 = i * L.Tc;
+    const int64_t tc = std::min<int64_t>(L.Tc, T - t0);
+    uint8_t* buf = base + L.buf0 + size_t(b) * L.buf_bytes;
+    // H2D of the chunk's X and R rows (P strided blocks each)
+    if (i >= 2 && cudaStreamWaitEvent(hp->s_in, hp->ev_comp[b], 0)) return CAAT_ERR_CUDA;
+    if (cudaMemcpy2DAsync(buf + L.x, size_t(tc) * Kp * 2, hX + size_t(t0) * Kp * 2, size_t(T) * Kp * 2,
+                          size_t(tc) * Kp * 2, P, cudaMemcpyHostToDevice, hp->s_in) ||
+        cudaMemcpy2DAsync(buf + L.r, size_t(tc) * H * 2, hR + size_t(t0) * H * 2, size_t(T) * H * 2,
+                          size_t(tc) * H * 2, P, cudaMemcpyHostToDevice, hp->s_in) ||
+        cudaEventRecord(hp->ev_in[b], hp->s_in))
+      return CAAT_ERR_CUDA;
+    // kernels of the chunk on the caller's stream
+    if (cudaStreamWaitEvent(st, hp->ev_in[b], 0)) return CAAT_ERR_CUDA;
+    if (i >= 2 && cudaStreamWaitEvent(st, hp->ev_out[b], 0)) return CAAT_ERR_CUDA;
+    caat_rowpar_args d = *a;
+    d.X = reinterpret_cast<const caat_bf16*>(buf + L.x);
+    d.W = reinterpret_cast<const caat_bf16*>(base + L.w);
+    d.residual = reinterpret_cast<const caat_bf16*>(buf + L.r);
+    d.gamma = reinterpret_cast<const caat_bf16*>(base + L.g);
+    d.out = reinterpret_cast<caat_bf16*>(buf + L.o);
+    d.h_out = a->h_out ? reinterpret_cast<caat_bf16*>(buf + L.h) : nullptr;
+    d.workspace = base;
+    d.ws_bytes = L.w;
+    d.T = tc;
+    std::vector<uint8_t> m2;
+    s = validate_rowpar(&d, m2);
+    if (s != CAAT_OK) return s;
+    s = launch_rowpar(&d, mask, dev, reinterpret_cast<unsigned int*>(base));
+    if (s != CAAT_OK) return s;
+    if (cudaEventRecord(hp->ev_comp[b], st)) return CAAT_ERR_CUDA;
+    // D2H of the chunk's out (and h) rows
+    if (cudaStreamWaitEvent(hp->s_out, hp->ev_comp[b], 0) ||
+        cudaMemcpy2DAsync(hO + size_t(t0) * H * 2, size_t(T) * H * 2, buf + L.o, size_t(tc) * H * 2,
+                          size_t(tc) * H * 2, P, cudaMemcpyDeviceToHost, hp->s_out))
+      return CAAT_ERR_CUDA;
+    if (hH && cudaMemcpy2DAsync(hH + size_t(t0) * H * 2, size_t(T) * H * 2, buf + L.h, size_t(tc) * H * 2,
+                                size_t(tc) * H * 2, P, cudaMemcpyDeviceToHost, hp->s_out))
+      return CAAT_ERR_CUDA;
+    if (cudaEventRecord(hp->ev_out[b], hp->s_out)) return CAAT_ERR_CUDA;
+  }
+  // The call is complete on the caller's stream once the last copies back are done.
+  if (cudaStreamWaitEvent(st, hp->ev_out[(nch - 1) & 1], 0)) return CAAT_ERR_CUDA;
+  if (nch > 1 && cudaStreamWaitEvent(st, hp->ev_out[nch & 1], 0)) return CAAT_ERR_CUDA;
   return CAAT_OK;
 }
 

@@ -187,3 +187,25 @@ def test_stall_reports_timeout_and_context_survives(flags):
     assert st & 0xFF == C.CAAT_ERR_TIMEOUT
     assert C.caat_get_device_status() == 0     # cleared by the read
     _compare(d, 2, 0.5, what="after timeout")
+
+
+# ------------------------------------------------------------------ host-buffer entry point
+@pytest.mark.parametrize("T", [300, 2500])
+def test_host_buffer_entry_matches_device_entry(T):
+    """caat_rowpar_forward_host (pipelined over 1024-token chunks: 1 or 3 chunks here) gives
+    the same bits as the device entry point: rows are independent and every kernel is
+    deterministic per row."""
+    P, K, H = 4, 1024, 776
+    d = I.make_rowpar_inputs(T, K, H, P, seed=17, x_std=1.0, w_std=0.05, r_std=1.0, gamma="uniform")
+    out_dev, h_dev = run_rowpar(d, P, 0.5)
+    hX, hW, hR, hg = (d[k].contiguous().pin_memory() for k in ("X", "W", "R", "gamma"))
+    hout = torch.empty(P, T, H, dtype=torch.bfloat16).pin_memory()
+    hh = torch.empty(P, T, H, dtype=torch.bfloat16).pin_memory()
+    ws = C.alloc_workspace(C.caat_workspace_size(T, K, H, P, C.CAAT_VARIANT_ROWPAR_HOST))
+    for _ in range(2):   # a second call reuses the workspace and the copy streams
+        hout.zero_()
+        C.caat_rowpar_forward_host(hX, hW, hR, hg, None, P, 0.5, hout, ws, h_out=hh)
+        torch.cuda.synchronize()
+        assert C.caat_get_device_status() == 0
+        assert torch.equal(hout, out_dev)
+        assert torch.equal(hh, h_dev)
