@@ -79,6 +79,9 @@ typedef enum caat_status {
 #define CAAT_FLAG_ORDER_ROWBLOCK 0x10u   /* schedule the GEMM tiles row block by row block
                                             (default: shared-channel tiles first, then the
                                             private tiles rank by rank) */
+#define CAAT_FLAG_OVERLAP_NORM 0x20u     /* T >= 4096: run the GEMM in 2048-token launches and the
+                                            row norm of each launch's tokens on a library-owned
+                                            side stream, overlapping the next launch */
 #define CAAT_FLAG_SINGLE_CTA 0x4u        /* use the single-CTA GEMM kernel (128-token tiles)
                                             instead of the CTA-pair kernel (256-token tiles) */
 #define CAAT_FLAG_TEST_STALL 0x100u      /* test hook: the GEMM kernel's MMA warp never signals

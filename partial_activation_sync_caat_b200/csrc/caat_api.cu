@@ -279,6 +279,34 @@ HostLayout host_layout(int64_t T, int64_t K, int64_t H, int P) {
   return L;
 }
 
+constexpr int64_t kNormChunk = 2048;  // tokens per GEMM launch when the norm is overlapped
+
+// Side stream and events that let the row norm of one chunk of tokens run while the GEMM
+// kernel computes the next chunk (created once per device).
+struct NormSide {
+  bool init = false;
+  cudaStream_t s = nullptr;
+  cudaEvent_t ev_gemm = nullptr, ev_done = nullptr;
+};
+NormSide g_side[64];
+
+caat_status norm_side(NormSide** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return CAAT_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return CAAT_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_mu);
+  NormSide& ns = g_side[dev];
+  if (!ns.init) {
+    if (cudaStreamCreateWithFlags(&ns.s, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ns.ev_gemm, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ns.ev_done, cudaEventDisableTiming) != cudaSuccess)
+      return CAAT_ERR_CUDA;
+    ns.init = true;
+  }
+  *out = &ns;
+  return CAAT_OK;
+}
+
 // Copy streams and events of the host-buffer pipeline (created once per device).
 struct HostPipe {
   bool init = false;
@@ -447,7 +475,6 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
   prm.H = static_cast<int>(H);
   prm.Kp = static_cast<int>(Kp);
   prm.P = P;
-  prm.n_mblk = static_cast<int>((T + caat::K1_BM - 1) / caat::K1_BM);
   prm.kblk_per_rank = static_cast<int>((Kp + caat::K1_BK - 1) / caat::K1_BK);
   const int64_t tail = Kp - int64_t(prm.kblk_per_rank - 1) * caat::K1_BK;
   prm.last_k16 = static_cast<int>((tail + 15) / 16);
@@ -467,22 +494,14 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
   }
   for (int64_t c = 0; c < H; ++c)
     if (mask[c]) prm.mask_bits[c >> 5] |= 1u << (c & 31);
-  const int64_t units = int64_t(prm.n_mblk) * (prm.nS + int64_t(P) * prm.nPriv);
-  if (units > INT32_MAX / 2) return CAAT_ERR_UNSUPPORTED;
-  prm.n_units = static_cast<int>(units);
   prm.nslots = prm.nS + prm.nPriv;
-  prm.T_pad = static_cast<int>(int64_t(prm.n_mblk) * caat::K1_BM);
-  prm.n_rb = prm.n_mblk * P;
-
   // The CTA-pair kernel (256-token tiles) for all but the smallest token counts.
   const bool pair = !(a->flags & CAAT_FLAG_SINGLE_CTA) && dev->max_pairs > 0 && T > caat::K1_BM;
-  if (pair) {
-    prm.n_mblk = static_cast<int>((T + 2 * caat::K2P_BM - 1) / (2 * caat::K2P_BM));
-    const int64_t pu = int64_t(prm.n_mblk) * (prm.nS + int64_t(P) * prm.nPriv);
-    prm.n_units = static_cast<int>(pu);
-    prm.T_pad = prm.n_mblk * 2 * caat::K2P_BM;
-    prm.n_rb = 2 * prm.n_mblk * P;
-  }
+  const int64_t bm = pair ? 2 * caat::K2P_BM : caat::K1_BM;
+  if ((T + bm - 1) / bm * (prm.nS + int64_t(P) * prm.nPriv) > INT32_MAX / 2) return CAAT_ERR_UNSUPPORTED;
+  prm.T_pad = static_cast<int>((T + bm - 1) / bm * bm);
+  prm.n_rb = static_cast<int>(prm.T_pad / 128 * P);
+
   CUtensorMap tmX, tmW, tmR, tmH;
   caat_status s = make_map_3d(&tmX, a->X, Kp, T, P, caat::K1_BK, caat::K1_BM);
   if (s != CAAT_OK) return s;
@@ -494,48 +513,85 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
   s = make_map_3d(&tmH, hdst, H, T, P, 64, 32);
   if (s != CAAT_OK) return s;
 
+  // One GEMM launch over the token rows [t0, t0 + tc) (t0 a multiple of the tile height).
+  auto gemm = [&](int64_t t0, int64_t tc) -> caat_status {
+    prm.t_begin = static_cast<int>(t0);
+    prm.t_end = static_cast<int>(t0 + tc);
+    prm.n_mblk = static_cast<int>((tc + bm - 1) / bm);
+    const int64_t units = int64_t(prm.n_mblk) * (prm.nS + int64_t(P) * prm.nPriv);
+    prm.n_units = static_cast<int>(units);
+    if (cudaMemsetAsync(counter, 0, wl.zeroed, st) != cudaSuccess) return CAAT_ERR_CUDA;
+    if (pair) {
+      const int pairs = static_cast<int>(std::min<int64_t>(dev->max_pairs, units));
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.gridDim = dim3(2 * pairs, 1, 1);
+      cfg.blockDim = dim3(fused ? caat::K1Threads<true>::value : caat::K1Threads<false>::value, 1, 1);
+      cfg.dynamicSmemBytes = caat::K2P_SMEM_BYTES;
+      cfg.stream = st;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      const cudaError_t e =
+          fused ? cudaLaunchKernelEx(&cfg, caat::rowpar_gemm_pair_kernel<true>, tmX, tmW, tmR, tmH, prm)
+                : cudaLaunchKernelEx(&cfg, caat::rowpar_gemm_pair_kernel<false>, tmX, tmW, tmR, tmH, prm);
+      if (e != cudaSuccess) return CAAT_ERR_CUDA;
+    } else {
+      const int grid = static_cast<int>(std::min<int64_t>(dev->sm_count, units));
+      if (fused)
+        caat::rowpar_gemm_kernel<true><<<grid, caat::K1Threads<true>::value, caat::K1_SMEM_BYTES, st>>>(
+            tmX, tmW, tmR, tmH, prm);
+      else
+        caat::rowpar_gemm_kernel<false><<<grid, caat::K1Threads<false>::value, caat::K1_SMEM_BYTES, st>>>(
+            tmX, tmW, tmR, tmH, prm);
+    }
+    return cudaGetLastError() == cudaSuccess ? CAAT_OK : CAAT_ERR_CUDA;
+  };
+  // The row norm of the token rows [t0, t0 + tc) of every rank, on stream `ns`.
+  const __nv_bfloat16* g = reinterpret_cast<const __nv_bfloat16*>(a->gamma);
+  __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(a->out);
+  auto norm = [&](int64_t t0, int64_t tc, cudaStream_t ns, int64_t max_blocks) -> caat_status {
+    const int64_t rows = int64_t(P) * tc;
+    const int64_t warps_per_block = caat::K2_THREADS / 32;
+    const int64_t blocks = std::min<int64_t>((rows + warps_per_block - 1) / warps_per_block, max_blocks);
+    caat::rownorm_kernel<<<blocks, caat::K2_THREADS, 0, ns>>>(hdst, o, g, P, T, t0, tc, static_cast<int>(H),
+                                                              a->eps);
+    return cudaGetLastError() == cudaSuccess ? CAAT_OK : CAAT_ERR_CUDA;
+  };
+
   Recorder own;
   Recorder& rec = outer ? *outer : own;
   if (!outer) rec.begin(a->timing, st);
-  if (cudaMemsetAsync(counter, 0, wl.zeroed, st) != cudaSuccess) return CAAT_ERR_CUDA;
-  if (pair) {
-    const int pairs = static_cast<int>(std::min<int64_t>(dev->max_pairs, prm.n_units));
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.gridDim = dim3(2 * pairs, 1, 1);
-    cfg.blockDim = dim3(fused ? caat::K1Threads<true>::value : caat::K1Threads<false>::value, 1, 1);
-    cfg.dynamicSmemBytes = caat::K2P_SMEM_BYTES;
-    cfg.stream = st;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    const cudaError_t e =
-        fused ? cudaLaunchKernelEx(&cfg, caat::rowpar_gemm_pair_kernel<true>, tmX, tmW, tmR, tmH, prm)
-              : cudaLaunchKernelEx(&cfg, caat::rowpar_gemm_pair_kernel<false>, tmX, tmW, tmR, tmH, prm);
-    if (e != cudaSuccess) return CAAT_ERR_CUDA;
-  } else {
-    const int grid = static_cast<int>(std::min<int64_t>(dev->sm_count, units));
-    if (fused)
-      caat::rowpar_gemm_kernel<true><<<grid, caat::K1Threads<true>::value, caat::K1_SMEM_BYTES, st>>>(tmX, tmW, tmR,
-                                                                                                     tmH, prm);
-    else
-      caat::rowpar_gemm_kernel<false><<<grid, caat::K1Threads<false>::value, caat::K1_SMEM_BYTES, st>>>(tmX, tmW, tmR,
-                                                                                                       tmH, prm);
+  const bool overlap = !fused && (a->flags & CAAT_FLAG_OVERLAP_NORM) && T >= 2 * kNormChunk;
+  if (!overlap) {
+    s = gemm(0, T);
+    if (s != CAAT_OK) return s;
+    rec.after_kernel(st);
+    if (fused) return CAAT_OK;
+    s = norm(0, T, st, int64_t(dev->sm_count) * 4);
+    if (s != CAAT_OK) return s;
+    rec.after_kernel(st);
+    return CAAT_OK;
   }
-  if (cudaGetLastError() != cudaSuccess) return CAAT_ERR_CUDA;
+  // Chunked: the GEMM of chunk i + 1 runs on the caller's stream while the row norm of chunk i
+  // runs on the side stream (a norm block fits on an SM beside a GEMM CTA).  Recorded
+  // intervals: [start, last GEMM done], [last GEMM done, all norms done].
+  NormSide* side = nullptr;
+  s = norm_side(&side);
+  if (s != CAAT_OK) return s;
+  for (int64_t t0 = 0; t0 < T; t0 += kNormChunk) {
+    const int64_t tc = std::min<int64_t>(kNormChunk, T - t0);
+    s = gemm(t0, tc);
+    if (s != CAAT_OK) return s;
+    if (cudaEventRecord(side->ev_gemm, st) || cudaStreamWaitEvent(side->s, side->ev_gemm, 0)) return CAAT_ERR_CUDA;
+    s = norm(t0, tc, side->s, dev->sm_count);
+    if (s != CAAT_OK) return s;
+  }
   rec.after_kernel(st);
-  if (fused) return CAAT_OK;
-
-  const int64_t rows = int64_t(P) * T;
-  const int64_t warps_per_block = caat::K2_THREADS / 32;
-  const int64_t blocks = std::min<int64_t>((rows + warps_per_block - 1) / warps_per_block, int64_t(dev->sm_count) * 4);
-  const __nv_bfloat16* g = reinterpret_cast<const __nv_bfloat16*>(a->gamma);
-  __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(a->out);
-  caat::rownorm_kernel<<<blocks, caat::K2_THREADS, 0, st>>>(hdst, o, g, rows, static_cast<int>(H), a->eps);
-  if (cudaGetLastError() != cudaSuccess) return CAAT_ERR_CUDA;
+  if (cudaEventRecord(side->ev_done, side->s) || cudaStreamWaitEvent(st, side->ev_done, 0)) return CAAT_ERR_CUDA;
   rec.after_kernel(st);
   return CAAT_OK;
 }

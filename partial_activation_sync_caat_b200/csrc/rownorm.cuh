@@ -18,9 +18,11 @@ namespace caat {
 
 constexpr int K2_THREADS = 256;
 
+// Normalizes the rows (r, t) for every rank r and t in [t0, t0 + tc) of [P, T, H] tensors.
 __global__ void __launch_bounds__(K2_THREADS, 4)
-    rownorm_kernel(const __nv_bfloat16* h, __nv_bfloat16* out, const __nv_bfloat16* __restrict__ gamma,
-                   int64_t rows, int H, float eps) {
+    rownorm_kernel(const __nv_bfloat16* h, __nv_bfloat16* out, const __nv_bfloat16* __restrict__ gamma, int P,
+                   int64_t T, int64_t t0, int64_t tc, int H, float eps) {
+  const int64_t rows = static_cast<int64_t>(P) * tc;
   constexpr int U = 8;  // vectors per lane in flight
   const int lane = threadIdx.x & 31;
   const int64_t warp_global = (static_cast<int64_t>(blockIdx.x) * K2_THREADS + threadIdx.x) >> 5;
@@ -29,7 +31,9 @@ __global__ void __launch_bounds__(K2_THREADS, 4)
   const float inv_h = 1.0f / static_cast<float>(H);
   const uint4* g4 = reinterpret_cast<const uint4*>(gamma);
 
-  for (int64_t row = warp_global; row < rows; row += nwarps) {
+  for (int64_t i = warp_global; i < rows; i += nwarps) {
+    const int64_t r = i / tc;
+    const int64_t row = r * T + t0 + (i - r * tc);
     const uint4* hp = reinterpret_cast<const uint4*>(h + row * H);
     uint4* op = reinterpret_cast<uint4*>(out + row * H);
     float ss = 0.f;

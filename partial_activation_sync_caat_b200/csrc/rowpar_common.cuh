@@ -56,8 +56,9 @@ struct RowparParams {
   unsigned int* rb_count;      // [n_rb] tiles done per (row block, rank), zero at launch
   unsigned int* job_slots;     // [n_rb] published row-block ids + 1, zero at launch
   float* ss_part;              // [P][T_pad][nslots] per-row sum-of-squares partials
-  int T, H, Kp, P;
-  int n_mblk;                  // row blocks of the kernel's tile height
+  int T, H, Kp, P;             // T: token rows of the tensors (the row stride of rank blocks)
+  int t_begin, t_end;          // token rows this launch processes: [t_begin, t_end)
+  int n_mblk;                  // row blocks of the kernel's tile height over [t_begin, t_end)
   int kblk_per_rank;           // ceil(Kp / 64)
   int last_k16;                // 16-wide K steps in the last k-block of a rank (1..4)
   int nS, nPriv;               // n-blocks that have a shared unit / private units
@@ -226,7 +227,7 @@ __device__ __forceinline__ void k1_put_partial(const RowparParams& prm, int rank
 // [h0, h1) of the tile, each half's 16 residual pieces loaded up front.
 __device__ __forceinline__ void k1_epilogue_private(uint32_t trow, const RowparParams& prm, int row, int rank,
                                                     int n0, int slot, bool mixed, int h0, int h1) {
-  const bool row_ok = row < prm.T;
+  const bool row_ok = row < prm.t_end;
   const size_t rowoff = (static_cast<size_t>(rank) * prm.T + (row_ok ? row : 0)) * prm.H;
   const __nv_bfloat16* Rp = prm.R + rowoff + n0;
   __nv_bfloat16* Op = prm.Hout + rowoff + n0;
@@ -270,7 +271,7 @@ __device__ __forceinline__ void k1_epilogue_private(uint32_t trow, const RowparP
 __device__ __forceinline__ void k1_epilogue_shared(uint32_t trow, const RowparParams& prm, int row, int n0,
                                                    int slot, bool mixed, int c0, int c1) {
   constexpr int RG = 4;
-  const bool row_ok = row < prm.T;
+  const bool row_ok = row < prm.t_end;
   const size_t rstride = static_cast<size_t>(prm.T) * prm.H;
   const size_t base = static_cast<size_t>(row_ok ? row : 0) * prm.H + n0;
   const int ncols = min(256, prm.H - n0);
@@ -381,7 +382,7 @@ __device__ __forceinline__ bool k1_epilogue_tma(uint32_t trow, const RowparParam
       bulk_commit_group();
     }
     if (prm.fuse_norm && c == nch - 1) {  // this rank's row segment is complete
-      if (row < prm.T) k1_put_partial(prm, r, row, slot, ss);
+      if (row < prm.t_end) k1_put_partial(prm, r, row, slot, ss);
       ss = 0.f;
     }
     const int nx = i + K1_EPI_NBUF;

@@ -125,7 +125,7 @@ __global__ void __launch_bounds__(K1Threads<kFused>::value, 1)
           for (int kb = 0; kb < prm.kblk_per_rank; ++kb) {
             if (!mbar_wait(&empty[stage], phase ^ 1, tmo, 2)) { ok = false; break; }
             mbar_arrive_expect_tx(&full[stage], K1_A_BYTES + K1_B_BYTES);
-            tma_load_3d(sA + stage * K1_A_BYTES, &tmX, &full[stage], kb * K1_BK, un.m * K1_BM, r, pol_x);
+            tma_load_3d(sA + stage * K1_A_BYTES, &tmX, &full[stage], kb * K1_BK, prm.t_begin + un.m * K1_BM, r, pol_x);
             tma_load_3d(sB + stage * K1_B_BYTES, &tmW, &full[stage], kb * K1_BK, un.n * K1_BN, r, pol_w);
             issued_mask |= 1u << stage;
             last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
@@ -218,11 +218,11 @@ __global__ void __launch_bounds__(K1Threads<kFused>::value, 1)
       if (!ok) break;
       tc_fence_after();
       const uint32_t trow = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * K1_BN);
-      const int row = un.m * K1_BM + q * 32 + lane;
+      const int row = prm.t_begin + un.m * K1_BM + q * 32 + lane;
       const int n0 = un.n * K1_BN;
       const bool mixed = prm.ncls[un.n] == 2;
       if (!mixed) {
-        const int row0 = un.m * K1_BM + q * 32;
+        const int row0 = prm.t_begin + un.m * K1_BM + q * 32;
         if (!k1_epilogue_tma(trow, prm, &tmR, &tmH, row0, n0, un.rank, un.slot, my_bufs, my_rbar, rphase, lane,
                              pol_r))
           break;

@@ -126,7 +126,7 @@ __global__ void __launch_bounds__(K1Threads<kFused>::value, 1)
         const K1Unit un = k1_decode(u, prm);
         const int r0 = un.rank < 0 ? 0 : un.rank;
         const int r1 = un.rank < 0 ? prm.P : un.rank + 1;
-        const int xrow = un.m * (2 * K2P_BM) + static_cast<int>(cta) * K2P_BM;
+        const int xrow = prm.t_begin + un.m * (2 * K2P_BM) + static_cast<int>(cta) * K2P_BM;
         const int wrow = un.n * K2P_BN + static_cast<int>(cta) * (K2P_BN / 2);
         for (int r = r0; r < r1 && ok; ++r) {
           for (int kb = 0; kb < prm.kblk_per_rank; ++kb) {
@@ -222,11 +222,11 @@ __global__ void __launch_bounds__(K1Threads<kFused>::value, 1)
       if (!ok) break;
       tc_fence_after();
       const uint32_t trow = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * K2P_BN);
-      const int row = un.m * (2 * K2P_BM) + static_cast<int>(cta) * K2P_BM + q * 32 + lane;
+      const int row = prm.t_begin + un.m * (2 * K2P_BM) + static_cast<int>(cta) * K2P_BM + q * 32 + lane;
       const int n0 = un.n * K2P_BN;
       const bool mixed = prm.ncls[un.n] == 2;
       if (!mixed) {
-        const int row0 = un.m * (2 * K2P_BM) + static_cast<int>(cta) * K2P_BM + q * 32;
+        const int row0 = prm.t_begin + un.m * (2 * K2P_BM) + static_cast<int>(cta) * K2P_BM + q * 32;
         if (!k1_epilogue_tma(trow, prm, &tmR, &tmH, row0, n0, un.rank, un.slot, my_bufs, my_rbar, rphase, lane,
                              pol_r))
           break;

@@ -209,3 +209,15 @@ def test_host_buffer_entry_matches_device_entry(T):
         assert C.caat_get_device_status() == 0
         assert torch.equal(hout, out_dev)
         assert torch.equal(hh, h_dev)
+
+
+def test_overlapped_norm_chunks_match():
+    """CAAT_FLAG_OVERLAP_NORM (GEMM in 2048-token launches, each launch's row norm on a side
+    stream) gives the same bits as the single launch, and matches the oracle."""
+    T, K, H, P = 4352, 512, 776, 2
+    d = I.make_rowpar_inputs(T, K, H, P, seed=18, x_std=1.0, w_std=0.05, r_std=1.0, gamma="uniform")
+    o1, h1 = run_rowpar(d, P, 0.5)
+    o2, h2 = run_rowpar(d, P, 0.5, flags=C.CAAT_FLAG_OVERLAP_NORM)
+    assert torch.equal(o1, o2) and torch.equal(h1, h2)
+    ref = O.rowpar_forward(d["X"], d["W"], d["R"], d["gamma"], P, 0.5)
+    assert_out_close(o2, ref, "overlap")
