@@ -143,7 +143,6 @@ __global__ void __launch_bounds__(K4_THREADS, 1)
         const uint32_t dt = tmem_base + static_cast<uint32_t>(buf * K4_MAXN);
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&full[stage], phase, tmo, 63)) { ok = false; break; }
-          tc_fence_after();
           const int nk16 = (kb == prm.kblk - 1) ? prm.last_k16 : (K4_BK / 16);
           const uint32_t a_addr = smem_u32(sA + stage * K4_A_BYTES);
           const uint32_t b_addr = smem_u32(sB + stage * K4_B_BYTES);

@@ -177,7 +177,6 @@ __global__ void __launch_bounds__(K3_THREADS, 1)
         const uint32_t dt = tmem_base + static_cast<uint32_t>(buf * 2 * K3_BN);
         for (int j = 0; j < prm.kblk; ++j) {
           if (!mbar_wait(&full[stage], phase, tmo, 46)) { ok = false; break; }
-          tc_fence_after();
           const int nk16 = (j == prm.kblk - 1) ? prm.last_k16 : (K3_BK / 16);
           const uint32_t a_addr = smem_u32(sA + stage * K3_A_BYTES);
           const uint32_t b_addr = smem_u32(sB + stage * K3_B_BYTES);

@@ -167,7 +167,6 @@ __global__ void __launch_bounds__(K1Threads<kFused>::value, 1)
         int kb_in_rank = 0;
         for (int j = 0; j < nkb; ++j) {
           if (!mbar_wait(&full[stage], phase, tmo, 26)) { ok = false; break; }
-          tc_fence_after();
           const int nk16 = (kb_in_rank == prm.kblk_per_rank - 1) ? prm.last_k16 : (K2P_BK / 16);
           const uint32_t a_addr = smem_u32(sA + stage * K2P_A_BYTES);
           const uint32_t b_addr = smem_u32(sB + stage * K2P_B_BYTES);
