@@ -171,16 +171,20 @@ def cpu_baseline(T, K, H, P, p, sync_idx, target_s=10.0, seed=0):
     d = I.make_rowpar_inputs(min(T, 2048), K, H, P, seed=seed)
     flops_per_row = 2.0 * K * H
     t_total, rows_done = 0.0, 0
+    t_rows = d["X"].shape[1]
+    start = 0
     while True:
-        rows = np.arange(min(n_rows, d["X"].shape[1]))
+        # consecutive rows of the generated sample, wrapping around it
+        rows = (start + np.arange(min(n_rows, t_rows))) % t_rows
         t0 = time.perf_counter()
         O.rowpar_rows(d["X"], d["W"], d["R"], d["gamma"], P, p, rows, sync_idx)
         dt = time.perf_counter() - t0
         t_total += dt
         rows_done += len(rows)
-        if t_total >= target_s or len(rows) >= d["X"].shape[1]:
+        start = (start + len(rows)) % t_rows
+        if t_total >= target_s:
             break
-        n_rows = int(min(d["X"].shape[1], max(2 * n_rows, n_rows * (target_s - t_total) / max(dt, 1e-3))))
+        n_rows = int(max(16, min(2 * n_rows, len(rows) * (target_s - t_total) / max(dt, 1e-3))))
     tflops = flops_per_row * rows_done / t_total / 1e12
     return {"value": tflops, "unit": "TFLOP/s", "cores": int(threads), "kind": "oracle",
             "sample": f"{rows_done} token rows (all {P} ranks, full H={H}, K={K}) of the workload, "

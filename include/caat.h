@@ -82,6 +82,9 @@ typedef enum caat_status {
 #define CAAT_FLAG_OVERLAP_NORM 0x20u     /* T >= 4096: run the GEMM in 2048-token launches and the
                                             row norm of each launch's tokens on a library-owned
                                             side stream, overlapping the next launch */
+#define CAAT_FLAG_ORDER_GROUPED 0x40u    /* schedule the GEMM tiles in groups of row blocks
+                                            (shared tiles of the group, then its private tiles
+                                            rank by rank); the fused norm always does */
 #define CAAT_FLAG_SINGLE_CTA 0x4u        /* use the single-CTA GEMM kernel (128-token tiles)
                                             instead of the CTA-pair kernel (256-token tiles) */
 #define CAAT_FLAG_TEST_STALL 0x100u      /* test hook: the GEMM kernel's MMA warp never signals

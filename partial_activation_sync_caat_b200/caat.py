@@ -33,6 +33,7 @@ CAAT_FLAG_SINGLE_CTA = 0x4
 CAAT_FLAG_FUSED_NORM = 0x8
 CAAT_FLAG_ORDER_ROWBLOCK = 0x10
 CAAT_FLAG_OVERLAP_NORM = 0x20
+CAAT_FLAG_ORDER_GROUPED = 0x40
 CAAT_FLAG_TEST_STALL = 0x100
 
 CAAT_NOALLOC_SCRATCH_BYTES = 1048576

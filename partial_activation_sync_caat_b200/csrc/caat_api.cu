@@ -208,12 +208,16 @@ constexpr size_t kCounterBytes = 256;
 
 size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
 
-// Workspace of the row-parallel layer: [counters (256 B) | rb_count[n_rb] | job_slots[n_rb] |
-// ss_part[P][T_pad][nslots_max] floats].  The counter region (first `zeroed` bytes) is cleared
-// on the stream before every launch; ss_part needs no clearing (every slot of every valid row
-// is written once).  Sized for the larger of the two GEMM kernels' row blocking.
+// Workspace of the row-parallel layer.  Fused norm: [counters (256 B) | rb_count[n_rb] |
+// job_slots[n_rb] | ss_part[P][T_pad][nslots_max] floats]; the counter region (first `zeroed`
+// bytes) is cleared on the stream before every launch; ss_part needs no clearing (every slot
+// of every valid row is written once).  Separate norm: [counters (256 B) | sdone], where the
+// optional sdone flags ([T_pad/32][n-blocks] u32, cleared before the launch when used) let
+// the CTA-pair kernel give mixed column blocks the TMA epilogue; with a workspace of only
+// the 256 B (`min_total`) those blocks take the register epilogue.  Sized for the larger of
+// the two GEMM kernels' row blocking.
 struct RowparWs {
-  size_t rb_count, job_slots, ss_part, zeroed, total;
+  size_t rb_count, job_slots, ss_part, zeroed, total, min_total, sdone, sdone_bytes;
   int64_t T_pad, n_rb, nslots_max;
 };
 
@@ -222,12 +226,20 @@ RowparWs rowpar_ws_layout(int64_t T, int64_t H, int P, bool fused) {
   L.T_pad = (T + 255) / 256 * 256;
   L.n_rb = (L.T_pad / 128) * P;
   L.nslots_max = 2 * ((H + 255) / 256);
-  L.rb_count = kCounterBytes;
-  L.job_slots = L.rb_count + size_t(L.n_rb) * 4;
-  L.zeroed = L.job_slots + size_t(L.n_rb) * 4;
-  L.ss_part = align256(L.zeroed);
-  L.total = fused ? L.ss_part + align256(size_t(P) * L.T_pad * L.nslots_max * 4) : kCounterBytes;
-  if (!fused) L.zeroed = kCounterBytes;
+  if (fused) {
+    L.rb_count = kCounterBytes;
+    L.job_slots = L.rb_count + size_t(L.n_rb) * 4;
+    L.zeroed = L.job_slots + size_t(L.n_rb) * 4;
+    L.ss_part = align256(L.zeroed);
+    L.total = L.ss_part + align256(size_t(P) * L.T_pad * L.nslots_max * 4);
+    L.min_total = L.total;
+  } else {
+    L.zeroed = kCounterBytes;
+    L.sdone = kCounterBytes;
+    L.sdone_bytes = size_t(L.T_pad / 32) * size_t((H + 255) / 256) * 4;
+    L.total = L.sdone + align256(L.sdone_bytes);
+    L.min_total = kCounterBytes;
+  }
   return L;
 }
 
@@ -243,9 +255,12 @@ size_t decode_workspace(int64_t T, int64_t H, int P) {
   return kCounterBytes + align256(size_t(decode_splits(T)) * P * T * H * 4);
 }
 
-size_t rowpar_workspace(int64_t T, int64_t K, int64_t H, int P, bool fused = true) {
+// Workspace a call needs at least (`fused`: with the fused norm), or, with full = true, the size
+// that also enables every fast path (the value caat_workspace_size reports).
+size_t rowpar_workspace(int64_t T, int64_t K, int64_t H, int P, bool fused = true, bool full = true) {
   (void)K;
-  size_t n = rowpar_ws_layout(T, H, P, fused).total;
+  size_t n = full ? std::max(rowpar_ws_layout(T, H, P, true).total, rowpar_ws_layout(T, H, P, false).total)
+                  : rowpar_ws_layout(T, H, P, fused).min_total;
   if (decode_eligible(T, P, H)) n = std::max(n, decode_workspace(T, H, P));
   return n;
 }
@@ -462,13 +477,13 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
   prm.counter = counter;
   prm.piece_claim = counter + 1;
   prm.job_pub = counter + 2;
-  prm.rb_count = reinterpret_cast<unsigned int*>(wsb + wl.rb_count);
-  prm.job_slots = reinterpret_cast<unsigned int*>(wsb + wl.job_slots);
-  prm.ss_part = reinterpret_cast<float*>(wsb + wl.ss_part);
+  prm.rb_count = fused ? reinterpret_cast<unsigned int*>(wsb + wl.rb_count) : nullptr;
+  prm.job_slots = fused ? reinterpret_cast<unsigned int*>(wsb + wl.job_slots) : nullptr;
+  prm.ss_part = fused ? reinterpret_cast<float*>(wsb + wl.ss_part) : nullptr;
   prm.fuse_norm = fused ? 1 : 0;
   // Tile order: the fused norm wants row blocks to complete throughout the kernel (grouped
   // order); otherwise shared tiles first, then private tiles rank by rank.
-  prm.order = (a->flags & CAAT_FLAG_ORDER_ROWBLOCK) ? 1 : (fused ? 2 : 0);
+  prm.order = (a->flags & CAAT_FLAG_ORDER_ROWBLOCK) ? 1 : ((fused || (a->flags & CAAT_FLAG_ORDER_GROUPED)) ? 2 : 0);
   prm.group_m = group_m_setting();
   prm.eps = a->eps;
   prm.T = static_cast<int>(T);
@@ -501,6 +516,14 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
   if ((T + bm - 1) / bm * (prm.nS + int64_t(P) * prm.nPriv) > INT32_MAX / 2) return CAAT_ERR_UNSUPPORTED;
   prm.T_pad = static_cast<int>((T + bm - 1) / bm * bm);
   prm.n_rb = static_cast<int>(prm.T_pad / 128 * P);
+  // Mixed column blocks on the pair kernel: TMA epilogue behind per-32-row completion flags of
+  // their shared tiles, when the workspace holds the flags.
+  bool any_mixed = false;
+  for (int nb = 0; nb < nblk; ++nb) any_mixed |= prm.ncls[nb] == 2;
+  const bool merge = pair && !fused && any_mixed && a->ws_bytes >= wl.total;
+  prm.merge_mixed = merge ? 1 : 0;
+  prm.sdone = merge ? reinterpret_cast<unsigned int*>(wsb + wl.sdone) : nullptr;
+  const size_t zero_bytes = merge ? wl.sdone + wl.sdone_bytes : wl.zeroed;
 
   CUtensorMap tmX, tmW, tmR, tmH;
   caat_status s = make_map_3d(&tmX, a->X, Kp, T, P, caat::K1_BK, caat::K1_BM);
@@ -520,7 +543,7 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
     prm.n_mblk = static_cast<int>((tc + bm - 1) / bm);
     const int64_t units = int64_t(prm.n_mblk) * (prm.nS + int64_t(P) * prm.nPriv);
     prm.n_units = static_cast<int>(units);
-    if (cudaMemsetAsync(counter, 0, wl.zeroed, st) != cudaSuccess) return CAAT_ERR_CUDA;
+    if (cudaMemsetAsync(counter, 0, zero_bytes, st) != cudaSuccess) return CAAT_ERR_CUDA;
     if (pair) {
       const int pairs = static_cast<int>(std::min<int64_t>(dev->max_pairs, units));
       cudaLaunchConfig_t cfg = {};
@@ -608,7 +631,7 @@ caat_status validate_rowpar(const caat_rowpar_args* a, std::vector<uint8_t>& mas
   if (!aligned16(a->X) || !aligned16(a->W) || !aligned16(a->residual) || !aligned16(a->gamma) ||
       !aligned16(a->out) || (a->h_out && !aligned16(a->h_out)))
     return CAAT_ERR_UNSUPPORTED;
-  const size_t need = rowpar_workspace(a->T, a->K, a->H, a->P, (a->flags & CAAT_FLAG_FUSED_NORM) != 0);
+  const size_t need = rowpar_workspace(a->T, a->K, a->H, a->P, (a->flags & CAAT_FLAG_FUSED_NORM) != 0, false);
   if (need > 0) {
     if (!a->workspace || a->ws_bytes < need || (reinterpret_cast<uintptr_t>(a->workspace) & 255u))
       return CAAT_ERR_WORKSPACE;
@@ -803,9 +826,10 @@ caat_status caat_rowpar_forward_noalloc(const caat_rowpar_args* a) {
   // The fused RMSNorm needs scratch that grows with T; when it does not fit the built-in
   // array, the norm runs as the separate row kernel, which needs only the unit counter.
   if ((d.flags & CAAT_FLAG_FUSED_NORM) &&
-      rowpar_workspace(d.T, d.K, d.H, d.P, true) > CAAT_NOALLOC_SCRATCH_BYTES)
+      rowpar_workspace(d.T, d.K, d.H, d.P, true, false) > CAAT_NOALLOC_SCRATCH_BYTES)
     d.flags &= ~CAAT_FLAG_FUSED_NORM;
-  if (rowpar_workspace(d.T, d.K, d.H, d.P, (d.flags & CAAT_FLAG_FUSED_NORM) != 0) > CAAT_NOALLOC_SCRATCH_BYTES)
+  if (rowpar_workspace(d.T, d.K, d.H, d.P, (d.flags & CAAT_FLAG_FUSED_NORM) != 0, false) >
+      CAAT_NOALLOC_SCRATCH_BYTES)
     return CAAT_ERR_WORKSPACE;
   void* scratch = nullptr;
   s = noalloc_scratch(&scratch);

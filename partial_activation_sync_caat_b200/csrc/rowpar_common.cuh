@@ -56,6 +56,8 @@ struct RowparParams {
   unsigned int* rb_count;      // [n_rb] tiles done per (row block, rank), zero at launch
   unsigned int* job_slots;     // [n_rb] published row-block ids + 1, zero at launch
   float* ss_part;              // [P][T_pad][nslots] per-row sum-of-squares partials
+  unsigned int* sdone;         // [T_pad/32][n-blocks] shared unit of a mixed block stored, zero at launch
+  int merge_mixed;             // 1: mixed blocks use the TMA epilogue (see k1_epilogue_tma)
   int T, H, Kp, P;             // T: token rows of the tensors (the row stride of rank blocks)
   int t_begin, t_end;          // token rows this launch processes: [t_begin, t_end)
   int n_mblk;                  // row blocks of the kernel's tile height over [t_begin, t_end)
@@ -326,9 +328,64 @@ __device__ __forceinline__ void k1_epilogue_shared(uint32_t trow, const RowparPa
 // by TMA.  Full 128-byte lines move in bulk; rows beyond T and columns beyond H are
 // zero-filled on load and clipped on store by the tensor maps.  Items are pipelined over
 // K1_EPI_NBUF buffers.  Returns false if a wait ran out.
+// Mixed column blocks (merge = true, private units only): the shared unit of the block has
+// already stored full boxes of h whose shared columns are final; the private unit loads that
+// h box together with the residual box, keeps the shared columns, writes its private columns
+// and stores the full box again (single-buffered).
 __device__ __forceinline__ bool k1_epilogue_tma(uint32_t trow, const RowparParams& prm, const void* tmR,
                                                 const void* tmH, int row0, int n0, int rank, int slot, uint8_t* bufs,
-                                                uint64_t* rbar, uint32_t& phase, int lane, uint64_t pol_r) {
+                                                uint64_t* rbar, uint32_t& phase, int lane, uint64_t pol_r,
+                                                bool merge = false) {
+  if (merge) {
+    const int nch = min(4, (prm.H - n0 + 63) / 64);
+    const float scale = prm.private_scale;
+    for (int c = 0; c < nch; ++c) {
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&rbar[0], 2 * K1_EPI_BOX_BYTES);
+        tma_load_3d(bufs, tmR, &rbar[0], n0 + 64 * c, row0, rank, pol_r);
+        tma_load_3d(bufs + K1_EPI_BOX_BYTES, tmH, &rbar[0], n0 + 64 * c, row0, rank, pol_r);
+      }
+      uint32_t v[64];
+      __syncwarp();
+      tmem_ld_32x32b_x32(trow + 64 * c, *reinterpret_cast<uint32_t(*)[32]>(v));
+      tmem_ld_32x32b_x32(trow + 64 * c + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+      tmem_wait_ld();
+      const bool ok = mbar_wait(&rbar[0], phase & 1u, prm.timeout_ns, 33);
+      phase ^= 1u;
+      if (!__all_sync(0xFFFFFFFFu, ok)) return false;
+      uint8_t* rrow = bufs + lane * 128;
+      uint8_t* hrow = bufs + K1_EPI_BOX_BYTES + lane * 128;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int col = n0 + 64 * c + 8 * j;
+        const uint32_t bits = (prm.mask_bits[col >> 5] >> (col & 31)) & 0xFFu;
+        const int g = (j ^ (lane & 7)) << 4;
+        const uint4 rr = *reinterpret_cast<const uint4*>(rrow + g);
+        const uint4 hh = *reinterpret_cast<const uint4*>(hrow + g);
+        const uint32_t rw[4] = {rr.x, rr.y, rr.z, rr.w};
+        const uint32_t hw[4] = {hh.x, hh.y, hh.z, hh.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t priv = pack_bf16x2(__uint_as_float(v[8 * j + 2 * e]) * scale + bf16lo(rw[e]),
+                                            __uint_as_float(v[8 * j + 2 * e + 1]) * scale + bf16hi(rw[e]));
+          const uint32_t keep = (((bits >> (2 * e)) & 1u) ? 0x0000FFFFu : 0u) |
+                                (((bits >> (2 * e + 1)) & 1u) ? 0xFFFF0000u : 0u);
+          o[e] = (hw[e] & keep) | (priv & ~keep);
+        }
+        *reinterpret_cast<uint4*>(hrow + g) = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_3d(tmH, bufs + K1_EPI_BOX_BYTES, n0 + 64 * c, row0, rank);
+        bulk_commit_group();
+        bulk_wait_group_read0();  // both boxes are reused by the next chunk
+      }
+      __syncwarp();
+    }
+    return true;
+  }
   const int nch = min(4, (prm.H - n0 + 63) / 64);
   const int nr = rank < 0 ? prm.P : 1;
   const int n_items = nch * nr;  // rank-major: item i = (rank i / nch, chunk i % nch)
@@ -409,6 +466,40 @@ __device__ __forceinline__ bool k1_epilogue_tma(uint32_t trow, const RowparParam
   }
   __syncwarp();
   return true;
+}
+
+// Shared unit of a mixed block, after its TMA epilogue (one epilogue warp, 32 rows): complete
+// the warp's box stores, make them visible to the async proxy of other CTAs, and mark the
+// 32-row group's column block as stored.
+__device__ __forceinline__ void k1_signal_sdone(unsigned int* flag) {
+  if ((threadIdx.x & 31) == 0) {
+    bulk_wait_group0();
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    __threadfence();
+    st_release_gpu(flag, 1u);
+  }
+  __syncwarp();
+}
+
+// Private unit of a mixed block: wait (bounded) until the block's shared unit has stored its
+// boxes; returns false if the wait ran out.  Lane 0 polls, the warp follows.
+__device__ __forceinline__ bool k1_wait_sdone(const RowparParams& prm, const unsigned int* flag) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) {
+    if (ld_acquire_gpu(flag) == 0u) {
+      const uint64_t t0 = globaltimer_ns();
+      while (ld_acquire_gpu(flag) == 0u) {
+        __nanosleep(500);
+        if (status_poll() != 0 || globaltimer_ns() - t0 > prm.timeout_ns) {
+          if (status_poll() == 0) status_raise(4, 35);
+          ok = 0;
+          break;
+        }
+      }
+    }
+    asm volatile("fence.proxy.async.global;" ::: "memory");  // the TMA loads that follow see the boxes
+  }
+  return __shfl_sync(0xFFFFFFFFu, ok, 0) != 0;
 }
 
 // After a tile's epilogue (all 128 epilogue threads): make its h and partials visible, count

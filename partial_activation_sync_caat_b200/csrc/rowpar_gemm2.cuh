@@ -224,11 +224,19 @@ __global__ void __launch_bounds__(K1Threads<kFused>::value, 1)
       const int row = prm.t_begin + un.m * (2 * K2P_BM) + static_cast<int>(cta) * K2P_BM + q * 32 + lane;
       const int n0 = un.n * K2P_BN;
       const bool mixed = prm.ncls[un.n] == 2;
-      if (!mixed) {
+      const bool merge = mixed && !kFused && prm.merge_mixed;
+      if (!mixed || merge) {
         const int row0 = prm.t_begin + un.m * (2 * K2P_BM) + static_cast<int>(cta) * K2P_BM + q * 32;
+        // flag of this warp's 32 rows in column block n: [row group][n-block]
+        unsigned int* flag =
+            merge ? prm.sdone + (static_cast<size_t>((row0 - prm.t_begin) >> 5) * ((prm.H + K2P_BN - 1) / K2P_BN) +
+                                 un.n)
+                  : nullptr;
+        if (merge && un.rank >= 0 && !k1_wait_sdone(prm, flag)) break;
         if (!k1_epilogue_tma(trow, prm, &tmR, &tmH, row0, n0, un.rank, un.slot, my_bufs, my_rbar, rphase, lane,
-                             pol_r))
+                             pol_r, merge && un.rank >= 0))
           break;
+        if (merge && un.rank < 0) k1_signal_sdone(flag);
       } else if (un.rank < 0) {
         k1_epilogue_shared(trow, prm, row, n0, un.slot, mixed, 0, 8);
       } else {

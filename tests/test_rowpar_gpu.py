@@ -93,7 +93,7 @@ def test_single_cta_random_sync_idx():
     _compare(d, 4, 0.5, idx, flags=C.CAAT_FLAG_SINGLE_CTA, what="single-CTA random S")
 
 
-@pytest.mark.parametrize("flags", [C.CAAT_FLAG_FUSED_NORM, C.CAAT_FLAG_ORDER_ROWBLOCK,
+@pytest.mark.parametrize("flags", [C.CAAT_FLAG_FUSED_NORM, C.CAAT_FLAG_ORDER_ROWBLOCK, C.CAAT_FLAG_ORDER_GROUPED,
                                    C.CAAT_FLAG_FUSED_NORM | C.CAAT_FLAG_SINGLE_CTA,
                                    C.CAAT_FLAG_ORDER_ROWBLOCK | C.CAAT_FLAG_SINGLE_CTA])
 @pytest.mark.parametrize("p", [0.5, 0.7])
@@ -221,3 +221,32 @@ def test_overlapped_norm_chunks_match():
     assert torch.equal(o1, o2) and torch.equal(h1, h2)
     ref = O.rowpar_forward(d["X"], d["W"], d["R"], d["gamma"], P, 0.5)
     assert_out_close(o2, ref, "overlap")
+
+
+# ------------------------------------------------------------------ mixed column blocks
+@pytest.mark.parametrize("p,random_idx", [(0.3, True), (0.703125, False), (0.5, True)])
+def test_mixed_block_tma_merge_matches_register_epilogue(p, random_idx):
+    """Column blocks holding shared and private channels: with the full workspace the CTA-pair
+    kernel stores them with TMA boxes (the private unit merges its channels into the boxes its
+    shared unit stored first, behind per-row-group flags); with only the 256-byte minimum
+    workspace they take the register epilogue.  Same bits either way, and both match the
+    oracle.  T = 600: three 256-token row blocks, the last one ragged."""
+    T, K, H, P = 600, 1024, 1288, 4
+    d = I.make_rowpar_inputs(T, K, H, P, seed=21, x_std=1.0, w_std=0.05, r_std=1.0, gamma="uniform")
+    idx = I.random_sync_idx(H, O.n_sync(H, p), seed=5) if random_idx else None
+    g = to_dev(d)
+    res = []
+    for ws_bytes in (C.caat_workspace_size(T, K, H, P, C.CAAT_VARIANT_ROWPAR), 256):
+        ws = C.alloc_workspace(ws_bytes)
+        out = torch.empty_like(g["R"])
+        hb = torch.empty_like(g["R"])
+        C.caat_rowpar_forward(g["X"], g["W"], g["R"], g["gamma"], idx, P, p, out, h_out=hb, workspace=ws,
+                              private_scale=0.75)
+        torch.cuda.synchronize()
+        assert C.caat_get_device_status() == 0
+        res.append((out.cpu(), hb.cpu()))
+    assert torch.equal(res[0][1], res[1][1]) and torch.equal(res[0][0], res[1][0])
+    r = O.rowpar_forward(d["X"], d["W"], d["R"], d["gamma"], P, p, sync_idx=idx, private_scale=0.75,
+                         return_all=True)
+    assert_h_close(res[0][1], r["h"], "h merged")
+    assert_out_close(res[0][0], r["out"], "out merged")
