@@ -580,8 +580,19 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
     const int64_t rows = int64_t(P) * tc;
     const int64_t warps_per_block = caat::K2_THREADS / 32;
     const int64_t blocks = std::min<int64_t>((rows + warps_per_block - 1) / warps_per_block, max_blocks);
-    caat::rownorm_kernel<<<blocks, caat::K2_THREADS, 0, ns>>>(hdst, o, g, P, T, t0, tc, static_cast<int>(H),
-                                                              a->eps);
+    if (H <= 4096) {
+      // row held in registers: VPL 128-bit vectors per lane
+      const int64_t rb = std::min<int64_t>((rows + warps_per_block - 1) / warps_per_block, int64_t(dev->sm_count) * 2);
+      if (H <= 1024)
+        caat::rownorm_reg_kernel<4><<<rb, caat::K2_THREADS, 0, ns>>>(hdst, o, g, P, T, t0, tc, static_cast<int>(H), a->eps);
+      else if (H <= 2048)
+        caat::rownorm_reg_kernel<8><<<rb, caat::K2_THREADS, 0, ns>>>(hdst, o, g, P, T, t0, tc, static_cast<int>(H), a->eps);
+      else
+        caat::rownorm_reg_kernel<16><<<rb, caat::K2_THREADS, 0, ns>>>(hdst, o, g, P, T, t0, tc, static_cast<int>(H), a->eps);
+    } else {
+      caat::rownorm_kernel<<<blocks, caat::K2_THREADS, 0, ns>>>(hdst, o, g, P, T, t0, tc, static_cast<int>(H),
+                                                                a->eps);
+    }
     return cudaGetLastError() == cudaSuccess ? CAAT_OK : CAAT_ERR_CUDA;
   };
 

@@ -106,6 +106,16 @@ __device__ __forceinline__ void tma_store_3d(const void* map, const void* smem_s
                : "memory");
 }
 
+// Tile store with an L2 eviction-priority hint for the written lines.
+__device__ __forceinline__ void tma_store_3d(const void* map, const void* smem_src, int c0, int c1, int c2,
+                                             uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group.L2::cache_hint [%0, {%2, %3, %4}], [%1], %5;" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(smem_u32(smem_src)), "r"(c0), "r"(c1), "r"(c2), "l"(policy)
+      : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 
 // Waits until every committed bulk store of this thread has finished reading shared memory.

@@ -335,7 +335,7 @@ __device__ __forceinline__ void k1_epilogue_shared(uint32_t trow, const RowparPa
 __device__ __forceinline__ bool k1_epilogue_tma(uint32_t trow, const RowparParams& prm, const void* tmR,
                                                 const void* tmH, int row0, int n0, int rank, int slot, uint8_t* bufs,
                                                 uint64_t* rbar, uint32_t& phase, int lane, uint64_t pol_r,
-                                                bool merge = false) {
+                                                uint64_t pol_h, bool merge = false) {
   if (merge) {
     const int nch = min(4, (prm.H - n0 + 63) / 64);
     const float scale = prm.private_scale;
@@ -378,7 +378,7 @@ __device__ __forceinline__ bool k1_epilogue_tma(uint32_t trow, const RowparParam
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
-        tma_store_3d(tmH, bufs + K1_EPI_BOX_BYTES, n0 + 64 * c, row0, rank);
+        tma_store_3d(tmH, bufs + K1_EPI_BOX_BYTES, n0 + 64 * c, row0, rank, pol_h);
         bulk_commit_group();
         bulk_wait_group_read0();  // both boxes are reused by the next chunk
       }
@@ -435,7 +435,7 @@ __device__ __forceinline__ bool k1_epilogue_tma(uint32_t trow, const RowparParam
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
-      tma_store_3d(tmH, bufs + b * K1_EPI_BOX_BYTES, n0 + 64 * c, row0, r);
+      tma_store_3d(tmH, bufs + b * K1_EPI_BOX_BYTES, n0 + 64 * c, row0, r, pol_h);
       bulk_commit_group();
     }
     if (prm.fuse_norm && c == nch - 1) {  // this rank's row segment is complete

@@ -193,6 +193,7 @@ __global__ void __launch_bounds__(K1Threads<kFused>::value, 1)
     uint64_t* my_rbar = rbar + (warp - 2) * K1_EPI_NBUF;
     uint32_t rphase = 0;
     const uint64_t pol_r = policy_evict_first();
+    const uint64_t pol_h = kFused ? policy_evict_normal() : policy_evict_first();
     int local = 0;
     for (int i = 0;; ++i) {
       const int slot = i % K1_SCHED;
@@ -223,7 +224,7 @@ __global__ void __launch_bounds__(K1Threads<kFused>::value, 1)
       if (!mixed) {
         const int row0 = prm.t_begin + un.m * K1_BM + q * 32;
         if (!k1_epilogue_tma(trow, prm, &tmR, &tmH, row0, n0, un.rank, un.slot, my_bufs, my_rbar, rphase, lane,
-                             pol_r))
+                             pol_r, pol_h))
           break;
       } else if (un.rank < 0) {
         k1_epilogue_shared(trow, prm, row, n0, un.slot, mixed, 0, 8);

@@ -101,7 +101,7 @@ __global__ void __launch_bounds__(K1Threads<kFused>::value, 1)
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producers
     if (lane == 0) {
-      const uint64_t pol_x = policy_evict_normal();
+      const uint64_t pol_x = policy_evict_last();
       const uint64_t pol_w = policy_evict_last();
       int stage = 0;
       uint32_t phase = 0;
@@ -195,6 +195,8 @@ __global__ void __launch_bounds__(K1Threads<kFused>::value, 1)
     uint64_t* my_rbar = rbar + (warp - 2) * K1_EPI_NBUF;
     uint32_t rphase = 0;
     const uint64_t pol_r = policy_evict_first();
+    // h is read back by the fused norm (from L2); otherwise streamed out, behind X and W
+    const uint64_t pol_h = kFused ? policy_evict_normal() : policy_evict_first();
     const uint32_t tempty_leader[2] = {mapa_shared(smem_u32(&tempty[0]), 0), mapa_shared(smem_u32(&tempty[1]), 0)};
     int local = 0;
     for (int i = 0;; ++i) {
@@ -234,7 +236,7 @@ __global__ void __launch_bounds__(K1Threads<kFused>::value, 1)
                   : nullptr;
         if (merge && un.rank >= 0 && !k1_wait_sdone(prm, flag)) break;
         if (!k1_epilogue_tma(trow, prm, &tmR, &tmH, row0, n0, un.rank, un.slot, my_bufs, my_rbar, rphase, lane,
-                             pol_r, merge && un.rank >= 0))
+                             pol_r, pol_h, merge && un.rank >= 0))
           break;
         if (merge && un.rank < 0) k1_signal_sdone(flag);
       } else if (un.rank < 0) {
