@@ -113,6 +113,16 @@ def recorded_traffic(workload: str, kernel: str):
     return None if e is None else int(e["read_bytes"] + e["write_bytes"])
 
 
+L2_BYTES = 126 * 1024 * 1024
+
+
+def alg_bytes_of(T, K, H, P, mlp=False):
+    """Bytes one step must move at least: X, W, residual in, h and out (bf16)."""
+    if mlp:   # K is the FFN size F: X [P,T,H/P], A [P,2F/P,H], Y, W2 [P,H,F/P], R, out
+        return 2.0 * (T * H + 2 * K * H + 2 * T * K + K * H + 2 * P * T * H)
+    return 2.0 * (T * K + H * K + 2 * P * T * H + H)
+
+
 def workload_desc(name, T, K, H, P, p, rand):
     return (f"{name}: partially synced row-parallel FC2 + residual + RMSNorm, T={T} H={H} K={K} P={P} "
             f"p={p} ({'seeded random' if rand else 'contiguous'} S)")
@@ -262,13 +272,14 @@ def run_caat(args):
         flops = 2.0 * T * K * H
     out = torch.empty_like(d["R"])
 
-    def step(tm=None):
+    def step(tm=None, st=None):
+        st = stream if st is None else st
         if mlp:
             C.caat_mlp_forward(d["X"], d["A"], d["W2"], d["R"], d["gamma"], sync_idx, P, p, out, workspace=ws,
-                               stream=stream, timing=tm, flags=args.flags)
+                               stream=st, timing=tm, flags=args.flags)
         else:
             C.caat_rowpar_forward(d["X"], d["W"], d["R"], d["gamma"], sync_idx, P, p, out, workspace=ws,
-                                  stream=stream, timing=tm, flags=args.flags)
+                                  stream=st, timing=tm, flags=args.flags)
 
     for _ in range(args.warmup):
         step()
@@ -276,22 +287,56 @@ def run_caat(args):
     if C.caat_get_device_status() != 0:
         raise SystemExit("device status set during warm-up")
 
+    # Workloads whose bytes fit in L2 (decode: W is 90 MB) get an L2 flush before every timed
+    # step: a READ of a buffer 3x the L2 size (a write flush would leave dirty lines whose
+    # write-back the next step would pay for).  Each step is then timed alone with CUDA events
+    # and the flush stays outside the timed intervals.  The step is one call of the library
+    # captured in a CUDA graph (the same kernels, launched from the graph), so that the
+    # host's submission of a call after the flush does not leave the GPU idle inside the
+    # timed interval; the per-kernel split comes from separate flushed calls with the timer.
+    step_bytes = alg_bytes_of(T, K, H, P, mlp)
+    flush = step_bytes < 2 * L2_BYTES
+    flush_buf = torch.ones(3 * L2_BYTES // 4, dtype=torch.float32, device="cuda") if flush else None
+    graph = None
+    if flush:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step(st=torch.cuda.current_stream())
+        graph.replay()
+        torch.cuda.synchronize()
     sampler = ClockSampler(local) if rank == 0 else None
     if sampler:
         sampler.start()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        step(timing)
-    e1.record(stream)
-    torch.cuda.synchronize()
+    if flush:
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        for a_ev, b_ev in evs:
+            flush_buf.sum()
+            a_ev.record(stream)
+            graph.replay()
+            b_ev.record(stream)
+        torch.cuda.synchronize()
+        ms_local = sum(a_ev.elapsed_time(b_ev) for a_ev, b_ev in evs)
+        for _ in range(args.steps):   # per-kernel split (not part of the timed value)
+            flush_buf.sum()
+            step(timing)
+        torch.cuda.synchronize()
+    else:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step(timing)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms_local = e0.elapsed_time(e1)
     if world > 1:
         dist.barrier()
     clocks = sampler.stop() if sampler else None
-    ms = max_over_ranks(e0.elapsed_time(e1))
+    ms = max_over_ranks(ms_local)
+    del flush_buf, graph
     per_kernel = timing.read()
     n_kernels = max((len(r) for r in per_kernel), default=1)
     kernel_ms = [statistics.mean(r[j] for r in per_kernel if len(r) > j) for j in range(n_kernels)]
@@ -365,7 +410,7 @@ def run_caat(args):
     k1_tflops = fc2_flops / k1_ms / 1e9
     norm_bytes = 2.0 * P * T * H * 2
     k2_gbs = norm_bytes / k2_ms / 1e6 if k2_ms else None
-    alg_bytes = 2.0 * (P * T * (K // P) + P * H * (K // P) + 2 * P * T * H + H)
+    alg_bytes = alg_bytes_of(T, K, H, P)
     result = {
         "metric": "TFLOP/s & tokens/s of partially-synced row-parallel FC2 (7B shape), % bf16 peak",
         "value": round(value, 2),
@@ -381,7 +426,10 @@ def run_caat(args):
         "data": "synthetic (seeded N(0,1) activations and residual, N(0,0.02) weights, gamma=1)",
         "config": {"workload": workload_desc(args.workload, T, K, H, P, p, rand), "T": T, "H": H, "K": K,
                    "P": P, "p": p, "parallelism": f"{world} independent GPU(s), P={P} emulated TP ranks each",
-                   "l2": "inputs larger than L2 (%.2f GB touched per step); no flush" % (alg_bytes / 1e9)},
+                   "l2": ("step bytes (%.1f MB) fit in L2: read-flush of a %d MB buffer before every step, "
+                          "outside the per-step event intervals" % (step_bytes / 1e6, 3 * L2_BYTES // 2**20)
+                          if flush else
+                          "inputs larger than L2 (%.2f GB touched per step); no flush" % (step_bytes / 1e9))},
         "tokens_per_s": round(world * T / (ms_step / 1e3), 1),
         "pct_bf16_peak": {"measured_burst": round(100 * value / world / peaks["bf16_tflops"], 1),
                           "datasheet_2250": round(100 * value / world / 2250.0, 1)},

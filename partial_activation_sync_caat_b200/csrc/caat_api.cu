@@ -244,10 +244,16 @@ RowparWs rowpar_ws_layout(int64_t T, int64_t H, int P, bool fused) {
 }
 
 // Decode path (T <= CAAT_DECODE_MAX_T, P <= 16): K splits of the weight-streaming kernel.
-int decode_splits(int64_t T) { return T <= 8 ? 4 : (T <= 32 ? 2 : 1); }
+// One split: the stream of W runs at the same speed with 1, 4 or 8 splits (its time is W
+// bytes plus a fixed launch-to-first-byte cost), and every extra split is one more partial
+// for the reduce kernel to gather.
+int decode_splits(int64_t T) {
+  (void)T;
+  return 1;
+}
 
 bool decode_eligible(int64_t T, int P, int64_t H) {
-  return T >= 1 && T <= CAAT_DECODE_MAX_T && P <= caat::K4_MAXP && H <= 8 * caat::K4B_THREADS * caat::K4B_VEC;
+  return T >= 1 && T <= CAAT_DECODE_MAX_T && P <= caat::K4_MAXP && H <= 4 * caat::K4B_THREADS * caat::K4B_VEC;
 }
 
 // Decode workspace: [256 B | Zp fp32 [splits][P][T][H]].
@@ -447,8 +453,19 @@ caat_status launch_decode(const caat_rowpar_args* a, const std::vector<uint8_t>&
   caat::decode_partials_kernel<<<grid, caat::K4_THREADS, caat::K4_SMEM_BYTES, st>>>(tmW, tmX, prm);
   if (cudaGetLastError() != cudaSuccess) return CAAT_ERR_CUDA;
   rec.after_kernel(st);
-  caat::decode_reduce_norm_kernel<<<static_cast<unsigned>(P * T), caat::K4B_THREADS, 0, st>>>(prm);
-  if (cudaGetLastError() != cudaSuccess) return CAAT_ERR_CUDA;
+  // The reduce kernel is a programmatic dependent of the partials kernel: its launch overlaps
+  // the partials kernel's tail, and it waits in-kernel for that grid's completion.
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3(static_cast<unsigned>(P * T), 1, 1);
+  cfg.blockDim = dim3(caat::K4B_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, caat::decode_reduce_norm_kernel, prm) != cudaSuccess) return CAAT_ERR_CUDA;
   rec.after_kernel(st);
   return CAAT_OK;
 }

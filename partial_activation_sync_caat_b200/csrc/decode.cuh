@@ -14,8 +14,8 @@
 //     tokens are the N side, so W (the only large operand) is read exactly once.
 // K4b decode_reduce_norm_kernel: one CTA per (rank m, token t) row.  It sums the K splits
 //     of rank m's partial, forms the shared channels' cross-rank sum (ranks and splits in
-//     order, fp32), applies the private scale, adds the residual, stores h (bf16), reduces the sum
-//     of squares of the stored h over the CTA and rescales the row held in registers:
+//     order, fp32), applies the private scale, adds the residual, stores h (bf16), reduces the
+//     sum of squares of the stored h over the CTA and rescales the row held in registers:
 //     out = h / sqrt(sum/H + eps) * gamma.
 #pragma once
 
@@ -35,8 +35,8 @@ constexpr int K4_THREADS = 192;
 constexpr int K4_SMEM_BYTES = 1024 + K4_STAGES * K4_STAGE_BYTES + 256;
 constexpr int K4_TMEM_COLS = 128;          // two accumulators of up to 64 columns
 constexpr int K4_MAXP = 16;                // ranks supported by the reduce kernel
-constexpr int K4B_THREADS = 512;
-constexpr int K4B_VEC = 2;                 // 16-byte vectors per thread: H <= 8 * 512 * 2 = 8192
+constexpr int K4B_THREADS = 1024;
+constexpr int K4B_VEC = 2;                 // 4-channel groups per thread: H <= 4 * 1024 * 2 = 8192
 
 struct DecodeParams {
   float* Zp;                  // [splits][P][T][H] fp32 partials
@@ -94,6 +94,8 @@ __global__ void __launch_bounds__(K4_THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // K4b may be scheduled now: it waits (griddepcontrol.wait) for this grid to complete.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const uint32_t tmem_base = *tmem_holder;
   const uint64_t tmo = prm.timeout_ns;
   const int per_rank = prm.n_cb * prm.splits;
@@ -199,51 +201,13 @@ __global__ void __launch_bounds__(K4_THREADS, 1)
   if (warp == 1) tmem_dealloc(tmem_base, K4_TMEM_COLS);
 }
 
-// The partial sums a channel vector needs: own[8] = rank r's partial (all K splits) and, if
-// `shared`, s[8] = the cross-rank sum in rank order 0..P-1.  Loads go out in batches of 8
-// independent (rank, split) pairs so their latencies overlap.
-__device__ __forceinline__ void k4_gather(const DecodeParams& prm, int r, int t, int c, bool shared, float (&own)[8],
-                                          float (&s)[8]) {
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    own[e] = 0.f;
-    s[e] = 0.f;
-  }
-  const int q0 = shared ? 0 : r;
-  const int q1 = shared ? prm.P : r + 1;
-  const int n = (q1 - q0) * prm.splits;
-  for (int base = 0; base < n; base += 8) {
-    float4 a[8], b[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int idx = base + j;
-      a[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-      b[j] = a[j];
-      if (idx < n) {
-        const int q = q0 + idx / prm.splits;
-        const int sp = idx - (idx / prm.splits) * prm.splits;
-        const float4* p = reinterpret_cast<const float4*>(
-            prm.Zp + ((static_cast<size_t>(sp) * prm.P + q) * prm.T + t) * prm.H + c);
-        a[j] = __ldcg(p);
-        b[j] = __ldcg(p + 1);
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int idx = base + j;
-      if (idx >= n) break;
-      const int q = q0 + idx / prm.splits;
-      const float v[8] = {a[j].x, a[j].y, a[j].z, a[j].w, b[j].x, b[j].y, b[j].z, b[j].w};
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        s[e] += v[e];
-        if (q == r) own[e] += v[e];
-      }
-    }
-  }
-}
-
-__global__ void __launch_bounds__(K4B_THREADS)
+// K4b: one CTA per (rank m, token t) row, 4 channels per thread and pass.  All loads a thread
+// needs for its 4 channels go out before any is used: the residual, and the fp32 partials of
+// every rank (the shared channels' cross-rank sum, in rank order 0..P-1; rank m's own partial
+// for the private ones), in batches of 8 ranks.  The stored h stays in registers for the
+// rescale after the block's sum-of-squares reduction.  Launched as a programmatic dependent
+// of K4a: the launch overlaps K4a's tail and griddepcontrol.wait orders the reads.
+__global__ void __launch_bounds__(K4B_THREADS, 1)
     decode_reduce_norm_kernel(const __grid_constant__ DecodeParams prm) {
   __shared__ float red[K4B_THREADS / 32];
   __shared__ float s_rstd;
@@ -251,33 +215,60 @@ __global__ void __launch_bounds__(K4B_THREADS)
   const int t = blockIdx.x / prm.P;
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  const int nvec = prm.H >> 3;
+  const int nq = prm.H >> 2;  // 4-channel groups
   const size_t rowoff = (static_cast<size_t>(r) * prm.T + t) * prm.H;
-  uint4 hv[K4B_VEC];
+  const size_t zstride = static_cast<size_t>(prm.T) * prm.H;  // between ranks (one K split)
+  const float* zrow = prm.Zp + static_cast<size_t>(t) * prm.H;
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // K4a's partials are complete and visible
+
+  static_assert(K4B_VEC == 2, "h of the two passes is held in hv0 / hv1");
+  uint2 hv0 = make_uint2(0u, 0u), hv1 = make_uint2(0u, 0u);
   float ss = 0.f;
-#pragma unroll
+#pragma unroll 1
   for (int k = 0; k < K4B_VEC; ++k) {
-    const int v = threadIdx.x + k * K4B_THREADS;
-    hv[k] = make_uint4(0, 0, 0, 0);
-    if (v >= nvec) continue;
-    const int c = 8 * v;
-    const uint32_t bits = (prm.mask_bits[c >> 5] >> (c & 31)) & 0xFFu;  // 8 channels, 8-aligned
-    float z[8], s[8];
-    k4_gather(prm, r, t, c, bits != 0u, z, s);
-    const uint4 rv = *reinterpret_cast<const uint4*>(prm.R + rowoff + c);
-    const uint32_t rw[4] = {rv.x, rv.y, rv.z, rv.w};
-    uint32_t o[4];
+    const int g = threadIdx.x + k * K4B_THREADS;
+    if (g >= nq) continue;
+    const int c = 4 * g;
+    const uint32_t bits = (prm.mask_bits[c >> 5] >> (c & 31)) & 0xFu;  // 4 channels, 4-aligned
+    const uint2 rv = *reinterpret_cast<const uint2*>(prm.R + rowoff + c);
+    float S[4] = {0.f, 0.f, 0.f, 0.f};
+    float own[4] = {0.f, 0.f, 0.f, 0.f};
+    if (bits != 0u) {
+      for (int m0 = 0; m0 < prm.P; m0 += 8) {
+        for (int sp = 0; sp < prm.splits; ++sp) {
+          const float* zb = zrow + (static_cast<size_t>(sp) * prm.P + m0) * zstride + c;
+          float4 z[8];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float z0 = ((bits >> (2 * e)) & 1u) ? s[2 * e] : prm.private_scale * z[2 * e];
-      const float z1 = ((bits >> (2 * e + 1)) & 1u) ? s[2 * e + 1] : prm.private_scale * z[2 * e + 1];
+          for (int j = 0; j < 8; ++j)
+            z[j] = (m0 + j < prm.P) ? __ldcg(reinterpret_cast<const float4*>(zb + j * zstride))
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            S[0] += z[j].x; S[1] += z[j].y; S[2] += z[j].z; S[3] += z[j].w;
+            if (m0 + j == r) { own[0] += z[j].x; own[1] += z[j].y; own[2] += z[j].z; own[3] += z[j].w; }
+          }
+        }
+      }
+    } else {
+      for (int sp = 0; sp < prm.splits; ++sp) {
+        const float4 w = __ldcg(reinterpret_cast<const float4*>(zrow + (static_cast<size_t>(sp) * prm.P + r) * zstride + c));
+        own[0] += w.x; own[1] += w.y; own[2] += w.z; own[3] += w.w;
+      }
+    }
+    const uint32_t rw[2] = {rv.x, rv.y};
+    uint32_t o[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const float z0 = ((bits >> (2 * e)) & 1u) ? S[2 * e] : prm.private_scale * own[2 * e];
+      const float z1 = ((bits >> (2 * e + 1)) & 1u) ? S[2 * e + 1] : prm.private_scale * own[2 * e + 1];
       o[e] = pack_bf16x2(z0 + bf16lo(rw[e]), z1 + bf16hi(rw[e]));
       const float lo = bf16lo(o[e]), hi = bf16hi(o[e]);
       ss = fmaf(lo, lo, ss);
       ss = fmaf(hi, hi, ss);
     }
-    hv[k] = make_uint4(o[0], o[1], o[2], o[3]);
-    *reinterpret_cast<uint4*>(prm.Hout + rowoff + c) = hv[k];
+    const uint2 hk = make_uint2(o[0], o[1]);
+    if (k == 0) hv0 = hk; else hv1 = hk;
+    *reinterpret_cast<uint2*>(prm.Hout + rowoff + c) = hk;
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, off);
@@ -290,19 +281,19 @@ __global__ void __launch_bounds__(K4B_THREADS)
   }
   __syncthreads();
   const float rs = s_rstd;
-  const uint4* g4 = reinterpret_cast<const uint4*>(prm.gamma);
 #pragma unroll
   for (int k = 0; k < K4B_VEC; ++k) {
-    const int v = threadIdx.x + k * K4B_THREADS;
-    if (v >= nvec) continue;
-    const uint4 g = g4[v];
-    const uint32_t w[4] = {hv[k].x, hv[k].y, hv[k].z, hv[k].w};
-    const uint32_t gw[4] = {g.x, g.y, g.z, g.w};
-    uint32_t o[4];
+    const int g = threadIdx.x + k * K4B_THREADS;
+    if (g >= nq) continue;
+    const uint2 gv = *reinterpret_cast<const uint2*>(prm.gamma + 4 * g);
+    const uint2 hk = k == 0 ? hv0 : hv1;
+    const uint32_t w[2] = {hk.x, hk.y};
+    const uint32_t gw[2] = {gv.x, gv.y};
+    uint32_t o[2];
 #pragma unroll
-    for (int e = 0; e < 4; ++e)
+    for (int e = 0; e < 2; ++e)
       o[e] = pack_bf16x2(bf16lo(w[e]) * rs * bf16lo(gw[e]), bf16hi(w[e]) * rs * bf16hi(gw[e]));
-    *reinterpret_cast<uint4*>(prm.Out + rowoff + 8 * v) = make_uint4(o[0], o[1], o[2], o[3]);
+    *reinterpret_cast<uint2*>(prm.Out + rowoff + 4 * g) = make_uint2(o[0], o[1]);
   }
 }
 

@@ -11,7 +11,7 @@ from oracle import caat_oracle as O
 from partial_activation_sync_caat_b200 import caat as C
 from partial_activation_sync_caat_b200 import inputs as I
 
-from gpu_util import assert_h_close, assert_out_close, ensure_built, run_rowpar
+from gpu_util import assert_h_close, assert_out_close, ensure_built, run_rowpar, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -64,3 +64,47 @@ def test_decode_integer_construction_bit_exact():
         for m in range(P):
             want = np.where(mask[None, :], (2 ** P - 1) * a.numpy()[:, None], (2 ** m) * a.numpy()[:, None])
             np.testing.assert_array_equal(h[m].double().numpy(), want)
+
+
+@pytest.mark.parametrize("T", [1, 64])
+def test_decode_repeat_and_in_place(T):
+    """Back-to-back decode calls (the reduce kernel is a programmatic dependent of the
+    partials kernel) give identical bits, and normalizing h in place (no h_out) gives the same
+    out as with a separate h buffer."""
+    P, K, H = 8, 2048, 1032
+    d = I.make_rowpar_inputs(T, K, H, P, seed=40 + T, x_std=1.0, w_std=0.05, r_std=1.0, gamma="uniform")
+    o1, h1 = run_rowpar(d, P, 0.5)
+    o2, h2 = run_rowpar(d, P, 0.5)
+    o3, _ = run_rowpar(d, P, 0.5, h_out=False)
+    assert torch.equal(o1, o2) and torch.equal(h1, h2)
+    assert torch.equal(o1, o3)
+    ref = O.rowpar_forward(d["X"], d["W"], d["R"], d["gamma"], P, 0.5)
+    assert_out_close(o1, ref, f"decode T={T}")
+
+
+@pytest.mark.parametrize("T", [1, 64, 300])
+def test_call_captured_in_cuda_graph(T):
+    """One call of the device entry point captured in a CUDA graph (decode path: the reduce
+    kernel's programmatic-dependent launch becomes a graph edge; GEMM path at T=300: the
+    counter memset becomes a memset node) replays to the same bits as the eager call."""
+    P, K, H = 8, 2048, 1032
+    d = I.make_rowpar_inputs(T, K, H, P, seed=50 + T, x_std=1.0, w_std=0.05, r_std=1.0, gamma="uniform")
+    o_ref, h_ref = run_rowpar(d, P, 0.5)
+    g = to_dev(d)
+    out = torch.empty_like(g["R"])
+    hb = torch.empty_like(g["R"])
+    ws = C.alloc_workspace(C.caat_workspace_size(T, K, H, P, C.CAAT_VARIANT_ROWPAR))
+    C.caat_rowpar_forward(g["X"], g["W"], g["R"], g["gamma"], None, P, 0.5, out, h_out=hb, workspace=ws)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        C.caat_rowpar_forward(g["X"], g["W"], g["R"], g["gamma"], None, P, 0.5, out, h_out=hb, workspace=ws,
+                              stream=torch.cuda.current_stream())
+    for _ in range(2):
+        out.zero_()
+        hb.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        assert C.caat_get_device_status() == 0
+        assert torch.equal(out.cpu(), o_ref) and torch.equal(hb.cpu(), h_ref)
+    del graph
