@@ -271,6 +271,23 @@ def run_caat(args):
         ws = C.alloc_workspace(C.caat_workspace_size(T, K, H, P), "cuda")
         flops = 2.0 * T * K * H
     out = torch.empty_like(d["R"])
+    # A random sync list: W's output channels are permuted once (as at weight load time) so
+    # that the shared channels are contiguous; every step then runs the permuted path.
+    user_flags = args.flags
+    permute = rand and not mlp and not args.no_permute
+    permute_ms = None
+    if permute:
+        Wp = torch.empty_like(d["W"])
+        C.caat_permute_weights(d["W"], Wp, sync_idx, P, p)       # warm-up
+        torch.cuda.synchronize()
+        pa, pb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        pa.record(stream)
+        C.caat_permute_weights(d["W"], Wp, sync_idx, P, p, stream=stream)
+        pb.record(stream)
+        torch.cuda.synchronize()
+        permute_ms = pa.elapsed_time(pb)
+        d["W"] = Wp
+        args.flags |= C.CAAT_FLAG_W_PERMUTED
 
     def step(tm=None, st=None):
         st = stream if st is None else st
@@ -348,7 +365,7 @@ def run_caat(args):
 
     # optional p sweep (same shapes, fewer steps), rank 0 only
     sweep = None
-    if args.sweep and rank == 0 and not mlp:
+    if args.sweep and rank == 0 and not mlp and not permute:   # W is permuted for one (p, S) only
         sweep = {}
         for ps in (0.0, 0.25, 0.5, 0.75, 1.0):
             idx_s = I.random_sync_idx(H, int((H * ps) // 1), seed=0) if rand else None
@@ -374,7 +391,7 @@ def run_caat(args):
         hout = torch.empty(hR.shape, dtype=torch.bfloat16).pin_memory()
         wsh = C.alloc_workspace(C.caat_workspace_size(T, K, H, P, C.CAAT_VARIANT_ROWPAR_HOST), "cuda")
         for _ in range(2):
-            C.caat_rowpar_forward_host(hX, hW, hR, hg, sync_idx, P, p, hout, wsh, stream=stream)
+            C.caat_rowpar_forward_host(hX, hW, hR, hg, sync_idx, P, p, hout, wsh, stream=stream, flags=args.flags)
         torch.cuda.synchronize()
         n_e2e = max(3, min(args.steps, 10))
         if world > 1:
@@ -382,7 +399,7 @@ def run_caat(args):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         for _ in range(n_e2e):
-            C.caat_rowpar_forward_host(hX, hW, hR, hg, sync_idx, P, p, hout, wsh, stream=stream)
+            C.caat_rowpar_forward_host(hX, hW, hR, hg, sync_idx, P, p, hout, wsh, stream=stream, flags=args.flags)
         b.record(stream)
         torch.cuda.synchronize()
         e_ms = max_over_ranks(a.elapsed_time(b) / n_e2e)
@@ -401,7 +418,7 @@ def run_caat(args):
         return
 
     peaks, peak_src = load_peaks()
-    default_case = not args.tokens and args.p is None and not args.flags  # the recorded ncu case
+    default_case = not args.tokens and args.p is None and not user_flags  # the recorded ncu case
     ms_step = ms / args.steps
     value = whole_job_tflops(flops, world, ms_step)
     k1_ms = statistics.mean(k1) if k1 else float("nan")
@@ -462,6 +479,9 @@ def run_caat(args):
                                  "launch_ms": round(k2_ms, 4), "algorithmic": "2*P*T*H*2 bytes (read h, write out)"}
     if args.flags:
         result["config"]["flags"] = hex(args.flags)
+    if permute:
+        result["w_permuted"] = {"api": "caat_permute_weights, once before the steps (weights are static)",
+                                "once_ms": round(permute_ms, 4)}
     if sweep is not None:
         result["p_sweep"] = sweep
     if e2e is not None:
@@ -528,6 +548,8 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="fc2-7b")
     ap.add_argument("--p", type=float, default=None)
     ap.add_argument("--tokens", type=int, default=None, help="override T (profiling a smaller case)")
+    ap.add_argument("--no-permute", action="store_true",
+                    help="random sync list: run on the original W (mixed tiles) instead of permuting it once")
     ap.add_argument("--flags", type=lambda x: int(x, 0), default=0, help="CAAT_FLAG_* bits (tuning variants)")
     ap.add_argument("--sweep", action="store_true", help="also time p in {0,.25,.5,.75,1}")
     ap.add_argument("--no-e2e", action="store_true")

@@ -87,6 +87,16 @@ typedef enum caat_status {
                                             rank by rank); the fused norm always does */
 #define CAAT_FLAG_SINGLE_CTA 0x4u        /* use the single-CTA GEMM kernel (128-token tiles)
                                             instead of the CTA-pair kernel (256-token tiles) */
+#define CAAT_FLAG_W_PERMUTED 0x80u       /* W is the channel-permuted weight written by
+                                            caat_permute_weights for this (sync_idx, p):
+                                            the GEMM sees a contiguous sync set (no column
+                                            block mixes shared and private channels) and the
+                                            norm kernel restores the original channel order.
+                                            Outputs stay in the original order.  Needs a
+                                            buffer for Z' (h_out if given and distinct from
+                                            residual, else out, which must then not alias
+                                            residual); not with CAAT_FLAG_FUSED_NORM; the
+                                            GEMM path needs H <= 4096. */
 #define CAAT_FLAG_TEST_STALL 0x100u      /* test hook: the GEMM kernel's MMA warp never signals
                                             its accumulator, so every consumer wait runs out
                                             and the call reports CAAT_ERR_TIMEOUT through
@@ -218,6 +228,23 @@ typedef struct caat_mlp_args {
 } caat_mlp_args;
 
 CAAT_API caat_status caat_mlp_forward_ex(const caat_mlp_args* args);
+
+/*
+ * caat_permute_weights - reorders the output channels (rows) of W for a sync set: with
+ * perm(i) = the i-th shared channel for i < n_s and the (i - n_s)-th private channel
+ * otherwise (both ascending), W_out[m, i, :] = W[m, perm(i), :] for every rank m.  The
+ * layer's result does not depend on the order of the output channels (Eq. 22 sums each
+ * shared channel over the ranks, whatever its index), so a forward call given W_out and
+ * CAAT_FLAG_W_PERMUTED computes the same layer with the shared channels contiguous, which
+ * keeps every 256-channel tile of the GEMM pure when S is an arbitrary list.  Done once per
+ * weight (static weights: at load time).  No counterpart in the paper.
+ *
+ *   W, W_out  device, bf16 [P, H, K/P], 16-byte aligned, must not overlap.
+ *   sync_idx, p, P, H, K  as for caat_rowpar_forward (same validation).
+ * Asynchronous on `stream`; returns CAAT_OK once the copy kernel is queued.
+ */
+CAAT_API caat_status caat_permute_weights(const caat_bf16* W, caat_bf16* W_out, const int32_t* sync_idx, double p,
+                                          int P, int64_t H, int64_t K, caat_stream_t stream);
 
 /* Bytes of device workspace a forward call of this shape needs (0 for invalid shapes is
  * never returned: invalid shapes give SIZE_MAX).  variant: CAAT_VARIANT_*; for the MLP

@@ -34,6 +34,7 @@ CAAT_FLAG_FUSED_NORM = 0x8
 CAAT_FLAG_ORDER_ROWBLOCK = 0x10
 CAAT_FLAG_OVERLAP_NORM = 0x20
 CAAT_FLAG_ORDER_GROUPED = 0x40
+CAAT_FLAG_W_PERMUTED = 0x80
 CAAT_FLAG_TEST_STALL = 0x100
 
 CAAT_NOALLOC_SCRATCH_BYTES = 1048576
@@ -44,7 +45,7 @@ EXPORTS = [
     "caat_rowpar_forward_noalloc", "caat_mlp_forward", "caat_mlp_forward_ex",
     "caat_workspace_size", "caat_sync_mask", "caat_get_device_status", "caat_timing_create",
     "caat_timing_destroy", "caat_timing_reset", "caat_timing_read", "caat_status_string",
-    "caat_version",
+    "caat_version", "caat_permute_weights",
 ]
 
 
@@ -106,6 +107,8 @@ def lib() -> ctypes.CDLL:
     L.caat_workspace_size.argtypes = [i64, i64, i64, ctypes.c_int, ctypes.c_int]
     L.caat_workspace_size.restype = sz
     L.caat_sync_mask.argtypes = [i64, dbl, vp, vp, ctypes.POINTER(i64)]
+    L.caat_permute_weights.restype = ctypes.c_int
+    L.caat_permute_weights.argtypes = [vp, vp, vp, dbl, ctypes.c_int, i64, i64, vp]
     L.caat_sync_mask.restype = ctypes.c_int
     L.caat_get_device_status.argtypes = [vp, ctypes.POINTER(i32)]
     L.caat_get_device_status.restype = ctypes.c_int
@@ -189,6 +192,18 @@ def caat_sync_mask(H: int, p: float, sync_idx=None):
     code = lib().caat_sync_mask(int(H), float(p), ptr, mask.ctypes.data, ctypes.byref(ns))
     _check(code, "caat_sync_mask")
     return mask, int(ns.value)
+
+
+def caat_permute_weights(W, W_out, sync_idx, P: int, p: float, stream=None):
+    """W_out[m, i] = W[m, perm(i)]: the shared channels first, then the private ones (both
+    ascending).  W, W_out: device bf16 [P, H, K/P], not overlapping.  Asynchronous."""
+    P_, H, Kp = W.shape
+    if P_ != P or tuple(W_out.shape) != tuple(W.shape):
+        raise CaatError(CAAT_ERR_INVALID_ARG, "caat_permute_weights: shapes")
+    arr, ptr = _sync_idx_host(sync_idx)
+    code = lib().caat_permute_weights(_ptr(W), _ptr(W_out), ptr, float(p), int(P), int(H), int(Kp * P),
+                                      _stream_ptr(stream))
+    _check(code, "caat_permute_weights")
 
 
 def caat_workspace_size(T: int, K: int, H: int, P: int, variant: int = CAAT_VARIANT_ROWPAR) -> int:

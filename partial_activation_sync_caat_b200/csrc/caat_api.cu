@@ -19,6 +19,7 @@
 #include "rowpar_gemm2.cuh"
 #include "fc1_swiglu.cuh"
 #include "decode.cuh"
+#include "permuted.cuh"
 #include "rownorm.cuh"
 
 namespace {
@@ -65,7 +66,13 @@ caat_status device_info(DeviceInfo** out) {
           cudaFuncSetAttribute(caat::fc1_swiglu_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                caat::K3_SMEM_BYTES) != cudaSuccess ||
           cudaFuncSetAttribute(caat::decode_partials_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               caat::K4_SMEM_BYTES) != cudaSuccess)
+                               caat::K4_SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(caat::rownorm_gather_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(caat::gather_smem_bytes(1024))) != cudaSuccess ||
+          cudaFuncSetAttribute(caat::rownorm_gather_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(caat::gather_smem_bytes(2048))) != cudaSuccess ||
+          cudaFuncSetAttribute(caat::rownorm_gather_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(caat::gather_smem_bytes(4096))) != cudaSuccess)
         return CAAT_ERR_CUDA;
       cudaLaunchConfig_t cfg = {};
       cudaLaunchAttribute attr[1];
@@ -438,8 +445,12 @@ caat_status launch_decode(const caat_rowpar_args* a, const std::vector<uint8_t>&
   prm.private_scale = a->private_scale;
   prm.eps = a->eps;
   prm.timeout_ns = timeout_ns();
+  prm.permuted = (a->flags & CAAT_FLAG_W_PERMUTED) ? 1 : 0;
   for (int64_t c = 0; c < H; ++c)
-    if (mask[c]) prm.mask_bits[c >> 5] |= 1u << (c & 31);
+    if (mask[c]) {
+      prm.mask_bits[c >> 5] |= 1u << (c & 31);
+      ++prm.n_s;
+    }
 
   CUtensorMap tmW, tmX;
   caat_status s = make_map_3d(&tmW, a->W, Kp, H, P, caat::K4_BK, caat::K4_BM);
@@ -482,9 +493,28 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
   cudaStream_t st = a->stream;
   __nv_bfloat16* hdst = reinterpret_cast<__nv_bfloat16*>(a->h_out ? a->h_out : a->out);
 
+  // Channel-permuted W (caat_permute_weights): the GEMM runs on a contiguous sync set and
+  // writes Z' (no residual) into zdst; the gather norm restores the channel order.
+  const bool permuted = (a->flags & CAAT_FLAG_W_PERMUTED) != 0;
+  std::vector<uint8_t> pmask;
+  const std::vector<uint8_t>* tmask = &mask;  // the mask the GEMM's tiles see
+  int n_s = 0;
+  for (int64_t c = 0; c < H; ++c) n_s += mask[c];
+  if (permuted) {
+    if (a->flags & CAAT_FLAG_FUSED_NORM) return CAAT_ERR_UNSUPPORTED;
+    if (H > 4096) return CAAT_ERR_UNSUPPORTED;
+    void* zd = (a->h_out && a->h_out != a->residual) ? a->h_out : a->out;
+    if (zd == a->residual) return CAAT_ERR_UNSUPPORTED;
+    hdst = reinterpret_cast<__nv_bfloat16*>(zd);
+    pmask.assign(static_cast<size_t>(H), 0);
+    for (int c = 0; c < n_s; ++c) pmask[c] = 1;
+    tmask = &pmask;
+  }
+
   static thread_local RowparParams prm;  // ~10 KiB: keep it off the stack
   std::memset(&prm, 0, sizeof(prm));
   const bool fused = (a->flags & CAAT_FLAG_FUSED_NORM) != 0;
+  prm.no_residual = permuted ? 1 : 0;
   const RowparWs wl = rowpar_ws_layout(T, H, P, fused);
   uint8_t* wsb = reinterpret_cast<uint8_t*>(counter);
   prm.R = reinterpret_cast<const __nv_bfloat16*>(a->residual);
@@ -518,14 +548,14 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
     const int64_t c0 = int64_t(nb) * caat::K1_BN;
     const int64_t c1 = std::min<int64_t>(H, c0 + caat::K1_BN);
     int64_t cnt = 0;
-    for (int64_t c = c0; c < c1; ++c) cnt += mask[c];
+    for (int64_t c = c0; c < c1; ++c) cnt += (*tmask)[c];
     const uint8_t cls = cnt == 0 ? 0 : (cnt == c1 - c0 ? 1 : 2);
     prm.ncls[nb] = cls;
     if (cls != 0) prm.slist[prm.nS++] = static_cast<uint16_t>(nb);
     if (cls != 1) prm.plist[prm.nPriv++] = static_cast<uint16_t>(nb);
   }
   for (int64_t c = 0; c < H; ++c)
-    if (mask[c]) prm.mask_bits[c >> 5] |= 1u << (c & 31);
+    if ((*tmask)[c]) prm.mask_bits[c >> 5] |= 1u << (c & 31);
   prm.nslots = prm.nS + prm.nPriv;
   // The CTA-pair kernel (256-token tiles) for all but the smallest token counts.
   const bool pair = !(a->flags & CAAT_FLAG_SINGLE_CTA) && dev->max_pairs > 0 && T > caat::K1_BM;
@@ -595,6 +625,31 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
   __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(a->out);
   auto norm = [&](int64_t t0, int64_t tc, cudaStream_t ns, int64_t max_blocks) -> caat_status {
     const int64_t rows = int64_t(P) * tc;
+    if (permuted) {
+      static thread_local caat::PermParams pp;
+      std::memset(&pp, 0, sizeof(pp));
+      pp.P = P;
+      pp.H = static_cast<int>(H);
+      pp.Kp = static_cast<int>(Kp);
+      pp.n_s = n_s;
+      pp.T = T;
+      pp.eps = a->eps;
+      for (int64_t c = 0; c < H; ++c)
+        if (mask[c]) pp.mask_bits[c >> 5] |= 1u << (c & 31);
+      const size_t smem = caat::gather_smem_bytes(static_cast<int>(H));
+      const int64_t wpb = caat::K2P_THREADS / 32;
+      const int64_t per_sm = H <= 2048 ? 2 : 1;  // blocks resident per SM (registers, shared memory)
+      const int64_t gb = std::min<int64_t>((int64_t(P) * T + wpb - 1) / wpb, int64_t(dev->sm_count) * per_sm);
+      __nv_bfloat16* hk = reinterpret_cast<__nv_bfloat16*>(a->h_out);  // may equal hdst (in place)
+      const __nv_bfloat16* rr = reinterpret_cast<const __nv_bfloat16*>(a->residual);
+      if (H <= 1024)
+        caat::rownorm_gather_kernel<4><<<gb, caat::K2P_THREADS, smem, ns>>>(hdst, rr, hk, o, g, pp);
+      else if (H <= 2048)
+        caat::rownorm_gather_kernel<8><<<gb, caat::K2P_THREADS, smem, ns>>>(hdst, rr, hk, o, g, pp);
+      else
+        caat::rownorm_gather_kernel<16><<<gb, caat::K2P_THREADS, smem, ns>>>(hdst, rr, hk, o, g, pp);
+      return cudaGetLastError() == cudaSuccess ? CAAT_OK : CAAT_ERR_CUDA;
+    }
     const int64_t warps_per_block = caat::K2_THREADS / 32;
     const int64_t blocks = std::min<int64_t>((rows + warps_per_block - 1) / warps_per_block, max_blocks);
     if (H <= 4096) {
@@ -616,7 +671,7 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
   Recorder own;
   Recorder& rec = outer ? *outer : own;
   if (!outer) rec.begin(a->timing, st);
-  const bool overlap = !fused && (a->flags & CAAT_FLAG_OVERLAP_NORM) && T >= 2 * kNormChunk;
+  const bool overlap = !fused && !permuted && (a->flags & CAAT_FLAG_OVERLAP_NORM) && T >= 2 * kNormChunk;
   if (!overlap) {
     s = gemm(0, T);
     if (s != CAAT_OK) return s;
@@ -697,6 +752,38 @@ caat_status caat_sync_mask(int64_t H, double p, const int32_t* sync_idx, uint8_t
   if (mask_out) std::memcpy(mask_out, mask.data(), static_cast<size_t>(H));
   if (n_sync_out) *n_sync_out = ns;
   return CAAT_OK;
+}
+
+caat_status caat_permute_weights(const caat_bf16* W, caat_bf16* W_out, const int32_t* sync_idx, double p, int P,
+                                 int64_t H, int64_t K, caat_stream_t stream) {
+  caat_status s = check_shapes(0, K, H, P, p);
+  if (s != CAAT_OK) return s;
+  std::vector<uint8_t> mask;
+  int64_t ns = 0;
+  s = build_mask(H, p, sync_idx, mask, &ns);
+  if (s != CAAT_OK) return s;
+  if (!W || !W_out) return CAAT_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(W_out)) return CAAT_ERR_UNSUPPORTED;
+  const size_t bytes = static_cast<size_t>(K) * static_cast<size_t>(H) * 2;  // P * H * (K/P) bf16
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(W), b0 = reinterpret_cast<uintptr_t>(W_out);
+  if (a0 < b0 + bytes && b0 < a0 + bytes) return CAAT_ERR_INVALID_ARG;  // overlap
+  DeviceInfo* dev = nullptr;
+  s = device_info(&dev);
+  if (s != CAAT_OK) return s;
+  static thread_local caat::PermParams pp;
+  std::memset(&pp, 0, sizeof(pp));
+  pp.P = P;
+  pp.H = static_cast<int>(H);
+  pp.Kp = static_cast<int>(K / P);
+  pp.n_s = static_cast<int>(ns);
+  for (int64_t c = 0; c < H; ++c)
+    if (mask[c]) pp.mask_bits[c >> 5] |= 1u << (c & 31);
+  const int64_t rows = int64_t(P) * H;
+  const int64_t wpb = caat::K5_THREADS / 32;
+  const int64_t blocks = std::min<int64_t>((rows + wpb - 1) / wpb, int64_t(dev->sm_count) * 8);
+  caat::permute_rows_kernel<<<static_cast<unsigned>(blocks), caat::K5_THREADS, 0, static_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const __nv_bfloat16*>(W), reinterpret_cast<__nv_bfloat16*>(W_out), pp);
+  return cudaGetLastError() == cudaSuccess ? CAAT_OK : CAAT_ERR_CUDA;
 }
 
 size_t caat_workspace_size(int64_t T, int64_t K, int64_t H, int P, int variant) {

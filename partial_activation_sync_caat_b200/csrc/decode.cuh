@@ -19,6 +19,7 @@
 //     out = h / sqrt(sum/H + eps) * gamma.
 #pragma once
 
+#include "permuted.cuh"
 #include "ptx.cuh"
 #include "rowpar_common.cuh"
 
@@ -53,6 +54,8 @@ struct DecodeParams {
   int n_units;                // P * n_cb * splits
   float private_scale, eps;
   uint64_t timeout_ns;
+  int permuted;               // 1: W's rows are channel-permuted (permuted.cuh): Zp columns are permuted
+  int n_s;                    // shared channels (the permuted path's prefix length)
   uint32_t mask_bits[K1_MASK_WORDS];
 };
 
@@ -219,6 +222,9 @@ __global__ void __launch_bounds__(K4B_THREADS, 1)
   const size_t rowoff = (static_cast<size_t>(r) * prm.T + t) * prm.H;
   const size_t zstride = static_cast<size_t>(prm.T) * prm.H;  // between ranks (one K split)
   const float* zrow = prm.Zp + static_cast<size_t>(t) * prm.H;
+  __shared__ uint32_t s_mask[K1_MASK_WORDS];
+  __shared__ int s_pre[K1_MASK_WORDS + 1];
+  if (prm.permuted) mask_prefix(prm.mask_bits, (prm.H + 31) >> 5, s_mask, s_pre);
   asm volatile("griddepcontrol.wait;" ::: "memory");  // K4a's partials are complete and visible
 
   static_assert(K4B_VEC == 2, "h of the two passes is held in hv0 / hv1");
@@ -233,7 +239,30 @@ __global__ void __launch_bounds__(K4B_THREADS, 1)
     const uint2 rv = *reinterpret_cast<const uint2*>(prm.R + rowoff + c);
     float S[4] = {0.f, 0.f, 0.f, 0.f};
     float own[4] = {0.f, 0.f, 0.f, 0.f};
-    if (bits != 0u) {
+    if (prm.permuted) {
+      // channel c + e's partials sit at column pos(c + e) of Zp; one channel at a time
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int pe = perm_pos(c + e, prm.n_s, s_mask, s_pre);
+        const bool shared_e = (bits >> e) & 1u;
+        for (int sp = 0; sp < prm.splits; ++sp) {
+          const float* zb = zrow + static_cast<size_t>(sp) * prm.P * zstride + pe;
+          for (int m0 = 0; m0 < prm.P; m0 += 8) {
+            float z[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int m = m0 + j;
+              z[j] = (m < prm.P && (shared_e || m == r)) ? __ldcg(zb + m * zstride) : 0.f;
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              S[e] += z[j];
+              if (m0 + j == r) own[e] += z[j];
+            }
+          }
+        }
+      }
+    } else if (bits != 0u) {
       for (int m0 = 0; m0 < prm.P; m0 += 8) {
         for (int sp = 0; sp < prm.splits; ++sp) {
           const float* zb = zrow + (static_cast<size_t>(sp) * prm.P + m0) * zstride + c;

@@ -35,7 +35,7 @@ struct K1Threads {
 
 // TMA epilogue of pure column blocks: per epilogue warp, K1_EPI_NBUF shared-memory buffers of
 // one 32-row x 64-column bf16 box (128-byte rows, 128-byte swizzle).
-constexpr int K1_EPI_NBUF = 2;
+constexpr int K1_EPI_NBUF = 2;  // the no-residual epilogue's buffer reuse relies on 2 (wait_group.read 1)
 constexpr int K1_EPI_BOX_BYTES = 32 * 64 * 2;
 constexpr int K1_EPI_BYTES = 4 * K1_EPI_NBUF * K1_EPI_BOX_BYTES;  // per CTA
 constexpr int K1_NORM_WARP0 = 6;                 // first normalizer warp (fused RMSNorm)
@@ -58,6 +58,7 @@ struct RowparParams {
   float* ss_part;              // [P][T_pad][nslots] per-row sum-of-squares partials
   unsigned int* sdone;         // [T_pad/32][n-blocks] shared unit of a mixed block stored, zero at launch
   int merge_mixed;             // 1: mixed blocks use the TMA epilogue (see k1_epilogue_tma)
+  int no_residual;             // 1: store Z (no residual add) -- channel-permuted path, see rownorm.cuh
   int T, H, Kp, P;             // T: token rows of the tensors (the row stride of rank blocks)
   int t_begin, t_end;          // token rows this launch processes: [t_begin, t_end)
   int n_mblk;                  // row blocks of the kernel's tile height over [t_begin, t_end)
@@ -245,7 +246,7 @@ __device__ __forceinline__ void k1_epilogue_private(uint32_t trow, const RowparP
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       rv[j] = make_uint4(0, 0, 0, 0);
-      if (row_ok && cb + 8 * j < ncols) rv[j] = ld_nc_v4(Rp + cb + 8 * j);
+      if (row_ok && !prm.no_residual && cb + 8 * j < ncols) rv[j] = ld_nc_v4(Rp + cb + 8 * j);
     }
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
@@ -296,7 +297,7 @@ __device__ __forceinline__ void k1_epilogue_shared(uint32_t trow, const RowparPa
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           rv[rr][k] = make_uint4(0, 0, 0, 0);
-          if (row_ok && r0 + rr < prm.P && cc + 8 * k < ncols)
+          if (row_ok && !prm.no_residual && r0 + rr < prm.P && cc + 8 * k < ncols)
             rv[rr][k] = ld_nc_v4(prm.R + (r0 + rr) * rstride + base + cc + 8 * k);
         }
       tmem_wait_ld();
@@ -341,8 +342,8 @@ __device__ __forceinline__ bool k1_epilogue_tma(uint32_t trow, const RowparParam
     const float scale = prm.private_scale;
     for (int c = 0; c < nch; ++c) {
       if (lane == 0) {
-        mbar_arrive_expect_tx(&rbar[0], 2 * K1_EPI_BOX_BYTES);
-        tma_load_3d(bufs, tmR, &rbar[0], n0 + 64 * c, row0, rank, pol_r);
+        mbar_arrive_expect_tx(&rbar[0], (prm.no_residual ? 1 : 2) * K1_EPI_BOX_BYTES);
+        if (!prm.no_residual) tma_load_3d(bufs, tmR, &rbar[0], n0 + 64 * c, row0, rank, pol_r);
         tma_load_3d(bufs + K1_EPI_BOX_BYTES, tmH, &rbar[0], n0 + 64 * c, row0, rank, pol_r);
       }
       uint32_t v[64];
@@ -360,7 +361,7 @@ __device__ __forceinline__ bool k1_epilogue_tma(uint32_t trow, const RowparParam
         const int col = n0 + 64 * c + 8 * j;
         const uint32_t bits = (prm.mask_bits[col >> 5] >> (col & 31)) & 0xFFu;
         const int g = (j ^ (lane & 7)) << 4;
-        const uint4 rr = *reinterpret_cast<const uint4*>(rrow + g);
+        const uint4 rr = prm.no_residual ? make_uint4(0u, 0u, 0u, 0u) : *reinterpret_cast<const uint4*>(rrow + g);
         const uint4 hh = *reinterpret_cast<const uint4*>(hrow + g);
         const uint32_t rw[4] = {rr.x, rr.y, rr.z, rr.w};
         const uint32_t hw[4] = {hh.x, hh.y, hh.z, hh.w};
@@ -391,6 +392,39 @@ __device__ __forceinline__ bool k1_epilogue_tma(uint32_t trow, const RowparParam
   const int n_items = nch * nr;  // rank-major: item i = (rank i / nch, chunk i % nch)
   const float scale = rank < 0 ? 1.0f : prm.private_scale;
   const int row = row0 + lane;
+  if (prm.no_residual) {
+    // Z only: no residual boxes to load; each item is composed straight into a free buffer.
+    for (int i = 0; i < n_items; ++i) {
+      const int ri = i / nch, c = i - ri * nch;
+      const int r = rank < 0 ? ri : rank;
+      const int b = i % K1_EPI_NBUF;
+      uint32_t v[64];
+      __syncwarp();
+      tmem_ld_32x32b_x32(trow + 64 * c, *reinterpret_cast<uint32_t(*)[32]>(v));
+      tmem_ld_32x32b_x32(trow + 64 * c + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+      tmem_wait_ld();
+      if (lane == 0 && i >= K1_EPI_NBUF) bulk_wait_group_read1();  // the store from buffer b has read it
+      __syncwarp();
+      uint8_t* rowp = bufs + b * K1_EPI_BOX_BYTES + lane * 128;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        uint32_t o[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          o[e] = pack_bf16x2(__uint_as_float(v[8 * j + 2 * e]) * scale, __uint_as_float(v[8 * j + 2 * e + 1]) * scale);
+        *reinterpret_cast<uint4*>(rowp + ((j ^ (lane & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_3d(tmH, bufs + b * K1_EPI_BOX_BYTES, n0 + 64 * c, row0, r, pol_h);
+        bulk_commit_group();
+      }
+    }
+    if (lane == 0) bulk_wait_group_read0();
+    __syncwarp();
+    return true;
+  }
   const int npre = min(K1_EPI_NBUF, n_items);
   for (int i = 0; i < npre; ++i) {
     const int ri = i / nch, c = i - ri * nch;

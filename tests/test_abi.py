@@ -130,3 +130,17 @@ def test_ex_rejects_null_and_bad_eps(L):
     assert L.caat_rowpar_forward_ex(ctypes.byref(a)) == C.CAAT_ERR_INVALID_ARG
     a.eps, a.private_scale = 1e-5, float("nan")
     assert L.caat_rowpar_forward_ex(ctypes.byref(a)) == C.CAAT_ERR_INVALID_ARG
+
+
+def test_permute_weights_rejects_invalid_arguments_without_device_work(L):
+    def call(W=0x100000, Wo=0x900000, idx=None, p=0.5, P=2, H=768, K=768):
+        return L.caat_permute_weights(W, Wo, idx, p, P, H, K, None)
+    assert call(P=0) == C.CAAT_ERR_INVALID_ARG
+    assert call(p=-0.1) == C.CAAT_ERR_INVALID_ARG
+    assert call(H=770) == C.CAAT_ERR_UNSUPPORTED
+    assert call(K=770) == C.CAAT_ERR_UNSUPPORTED
+    assert call(W=None) == C.CAAT_ERR_INVALID_ARG
+    assert call(Wo=0x100008) == C.CAAT_ERR_UNSUPPORTED          # misaligned
+    assert call(Wo=0x100000 + 768 * 768) == C.CAAT_ERR_INVALID_ARG  # overlaps W (W is 768*768*2 bytes)
+    bad = np.array([5, 3], dtype=np.int32)
+    assert call(H=8, K=16, p=0.25, idx=bad.ctypes.data) == C.CAAT_ERR_INVALID_ARG

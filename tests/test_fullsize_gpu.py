@@ -57,6 +57,13 @@ def test_fc2_1b_random_sync_idx_full():
     out = _run(to_dev(d), 4, 0.5, idx)
     ref = O.rowpar_forward(d["X"], d["W"], d["R"], d["gamma"], 4, 0.5, idx)
     assert_out_close(out, ref, "fc2-1b random S")
+    # the channel-permuted path on the same inputs (W permuted once, as the bench does)
+    g = to_dev(d)
+    Wp = torch.empty_like(g["W"])
+    C.caat_permute_weights(g["W"], Wp, idx, 4, 0.5)
+    g["W"] = Wp
+    out_p = _run(g, 4, 0.5, idx, flags=C.CAAT_FLAG_W_PERMUTED)
+    assert_out_close(out_p, ref, "fc2-1b random S, permuted W")
 
 
 @pytest.mark.parametrize("T", [1, 8, 64])
