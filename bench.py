@@ -479,6 +479,18 @@ def run_caat(args):
                                  "launch_ms": round(k2_ms, 4), "algorithmic": "2*P*T*H*2 bytes (read h, write out)"}
     if args.flags:
         result["config"]["flags"] = hex(args.flags)
+    if not mlp:
+        # the paper's speed-up model (App. C Eq. 34-35) for this shape, fed with this pool's
+        # measured numbers: bf16 GEMM burst and the NVLink peer copy per direction (770 GB/s,
+        # bf16 activations on the wire): C = operations per exchanged activation
+        nvlink_gbs = 770.0
+        c_ratio = peaks["bf16_tflops"] * 1e12 / (nvlink_gbs * 1e9 / 2.0)
+        sp_m, ps_m = C.caat_speedup_model(H, T, P, p, c_ratio)
+        result["speedup_model"] = {"source": "App. C Eq. 34-35", "h": H, "s": T, "r": P, "p": p,
+                                   "C_ops_per_activation": round(c_ratio, 1),
+                                   "C_inputs": f"{peaks['bf16_tflops']} TFLOP/s {peak_src} bf16 / "
+                                               f"({nvlink_gbs} GB/s NVLink per direction / 2 B)",
+                                   "speedup_vs_full_sync": round(sp_m, 4), "p_star": round(ps_m, 4)}
     if permute:
         result["w_permuted"] = {"api": "caat_permute_weights, once before the steps (weights are static)",
                                 "once_ms": round(permute_ms, 4)}

@@ -246,6 +246,18 @@ CAAT_API caat_status caat_mlp_forward_ex(const caat_mlp_args* args);
 CAAT_API caat_status caat_permute_weights(const caat_bf16* W, caat_bf16* W_out, const int32_t* sync_idx, double p,
                                           int P, int64_t H, int64_t K, caat_stream_t stream);
 
+/*
+ * caat_speedup_model - the paper's speed-up model of partial synchronization (App. C,
+ * Eq. 31-35), host only.  Per device and transformer layer (forward): G = (24 s h^2 +
+ * 4 s^2 h) / r GEMM operations and P(p) = 2 s h p exchanged activations; with C the ratio of
+ * compute to communication capacity in operations per exchanged activation, T(p) = G + C P(p),
+ *   speedup = (T(1) - T(p)) / T(1) = (1 - p) / (1 + (12 h + 2 s) / (C r)),
+ *   p*      = min((12 h + 2 s) / (C r), 1)   (C P(p*) = G: the exchange just fits under the compute).
+ * h hidden size, s tokens, r tensor-parallel ranks, p in [0, 1], C > 0; outputs may be NULL.
+ */
+CAAT_API caat_status caat_speedup_model(double h, double s, double r, double p, double C, double* speedup_out,
+                                        double* p_star_out);
+
 /* Bytes of device workspace a forward call of this shape needs (0 for invalid shapes is
  * never returned: invalid shapes give SIZE_MAX).  variant: CAAT_VARIANT_*; for the MLP
  * variant K is F. */

@@ -16,7 +16,8 @@ Karnieli, Hanani, Giladi, Soudry; arXiv 2506.19645):
   multiplied by sqrt(r) so that their variance matches the shared ones);
 * residual add and norm: §4 Eq. 9 and App. B Eq. 25 (X_m = Norm(sum Z + R)); the norm is
   RMSNorm here, with gamma shared by the ranks (§4: norm parameters are synchronized);
-* MLP block: §3.1 Eq. 6 (Y_m = sigma(X_m A_m), column-parallel A) with sigma = SwiGLU.
+* MLP block: §3.1 Eq. 6 (Y_m = sigma(X_m A_m), column-parallel A) with sigma = SwiGLU;
+* speed-up model: App. C Eq. 31-35 (compute and exchange per layer, T(p), speed-up, p*).
 
 Everything is plain NumPy float64: one library matmul per partial product, no blocking,
 fusion or reordering beyond the definitions above.  The inputs are the bf16 tensors
@@ -186,6 +187,31 @@ def mlp_rows(X, A, W2, R, gamma, P: int, p: float, rows, sync_idx=None, *, eps: 
     rows = np.asarray(rows, dtype=np.int64)
     return mlp_forward(_take_rows(X, rows), A, W2, _take_rows(R, rows), gamma, P, p, sync_idx,
                        eps=eps, private_scale=private_scale, return_all=return_all)
+
+
+def layer_compute_ops(h: float, s: float, r: float) -> float:
+    """Per-device GEMM operations of one transformer layer's forward (App. C, Eq. 31-32):
+    MLP (h -> 4h, 4h -> h) 16 s h^2, attention (qkv, scores and values, out) 4 s^2 h + 8 s h^2,
+    a product of m x p by p x n counted as 2 m p n; split over r tensor-parallel devices."""
+    mlp = 8 * s * h * h + 8 * s * h * h
+    attention = 6 * s * h * h + 4 * s * s * h + 2 * s * h * h
+    return (mlp + attention) / r
+
+
+def layer_exchange(h: float, s: float, p: float) -> float:
+    """Activations each device sends and receives per layer (App. C, Eq. 32): two all-reduces
+    of s h activations, of which the partial all-reduce keeps the fraction p."""
+    return 2 * s * h * p
+
+
+def speedup_model(h: float, s: float, r: float, p: float, C: float):
+    """App. C Eq. 33-35 from the definitions: T(p) = G + C P(p) with C the ratio of compute
+    to communication capacity (FLOP per exchanged activation), speed-up (T(1) - T(p)) / T(1),
+    and p* = the p at which C P(p) = G, capped at 1.  Returns (speedup, p_star)."""
+    G = layer_compute_ops(h, s, r)
+    T = lambda q: G + C * layer_exchange(h, s, q)  # noqa: E731
+    p_star = min(G / (C * layer_exchange(h, s, 1.0)), 1.0)
+    return (T(1.0) - T(p)) / T(1.0), p_star
 
 
 def within_tolerance(got, ref, atol: float = 2e-2, rtol: float = 1e-2):

@@ -45,7 +45,7 @@ EXPORTS = [
     "caat_rowpar_forward_noalloc", "caat_mlp_forward", "caat_mlp_forward_ex",
     "caat_workspace_size", "caat_sync_mask", "caat_get_device_status", "caat_timing_create",
     "caat_timing_destroy", "caat_timing_reset", "caat_timing_read", "caat_status_string",
-    "caat_version", "caat_permute_weights",
+    "caat_version", "caat_permute_weights", "caat_speedup_model",
 ]
 
 
@@ -107,6 +107,8 @@ def lib() -> ctypes.CDLL:
     L.caat_workspace_size.argtypes = [i64, i64, i64, ctypes.c_int, ctypes.c_int]
     L.caat_workspace_size.restype = sz
     L.caat_sync_mask.argtypes = [i64, dbl, vp, vp, ctypes.POINTER(i64)]
+    L.caat_speedup_model.restype = ctypes.c_int
+    L.caat_speedup_model.argtypes = [dbl, dbl, dbl, dbl, dbl, ctypes.POINTER(dbl), ctypes.POINTER(dbl)]
     L.caat_permute_weights.restype = ctypes.c_int
     L.caat_permute_weights.argtypes = [vp, vp, vp, dbl, ctypes.c_int, i64, i64, vp]
     L.caat_sync_mask.restype = ctypes.c_int
@@ -192,6 +194,14 @@ def caat_sync_mask(H: int, p: float, sync_idx=None):
     code = lib().caat_sync_mask(int(H), float(p), ptr, mask.ctypes.data, ctypes.byref(ns))
     _check(code, "caat_sync_mask")
     return mask, int(ns.value)
+
+
+def caat_speedup_model(h: float, s: float, r: float, p: float, C: float):
+    """(speedup, p_star) of the paper's model (App. C Eq. 34-35); host only."""
+    sp, ps = ctypes.c_double(0.0), ctypes.c_double(0.0)
+    _check(lib().caat_speedup_model(float(h), float(s), float(r), float(p), float(C), ctypes.byref(sp),
+                                    ctypes.byref(ps)), "caat_speedup_model")
+    return sp.value, ps.value
 
 
 def caat_permute_weights(W, W_out, sync_idx, P: int, p: float, stream=None):

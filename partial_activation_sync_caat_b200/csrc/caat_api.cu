@@ -754,6 +754,17 @@ caat_status caat_sync_mask(int64_t H, double p, const int32_t* sync_idx, uint8_t
   return CAAT_OK;
 }
 
+caat_status caat_speedup_model(double h, double s, double r, double p, double C, double* speedup_out,
+                               double* p_star_out) {
+  if (!(h > 0.0) || !(s > 0.0) || !(r > 0.0) || !(C > 0.0) || !(p >= 0.0 && p <= 1.0) || !std::isfinite(h) ||
+      !std::isfinite(s) || !std::isfinite(r) || !std::isfinite(C))
+    return CAAT_ERR_INVALID_ARG;
+  const double x = (12.0 * h + 2.0 * s) / (C * r);
+  if (speedup_out) *speedup_out = (1.0 - p) / (1.0 + x);
+  if (p_star_out) *p_star_out = std::min(x, 1.0);
+  return CAAT_OK;
+}
+
 caat_status caat_permute_weights(const caat_bf16* W, caat_bf16* W_out, const int32_t* sync_idx, double p, int P,
                                  int64_t H, int64_t K, caat_stream_t stream) {
   caat_status s = check_shapes(0, K, H, P, p);
