@@ -41,6 +41,9 @@ WORKLOADS = {
     "decode-1": (1, 11008, 4096, 8, 0.5, False),
     "decode-8": (8, 11008, 4096, 8, 0.5, False),
     "decode-64": (64, 11008, 4096, 8, 0.5, False),
+    # attention output projection (App. A.1 Eq. 24): the same row-parallel layer with
+    # K = heads x head_dim = 4096 (Llama-2-7B: 32 heads of 128), 4 heads per rank
+    "attn-out-7b": (8192, 4096, 4096, 8, 0.5, False),
 }
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -124,7 +127,9 @@ def alg_bytes_of(T, K, H, P, mlp=False):
 
 
 def workload_desc(name, T, K, H, P, p, rand):
-    return (f"{name}: partially synced row-parallel FC2 + residual + RMSNorm, T={T} H={H} K={K} P={P} "
+    layer = ("attention output projection (K = heads x head_dim)" if name.startswith("attn")
+             else "row-parallel FC2")
+    return (f"{name}: partially synced {layer} + residual + RMSNorm, T={T} H={H} K={K} P={P} "
             f"p={p} ({'seeded random' if rand else 'contiguous'} S)")
 
 

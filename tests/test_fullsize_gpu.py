@@ -73,3 +73,14 @@ def test_decode_shapes_full(T):
     out = _run(to_dev(d), 8, 0.5)
     ref = O.rowpar_forward(d["X"], d["W"], d["R"], d["gamma"], 8, 0.5)
     assert_out_close(out, ref, f"decode T={T}")
+
+
+def test_attention_out_projection_7b_sampled():
+    """The attention output projection of App. A.1 Eq. 24 is the same row-parallel layer with
+    X_m = rank m's head outputs and K = heads x head_dim: Llama-2-7B shape (32 heads of 128,
+    4 per rank), T = 8192, H = 4096, P = 8, p = 0.5, checked on sampled rows."""
+    d = I.make_rowpar_inputs(8192, 4096, 4096, 8, seed=4000, x_std=1.0, w_std=0.02, r_std=1.0)
+    out = _run(to_dev(d), 8, 0.5)
+    rows = I.sample_rows(8192, 24, seed=11)
+    ref = O.rowpar_rows(d["X"], d["W"], d["R"], d["gamma"], 8, 0.5, rows)
+    assert_out_close(out[:, torch.as_tensor(rows), :], ref, "attention out-projection 7B")
