@@ -17,7 +17,9 @@ Karnieli, Hanani, Giladi, Soudry; arXiv 2506.19645):
 * residual add and norm: §4 Eq. 9 and App. B Eq. 25 (X_m = Norm(sum Z + R)); the norm is
   RMSNorm here, with gamma shared by the ranks (§4: norm parameters are synchronized);
 * MLP block: §3.1 Eq. 6 (Y_m = sigma(X_m A_m), column-parallel A) with sigma = SwiGLU;
-* speed-up model: App. C Eq. 31-35 (compute and exchange per layer, T(p), speed-up, p*).
+* speed-up model: App. C Eq. 31-35 (compute and exchange per layer, T(p), speed-up, p*);
+* backward: §4 Eq. 10-13 (the reduction over ranks follows the norm derivative; the shared
+  norm weight's gradient is summed over the ranks), chain rule through Eq. 22 and Eq. 9.
 
 Everything is plain NumPy float64: one library matmul per partial product, no blocking,
 fusion or reordering beyond the definitions above.  The inputs are the bf16 tensors
@@ -125,6 +127,52 @@ def rowpar_forward(X, W, R, gamma, P: int, p: float, sync_idx=None, *, eps: floa
     if return_all:
         return {"Zt": Zt, "Z": Z, "h": h, "out": out, "mask": mask}
     return out
+
+
+def rmsnorm_backward(h: np.ndarray, gamma, dout: np.ndarray, eps: float):
+    """Backward of out = h / sqrt(mean(h^2) + eps) * gamma over the last axis, per row:
+    with r = 1 / sqrt(mean(h^2) + eps), xhat = h r and g = dout * gamma,
+    dh = r (g - xhat mean(g xhat)) and dgamma_row = dout * xhat.  Returns (dh, dout * xhat)."""
+    gamma = _f64(gamma)
+    r = 1.0 / np.sqrt(np.mean(h * h, axis=-1, keepdims=True) + np.float64(eps))
+    xhat = h * r
+    g = dout * gamma
+    dh = r * (g - xhat * np.mean(g * xhat, axis=-1, keepdims=True))
+    return dh, dout * xhat
+
+
+def partial_channel_reduce_backward(dZ: np.ndarray, mask: np.ndarray, private_scale: float = 1.0) -> np.ndarray:
+    """Transpose of partial_channel_reduce: a shared channel of every rank's partial receives
+    the sum over ranks of dZ (the reduction after the norm derivative, §4 Eq. 10-11: the 'h'
+    operation of Fig. 2b), a private channel private_scale times its own rank's dZ."""
+    dZt = dZ * np.float64(private_scale)
+    dZt[:, :, mask] = dZ[:, :, mask].sum(axis=0)[None, :, :]
+    return dZt
+
+
+def rowpar_backward(X, W, h, gamma, dout, P: int, p: float, sync_idx=None, *, eps: float = 1e-5,
+                    private_scale: float = 1.0):
+    """Gradients of rowpar_forward given dL/d(out) [P,T,H] and the pre-norm stream h the
+    forward produced (h = Z + R).  The chain rule, step by step:
+      RMSNorm per rank (§4 Eq. 9)         -> dh, and dgamma summed over ranks and tokens
+                                             (gamma is shared: its gradient is reduced over
+                                             the ranks, §4 Eq. 12-13)
+      residual add h = Z + R              -> dR = dZ = dh
+      partial channel-reduce (Eq. 22)     -> dZt (shared: sum over ranks; private: scale x own)
+      partial products Zt_m = X_m W_m^T   -> dX_m = dZt_m W_m, dW_m = dZt_m^T X_m
+    Returns a dict with dX [P,T,K/P], dW [P,H,K/P], dR [P,T,H], dgamma [H] and dZt."""
+    X = _f64(X)
+    W = _f64(W)
+    h = _f64(h)
+    dout = _f64(dout)
+    if X.shape[0] != P or W.shape[0] != P or h.shape[0] != P:
+        raise ValueError("leading dimension must be P")
+    mask = sync_mask(W.shape[1], p, sync_idx)
+    dh, dg_rows = rmsnorm_backward(h, gamma, dout, eps)
+    dZt = partial_channel_reduce_backward(dh, mask, private_scale)
+    dX = np.stack([dZt[m] @ W[m] for m in range(P)])
+    dW = np.stack([dZt[m].T @ X[m] for m in range(P)])
+    return {"dX": dX, "dW": dW, "dR": dh, "dgamma": dg_rows.sum(axis=(0, 1)), "dZt": dZt}
 
 
 def silu(x: np.ndarray) -> np.ndarray:
