@@ -279,7 +279,7 @@ def run_caat(args):
     # A random sync list: W's output channels are permuted once (as at weight load time) so
     # that the shared channels are contiguous; every step then runs the permuted path.
     user_flags = args.flags
-    permute = rand and not mlp and not args.no_permute
+    permute = rand and not mlp and not args.no_permute and not args.backward
     permute_ms = None
     if permute:
         Wp = torch.empty_like(d["W"])
@@ -294,8 +294,25 @@ def run_caat(args):
         d["W"] = Wp
         args.flags |= C.CAAT_FLAG_W_PERMUTED
 
+    bwd = args.backward and not mlp
+    if bwd:
+        # the layer's backward: the forward's h and a random dout are its inputs
+        permute = False
+        h_saved = torch.empty_like(d["R"])
+        C.caat_rowpar_forward(d["X"], d["W"], d["R"], d["gamma"], sync_idx, P, p, out, workspace=ws, h_out=h_saved)
+        gen = torch.Generator(device="cuda").manual_seed(rank_seed(rank) + 7)
+        dout = torch.randn(d["R"].shape, generator=gen, device="cuda").to(torch.bfloat16)
+        dX_b, dW_b, dR_b = torch.empty_like(d["X"]), torch.empty_like(d["W"]), torch.empty_like(d["R"])
+        dg_b = torch.empty(H, dtype=torch.float32, device="cuda")
+        ws_b = C.alloc_workspace(C.caat_workspace_size(T, K, H, P, C.CAAT_VARIANT_ROWPAR_BWD), "cuda")
+        flops = 4.0 * T * K * H
+
     def step(tm=None, st=None):
         st = stream if st is None else st
+        if bwd:
+            C.caat_rowpar_backward(d["X"], d["W"], h_saved, d["gamma"], dout, sync_idx, P, p, dX_b, dW_b, dg_b,
+                                   dR=dR_b, workspace=ws_b, stream=st, timing=tm)
+            return
         if mlp:
             C.caat_mlp_forward(d["X"], d["A"], d["W2"], d["R"], d["gamma"], sync_idx, P, p, out, workspace=ws,
                                stream=st, timing=tm, flags=args.flags)
@@ -370,7 +387,7 @@ def run_caat(args):
 
     # optional p sweep (same shapes, fewer steps), rank 0 only
     sweep = None
-    if args.sweep and rank == 0 and not mlp and not permute:   # W is permuted for one (p, S) only
+    if args.sweep and rank == 0 and not mlp and not permute and not bwd:   # W permuted for one (p, S) only
         sweep = {}
         for ps in (0.0, 0.25, 0.5, 0.75, 1.0):
             idx_s = I.random_sync_idx(H, int((H * ps) // 1), seed=0) if rand else None
@@ -391,7 +408,7 @@ def run_caat(args):
 
     # end to end through the host-buffer entry point (pinned host tensors, copies timed)
     e2e = None
-    if not args.no_e2e and not mlp:
+    if not args.no_e2e and not mlp and not bwd:
         hX, hW, hR, hg = (d[k].cpu().pin_memory() for k in ("X", "W", "R", "gamma"))
         hout = torch.empty(hR.shape, dtype=torch.bfloat16).pin_memory()
         wsh = C.alloc_workspace(C.caat_workspace_size(T, K, H, P, C.CAAT_VARIANT_ROWPAR_HOST), "cuda")
@@ -496,6 +513,20 @@ def run_caat(args):
                                    "C_inputs": f"{peaks['bf16_tflops']} TFLOP/s {peak_src} bf16 / "
                                                f"({nvlink_gbs} GB/s NVLink per direction / 2 B)",
                                    "speedup_vs_full_sync": round(sp_m, 4), "p_star": round(ps_m, 4)}
+    if bwd:
+        names = ["rownorm_bwd_kernel (norm backward + reduction over ranks)", "dgamma_reduce_kernel",
+                 "transpose W", "GEMM dX = dZt W", "transpose dZt", "transpose X", "GEMM dW = dZt^T X"]
+        result["metric"] = "TFLOP/s of the partially-synced row-parallel layer's backward (dX + dW, 4 T K H flop)"
+        result["backward_kernels_ms"] = {n: round(x, 4) for n, x in zip(names, kernel_ms)}
+        if len(kernel_ms) >= 7:
+            gx, gw = kernel_ms[3], kernel_ms[6]
+            result["roofline"] = {"kernel": "rowpar_gemm_pair_kernel as the batched dX GEMM", "bound": "tensor",
+                                  "achieved": round(fc2_flops / gx / 1e9, 1), "peak": peaks["bf16_tflops"],
+                                  "peak_source": f"{peak_src} bf16 burst", "unit": "TFLOP/s",
+                                  "frac": round(fc2_flops / gx / 1e9 / peaks["bf16_tflops"], 3),
+                                  "traffic": None, "launch_ms": round(gx, 4), "algorithmic": "2*T*K*H flops",
+                                  "dW_gemm_tflops": round(fc2_flops / gw / 1e9, 1)}
+        result.pop("norm_kernel", None)
     if permute:
         result["w_permuted"] = {"api": "caat_permute_weights, once before the steps (weights are static)",
                                 "once_ms": round(permute_ms, 4)}
@@ -503,7 +534,7 @@ def run_caat(args):
         result["p_sweep"] = sweep
     if e2e is not None:
         result["e2e"] = e2e
-    if not args.no_cpu_baseline:
+    if not args.no_cpu_baseline and not bwd:
         result["cpu_baseline"] = cpu_baseline(T, K, H, P, p, sync_idx, target_s=args.cpu_seconds)
     print(json.dumps(result))
 
@@ -569,6 +600,8 @@ def main():
                     help="random sync list: run on the original W (mixed tiles) instead of permuting it once")
     ap.add_argument("--flags", type=lambda x: int(x, 0), default=0, help="CAAT_FLAG_* bits (tuning variants)")
     ap.add_argument("--sweep", action="store_true", help="also time p in {0,.25,.5,.75,1}")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the layer's backward (caat_rowpar_backward) instead of the forward")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)

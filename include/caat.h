@@ -69,6 +69,7 @@ typedef enum caat_status {
 #define CAAT_VARIANT_ROWPAR 0 /* caat_rowpar_forward[_ex]; K = FFN dim */
 #define CAAT_VARIANT_MLP 1    /* caat_mlp_forward[_ex]; K = F */
 #define CAAT_VARIANT_ROWPAR_HOST 2 /* caat_rowpar_forward_host; K = FFN dim */
+#define CAAT_VARIANT_ROWPAR_BWD 4  /* caat_rowpar_backward; K = FFN dim */
 
 /* Flags of caat_rowpar_args.flags / caat_mlp_args.flags. */
 #define CAAT_FLAG_FORCE_GEMM_PATH 0x1u   /* use the tensor-core GEMM path even for small T */
@@ -228,6 +229,49 @@ typedef struct caat_mlp_args {
 } caat_mlp_args;
 
 CAAT_API caat_status caat_mlp_forward_ex(const caat_mlp_args* args);
+
+/*
+ * caat_rowpar_backward - gradients of the row-parallel layer (forward: caat_rowpar_forward)
+ * for training, §4 Eq. 10-13 and Fig. 2b: the RMSNorm derivative per rank first, THEN the
+ * reduction over ranks of the shared channels' gradients (fp32 accumulation, §4 "32 bit
+ * gradient accumulation"), the private scale on the private channels, then the partial
+ * products' gradients dX_m = dZt_m W_m and dW_m = dZt_m^T X_m (tcgen05 GEMMs); the shared
+ * RMSNorm weight's gradient is summed over ranks and tokens (§4 Eq. 12-13).
+ *
+ *   X, W, gamma, sync_idx, p, P, T, K, H, eps, private_scale  as in the forward call
+ *   h        device bf16 [P, T, H]: the pre-norm stream of the forward (its h_out)
+ *   dout     device bf16 [P, T, H]: dL/d(out)
+ *   dX       device bf16 [P, T, K/P]   (out)
+ *   dW       device bf16 [P, H, K/P]   (out)
+ *   dR       device bf16 [P, T, H] or NULL: dL/d(residual) = dL/dh  (out)
+ *   dgamma   device fp32 [H]            (out)
+ *   workspace caat_workspace_size(T, K, H, P, CAAT_VARIANT_ROWPAR_BWD) bytes, 256-byte aligned
+ * Requires P <= 16 and H <= 8192.  Outputs must not overlap the inputs.  Asynchronous.
+ */
+typedef struct caat_rowpar_bwd_args {
+  const caat_bf16* X;
+  const caat_bf16* W;
+  const caat_bf16* h;
+  const caat_bf16* gamma;
+  const caat_bf16* dout;
+  const int32_t* sync_idx;     /* host */
+  caat_bf16* dX;
+  caat_bf16* dW;
+  caat_bf16* dR;
+  float* dgamma;
+  void* workspace;
+  size_t ws_bytes;
+  caat_stream_t stream;
+  caat_timing* timing;         /* optional: events around each of the backward's kernels */
+  int64_t T, K, H;
+  double p;
+  float eps;
+  float private_scale;
+  int32_t P;
+  uint32_t flags;              /* reserved, 0 */
+} caat_rowpar_bwd_args;
+
+CAAT_API caat_status caat_rowpar_backward(const caat_rowpar_bwd_args* args);
 
 /*
  * caat_permute_weights - reorders the output channels (rows) of W for a sync set: with

@@ -26,6 +26,7 @@ CAAT_ERR_WORKSPACE = 5
 CAAT_VARIANT_ROWPAR = 0
 CAAT_VARIANT_MLP = 1
 CAAT_VARIANT_ROWPAR_HOST = 2
+CAAT_VARIANT_ROWPAR_BWD = 4
 
 CAAT_FLAG_FORCE_GEMM_PATH = 0x1
 CAAT_FLAG_FORCE_DECODE_PATH = 0x2
@@ -45,7 +46,7 @@ EXPORTS = [
     "caat_rowpar_forward_noalloc", "caat_mlp_forward", "caat_mlp_forward_ex",
     "caat_workspace_size", "caat_sync_mask", "caat_get_device_status", "caat_timing_create",
     "caat_timing_destroy", "caat_timing_reset", "caat_timing_read", "caat_status_string",
-    "caat_version", "caat_permute_weights", "caat_speedup_model",
+    "caat_version", "caat_permute_weights", "caat_speedup_model", "caat_rowpar_backward",
 ]
 
 
@@ -62,6 +63,18 @@ class RowparArgs(ctypes.Structure):
         ("h_out", ctypes.c_void_p), ("workspace", ctypes.c_void_p), ("ws_bytes", ctypes.c_size_t),
         ("stream", ctypes.c_void_p), ("timing", ctypes.c_void_p),
         ("T", ctypes.c_int64), ("K", ctypes.c_int64), ("H", ctypes.c_int64),
+        ("p", ctypes.c_double), ("eps", ctypes.c_float), ("private_scale", ctypes.c_float),
+        ("P", ctypes.c_int32), ("flags", ctypes.c_uint32),
+    ]
+
+
+class BwdArgs(ctypes.Structure):
+    _fields_ = [
+        ("X", ctypes.c_void_p), ("W", ctypes.c_void_p), ("h", ctypes.c_void_p), ("gamma", ctypes.c_void_p),
+        ("dout", ctypes.c_void_p), ("sync_idx", ctypes.c_void_p), ("dX", ctypes.c_void_p),
+        ("dW", ctypes.c_void_p), ("dR", ctypes.c_void_p), ("dgamma", ctypes.c_void_p),
+        ("workspace", ctypes.c_void_p), ("ws_bytes", ctypes.c_size_t), ("stream", ctypes.c_void_p),
+        ("timing", ctypes.c_void_p), ("T", ctypes.c_int64), ("K", ctypes.c_int64), ("H", ctypes.c_int64),
         ("p", ctypes.c_double), ("eps", ctypes.c_float), ("private_scale", ctypes.c_float),
         ("P", ctypes.c_int32), ("flags", ctypes.c_uint32),
     ]
@@ -107,6 +120,8 @@ def lib() -> ctypes.CDLL:
     L.caat_workspace_size.argtypes = [i64, i64, i64, ctypes.c_int, ctypes.c_int]
     L.caat_workspace_size.restype = sz
     L.caat_sync_mask.argtypes = [i64, dbl, vp, vp, ctypes.POINTER(i64)]
+    L.caat_rowpar_backward.restype = ctypes.c_int
+    L.caat_rowpar_backward.argtypes = [ctypes.POINTER(BwdArgs)]
     L.caat_speedup_model.restype = ctypes.c_int
     L.caat_speedup_model.argtypes = [dbl, dbl, dbl, dbl, dbl, ctypes.POINTER(dbl), ctypes.POINTER(dbl)]
     L.caat_permute_weights.restype = ctypes.c_int
@@ -271,6 +286,40 @@ def caat_rowpar_forward(X, W, residual, gamma, sync_idx, P: int, p: float, out, 
     return out
 
 
+def caat_rowpar_backward(X, W, h, gamma, dout, sync_idx, P: int, p: float, dX, dW, dgamma, *, dR=None,
+                         workspace=None, eps: float = 1e-5, private_scale: float = 1.0, stream=None, timing=None):
+    """Queues the backward of the layer: dX [P,T,K/P], dW [P,H,K/P] (bf16), dgamma [H] (fp32)
+    and optionally dR [P,T,H] (bf16), from the forward's inputs, its pre-norm stream h and
+    dout = dL/d(out)."""
+    P = int(P)
+    T = int(X.shape[1])
+    K = int(X.shape[2]) * P
+    H = int(W.shape[1])
+    if workspace is None:
+        workspace = alloc_workspace(caat_workspace_size(T, K, H, P, CAAT_VARIANT_ROWPAR_BWD), X.device)
+    arr, idx_ptr = _sync_idx_host(sync_idx)
+    a = BwdArgs()
+    a.X, a.W, a.h = _bf16_dev(X, "X"), _bf16_dev(W, "W"), _bf16_dev(h, "h")
+    a.gamma, a.dout = _bf16_dev(gamma, "gamma"), _bf16_dev(dout, "dout")
+    a.sync_idx = idx_ptr
+    a.dX, a.dW = _bf16_dev(dX, "dX"), _bf16_dev(dW, "dW")
+    a.dR = _bf16_dev(dR, "dR") if dR is not None else None
+    if dgamma.dtype.__str__() != "torch.float32" or not dgamma.is_cuda:
+        raise TypeError("dgamma must be a float32 CUDA tensor")
+    a.dgamma = _ptr(dgamma)
+    a.workspace = _ptr(workspace)
+    a.ws_bytes = workspace.numel() * workspace.element_size()
+    a.stream = _stream_ptr(stream)
+    a.timing = timing.handle if timing is not None else None
+    a.T, a.K, a.H = T, K, H
+    a.p = float(p)
+    a.eps = float(eps)
+    a.private_scale = float(private_scale)
+    a.P = P
+    a.flags = 0
+    _check(lib().caat_rowpar_backward(ctypes.byref(a)), "caat_rowpar_backward")
+
+
 def caat_rowpar_forward_host(X, W, residual, gamma, sync_idx, P: int, p: float, out, workspace, *,
                              h_out=None, eps: float = 1e-5, private_scale: float = 1.0, flags: int = 0,
                              stream=None, timing=None):
@@ -384,7 +433,7 @@ def caat_get_device_status(stream=None) -> int:
 class Timing:
     """Per-kernel CUDA-event recorder of the library (caat_timing_*)."""
 
-    MAX_KERNELS = 4
+    MAX_KERNELS = 8
 
     def __init__(self, capacity: int = 256):
         h = ctypes.c_void_p()

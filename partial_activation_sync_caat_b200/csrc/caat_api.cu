@@ -18,6 +18,7 @@
 #include "rowpar_gemm.cuh"
 #include "rowpar_gemm2.cuh"
 #include "fc1_swiglu.cuh"
+#include "backward.cuh"
 #include "decode.cuh"
 #include "permuted.cuh"
 #include "rownorm.cuh"
@@ -67,6 +68,8 @@ caat_status device_info(DeviceInfo** out) {
                                caat::K3_SMEM_BYTES) != cudaSuccess ||
           cudaFuncSetAttribute(caat::decode_partials_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                caat::K4_SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(caat::rownorm_bwd_smem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(caat::KB_SMEM_MAX)) != cudaSuccess ||
           cudaFuncSetAttribute(caat::rownorm_gather_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(caat::gather_smem_bytes(1024))) != cudaSuccess ||
           cudaFuncSetAttribute(caat::rownorm_gather_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -212,6 +215,10 @@ caat_status build_mask(int64_t H, double p, const int32_t* sync_idx, std::vector
 }
 
 constexpr size_t kCounterBytes = 256;
+
+// Internal (not in caat.h): run only the GEMM kernel of the row-parallel path, storing the
+// per-rank products without residual or norm -- a batched GEMM C_b = A_b B_b^T (p = 0, P = b).
+constexpr uint32_t kFlagGemmOnly = 0x40000000u;
 
 size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
 
@@ -383,7 +390,7 @@ MlpWs mlp_ws_layout(int64_t T, int64_t H, int64_t F, int P, bool fused) {
 // ---------------------------------------------------------------------------------------
 struct caat_timing {
   int capacity = 0;
-  int max_kernels = 4;
+  int max_kernels = 8;
   int n = 0;
   std::vector<cudaEvent_t> ev;
   std::vector<int> nk;
@@ -514,7 +521,8 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
   static thread_local RowparParams prm;  // ~10 KiB: keep it off the stack
   std::memset(&prm, 0, sizeof(prm));
   const bool fused = (a->flags & CAAT_FLAG_FUSED_NORM) != 0;
-  prm.no_residual = permuted ? 1 : 0;
+  const bool gemm_only = (a->flags & kFlagGemmOnly) != 0;
+  prm.no_residual = (permuted || gemm_only) ? 1 : 0;
   const RowparWs wl = rowpar_ws_layout(T, H, P, fused);
   uint8_t* wsb = reinterpret_cast<uint8_t*>(counter);
   prm.R = reinterpret_cast<const __nv_bfloat16*>(a->residual);
@@ -671,12 +679,13 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
   Recorder own;
   Recorder& rec = outer ? *outer : own;
   if (!outer) rec.begin(a->timing, st);
-  const bool overlap = !fused && !permuted && (a->flags & CAAT_FLAG_OVERLAP_NORM) && T >= 2 * kNormChunk;
+  const bool overlap =
+      !fused && !permuted && !gemm_only && (a->flags & CAAT_FLAG_OVERLAP_NORM) && T >= 2 * kNormChunk;
   if (!overlap) {
     s = gemm(0, T);
     if (s != CAAT_OK) return s;
     rec.after_kernel(st);
-    if (fused) return CAAT_OK;
+    if (fused || gemm_only) return CAAT_OK;
     s = norm(0, T, st, int64_t(dev->sm_count) * 4);
     if (s != CAAT_OK) return s;
     rec.after_kernel(st);
@@ -722,6 +731,72 @@ caat_status validate_rowpar(const caat_rowpar_args* a, std::vector<uint8_t>& mas
   return CAAT_OK;
 }
 
+
+// ---------------------------------------------------------------------------------------
+// Backward
+// ---------------------------------------------------------------------------------------
+// Workspace of caat_rowpar_backward: [GEMM counters (256 B) | dZt [P,T,H] | dZt^T [P,H,Tp] |
+// X^T [P,K/P,Tp] | W^T [P,K/P,H] | dgamma partials [nb, H] fp32], Tp = T rounded up to 8.
+struct BwdLayout {
+  size_t dzt, dztT, xT, wT, dg, total;
+  int64_t Tp;
+  int nb;
+};
+
+BwdLayout bwd_layout(int64_t T, int64_t K, int64_t H, int P, int sm_count) {
+  BwdLayout L{};
+  const int64_t Kp = K / P;
+  L.Tp = (T + 7) / 8 * 8;
+  L.nb = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(T, sm_count)));
+  L.dzt = kCounterBytes;
+  L.dztT = L.dzt + align256(size_t(P) * T * H * 2);
+  L.xT = L.dztT + align256(size_t(P) * H * L.Tp * 2);
+  L.wT = L.xT + align256(size_t(P) * Kp * L.Tp * 2);
+  L.dg = L.wT + align256(size_t(P) * Kp * H * 2);
+  L.total = L.dg + align256(size_t(L.nb) * H * 4);
+  return L;
+}
+
+// Largest SM count the backward workspace is sized for (the dgamma partials: one row per CTA).
+constexpr int kBwdMaxCtas = 1024;
+
+caat_status launch_transpose(const void* in, void* out, int64_t nbatch, int64_t R, int64_t C, int64_t Rp,
+                             cudaStream_t st) {
+  const dim3 grid(static_cast<unsigned>((C + caat::KT_TILE - 1) / caat::KT_TILE),
+                  static_cast<unsigned>((Rp + caat::KT_TILE - 1) / caat::KT_TILE), static_cast<unsigned>(nbatch));
+  caat::transpose_pad_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(in),
+                                                   reinterpret_cast<__nv_bfloat16*>(out), R, C, Rp);
+  return cudaGetLastError() == cudaSuccess ? CAAT_OK : CAAT_ERR_CUDA;
+}
+
+// C_b = A_b B_b^T for b < nb: A [nb, M, Kr], B [nb, N, Kr] (K-major), C [nb, M, N] bf16, through
+// the row-parallel GEMM kernel with every channel private (p = 0) and no residual.
+caat_status launch_batched_gemm(const void* A, const void* B, void* Cm, int nb, int64_t M, int64_t N, int64_t Kr,
+                                unsigned int* counter, cudaStream_t st, const DeviceInfo* dev, Recorder* rec) {
+  caat_rowpar_args g;
+  std::memset(&g, 0, sizeof(g));
+  g.X = reinterpret_cast<const caat_bf16*>(A);
+  g.W = reinterpret_cast<const caat_bf16*>(B);
+  g.residual = reinterpret_cast<const caat_bf16*>(Cm);
+  g.gamma = reinterpret_cast<const caat_bf16*>(Cm);
+  g.out = reinterpret_cast<caat_bf16*>(Cm);
+  g.h_out = reinterpret_cast<caat_bf16*>(Cm);
+  g.workspace = counter;
+  g.ws_bytes = kCounterBytes;
+  g.stream = st;
+  g.T = M;
+  g.K = Kr * nb;
+  g.H = N;
+  g.p = 0.0;
+  g.eps = 1e-5f;
+  g.private_scale = 1.0f;
+  g.P = nb;
+  g.flags = CAAT_FLAG_FORCE_GEMM_PATH | kFlagGemmOnly;
+  static thread_local std::vector<uint8_t> zero_mask;
+  zero_mask.assign(static_cast<size_t>(N), 0);
+  return launch_rowpar(&g, zero_mask, dev, counter, rec);
+}
+
 }  // namespace
 
 // =======================================================================================
@@ -752,6 +827,78 @@ caat_status caat_sync_mask(int64_t H, double p, const int32_t* sync_idx, uint8_t
   if (mask_out) std::memcpy(mask_out, mask.data(), static_cast<size_t>(H));
   if (n_sync_out) *n_sync_out = ns;
   return CAAT_OK;
+}
+
+caat_status caat_rowpar_backward(const caat_rowpar_bwd_args* a) {
+  if (!a) return CAAT_ERR_INVALID_ARG;
+  caat_status s = check_shapes(a->T, a->K, a->H, a->P, a->p);
+  if (s != CAAT_OK) return s;
+  if (!(a->eps >= 0.f) || !std::isfinite(a->eps) || !std::isfinite(a->private_scale)) return CAAT_ERR_INVALID_ARG;
+  if (a->P > caat::KB_MAXP || a->H > int64_t(8) * caat::KB_THREADS * caat::KB_VEC) return CAAT_ERR_UNSUPPORTED;
+  std::vector<uint8_t> mask;
+  s = build_mask(a->H, a->p, a->sync_idx, mask, nullptr);
+  if (s != CAAT_OK) return s;
+  if (a->T == 0) return CAAT_OK;
+  if (!a->X || !a->W || !a->h || !a->gamma || !a->dout || !a->dX || !a->dW || !a->dgamma)
+    return CAAT_ERR_INVALID_ARG;
+  if (!aligned16(a->X) || !aligned16(a->W) || !aligned16(a->h) || !aligned16(a->gamma) || !aligned16(a->dout) ||
+      !aligned16(a->dX) || !aligned16(a->dW) || !aligned16(a->dgamma) || (a->dR && !aligned16(a->dR)))
+    return CAAT_ERR_UNSUPPORTED;
+  DeviceInfo* dev = nullptr;
+  s = device_info(&dev);
+  if (s != CAAT_OK) return s;
+  if (dev->sm_count > kBwdMaxCtas) return CAAT_ERR_UNSUPPORTED;
+  const int P = a->P;
+  const int64_t T = a->T, H = a->H, Kp = a->K / P;
+  const BwdLayout L = bwd_layout(T, a->K, H, P, dev->sm_count);
+  if (!a->workspace || a->ws_bytes < L.total || (reinterpret_cast<uintptr_t>(a->workspace) & 255u))
+    return CAAT_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(a->workspace);
+  unsigned int* counter = reinterpret_cast<unsigned int*>(ws);
+  cudaStream_t st = a->stream;
+  Recorder rec;
+  rec.begin(a->timing, st);
+
+  static thread_local caat::BwdParams bp;
+  std::memset(&bp, 0, sizeof(bp));
+  bp.h = reinterpret_cast<const __nv_bfloat16*>(a->h);
+  bp.dout = reinterpret_cast<const __nv_bfloat16*>(a->dout);
+  bp.gamma = reinterpret_cast<const __nv_bfloat16*>(a->gamma);
+  bp.dR = reinterpret_cast<__nv_bfloat16*>(a->dR);
+  bp.dZt = reinterpret_cast<__nv_bfloat16*>(ws + L.dzt);
+  bp.dg_part = reinterpret_cast<float*>(ws + L.dg);
+  bp.P = P;
+  bp.H = static_cast<int>(H);
+  bp.T = T;
+  bp.eps = a->eps;
+  bp.private_scale = a->private_scale;
+  for (int64_t c = 0; c < H; ++c)
+    if (mask[c]) bp.mask_bits[c >> 5] |= 1u << (c & 31);
+  const size_t kb_smem = caat::bwd_smem_bytes(P, static_cast<int>(H));
+  if (H <= 8 * caat::KB_THREADS && kb_smem <= caat::KB_SMEM_MAX)
+    caat::rownorm_bwd_smem_kernel<<<L.nb, caat::KB_THREADS, kb_smem, st>>>(bp);
+  else
+    caat::rownorm_bwd_kernel<<<L.nb, caat::KB_THREADS, 0, st>>>(bp);
+  if (cudaGetLastError() != cudaSuccess) return CAAT_ERR_CUDA;
+  rec.after_kernel(st);
+  caat::dgamma_reduce_kernel<<<static_cast<unsigned>((H + 255) / 256), 256, 0, st>>>(bp.dg_part, a->dgamma, L.nb,
+                                                                                     static_cast<int>(H));
+  if (cudaGetLastError() != cudaSuccess) return CAAT_ERR_CUDA;
+  rec.after_kernel(st);
+  // dX_m = dZt_m W_m = dZt_m (W_m^T)^T
+  s = launch_transpose(a->W, ws + L.wT, P, H, Kp, H, st);
+  if (s != CAAT_OK) return s;
+  rec.after_kernel(st);
+  s = launch_batched_gemm(ws + L.dzt, ws + L.wT, a->dX, P, T, Kp, H, counter, st, dev, &rec);
+  if (s != CAAT_OK) return s;
+  // dW_m = dZt_m^T X_m = (dZt^T)_m ((X^T)_m)^T, reduction over the (zero-padded) tokens
+  s = launch_transpose(ws + L.dzt, ws + L.dztT, P, T, H, L.Tp, st);
+  if (s != CAAT_OK) return s;
+  rec.after_kernel(st);
+  s = launch_transpose(a->X, ws + L.xT, P, T, Kp, L.Tp, st);
+  if (s != CAAT_OK) return s;
+  rec.after_kernel(st);
+  return launch_batched_gemm(ws + L.dztT, ws + L.xT, a->dW, P, H, Kp, L.Tp, counter, st, dev, &rec);
 }
 
 caat_status caat_speedup_model(double h, double s, double r, double p, double C, double* speedup_out,
@@ -802,6 +949,7 @@ size_t caat_workspace_size(int64_t T, int64_t K, int64_t H, int P, int variant) 
   if (variant == CAAT_VARIANT_ROWPAR) return rowpar_workspace(T, K, H, P);
   if (variant == CAAT_VARIANT_ROWPAR_HOST) return host_layout(T, K, H, P).total;
   if (variant == CAAT_VARIANT_MLP) return mlp_ws_layout(T, H, K, P, true).total;
+  if (variant == CAAT_VARIANT_ROWPAR_BWD) return bwd_layout(T, K, H, P, kBwdMaxCtas).total;
   return SIZE_MAX;
 }
 
