@@ -304,23 +304,27 @@ __global__ void dgamma_reduce_kernel(const float* __restrict__ part, float* __re
 
 // KB3: batched transpose of bf16 matrices, in [B][R][C] -> out [B][C][Rp], out[b][c][r] =
 // in[b][r][c] for r < R and 0 for R <= r < Rp (the zero tail makes the reduction length of the
-// GEMM that reads it a multiple of 8).  64 x 64 tiles through shared memory; 16-byte loads
-// and stores.  C % 8 == 0 and Rp % 8 == 0.
-constexpr int KT_TILE = 64;
-constexpr int KT_PITCH = 72;  // u16 per shared row (16-byte aligned rows)
-__global__ void __launch_bounds__(256) transpose_pad_kernel(const __nv_bfloat16* __restrict__ in,
-                                                            __nv_bfloat16* __restrict__ out, int64_t R,
-                                                            int64_t C, int64_t Rp) {
-  __shared__ __align__(16) uint16_t tile[KT_TILE][KT_PITCH];
+// GEMM that reads it a multiple of 8).  KT_ROWS x KT_COLS tiles through shared memory; 16-byte
+// loads (a warp reads 4 rows x 128 bytes) and 16-byte stores (a warp reads one shared row
+// segment of 32 consecutive columns: no bank conflicts).  C % 8 == 0 and Rp % 8 == 0.
+constexpr int KT_ROWS = 128;
+constexpr int KT_COLS = 64;
+constexpr int KT_PITCH = KT_COLS + 8;  // u16 per shared row (16-byte aligned rows)
+constexpr int KT_THREADS = 256;
+__global__ void __launch_bounds__(KT_THREADS) transpose_pad_kernel(const __nv_bfloat16* __restrict__ in,
+                                                                   __nv_bfloat16* __restrict__ out, int64_t R,
+                                                                   int64_t C, int64_t Rp) {
+  __shared__ __align__(16) uint16_t tile[KT_ROWS][KT_PITCH];
   const int64_t b = blockIdx.z;
-  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * KT_TILE;
-  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * KT_TILE;
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * KT_COLS;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * KT_ROWS;
   const __nv_bfloat16* src = in + b * R * C;
   __nv_bfloat16* dst = out + b * C * Rp;
+  constexpr int VPR = KT_COLS / 8;  // 16-byte vectors per tile row
 #pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const int idx = threadIdx.x + i * 256;  // 64 rows x 8 vectors
-    const int rr = idx >> 3, vv = idx & 7;
+  for (int i = 0; i < KT_ROWS * VPR / KT_THREADS; ++i) {
+    const int idx = threadIdx.x + i * KT_THREADS;
+    const int rr = idx / VPR, vv = idx % VPR;
     const int64_t r = r0 + rr, c = c0 + 8 * vv;
     uint4 v = make_uint4(0, 0, 0, 0);
     if (r < R && c < C) v = *reinterpret_cast<const uint4*>(src + r * C + c);
@@ -328,9 +332,9 @@ __global__ void __launch_bounds__(256) transpose_pad_kernel(const __nv_bfloat16*
   }
   __syncthreads();
 #pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const int idx = threadIdx.x + i * 256;  // 8 vectors of r x 64 out rows (c); a warp reads one
-    const int cc = idx & 63, vv = idx >> 6;  // shared row segment (32 consecutive columns)
+  for (int i = 0; i < KT_COLS * (KT_ROWS / 8) / KT_THREADS; ++i) {
+    const int idx = threadIdx.x + i * KT_THREADS;
+    const int cc = idx % KT_COLS, vv = idx / KT_COLS;
     const int64_t c = c0 + cc, r = r0 + 8 * vv;
     if (c < C && r < Rp) {
       uint32_t w[4];

@@ -762,9 +762,9 @@ constexpr int kBwdMaxCtas = 1024;
 
 caat_status launch_transpose(const void* in, void* out, int64_t nbatch, int64_t R, int64_t C, int64_t Rp,
                              cudaStream_t st) {
-  const dim3 grid(static_cast<unsigned>((C + caat::KT_TILE - 1) / caat::KT_TILE),
-                  static_cast<unsigned>((Rp + caat::KT_TILE - 1) / caat::KT_TILE), static_cast<unsigned>(nbatch));
-  caat::transpose_pad_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(in),
+  const dim3 grid(static_cast<unsigned>((C + caat::KT_COLS - 1) / caat::KT_COLS),
+                  static_cast<unsigned>((Rp + caat::KT_ROWS - 1) / caat::KT_ROWS), static_cast<unsigned>(nbatch));
+  caat::transpose_pad_kernel<<<grid, caat::KT_THREADS, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(in),
                                                    reinterpret_cast<__nv_bfloat16*>(out), R, C, Rp);
   return cudaGetLastError() == cudaSuccess ? CAAT_OK : CAAT_ERR_CUDA;
 }

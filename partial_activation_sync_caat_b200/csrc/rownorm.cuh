@@ -99,7 +99,9 @@ __global__ void __launch_bounds__(K2_THREADS, 2)
   const float inv_h = 1.0f / static_cast<float>(H);
   const uint4* g4 = reinterpret_cast<const uint4*>(gamma);
 
-  for (int64_t i = warp_global; i < rows; i += nwarps) {
+  // Rows in reverse order: the rows the GEMM wrote last (rank P-1's) may still be in L2.
+  for (int64_t i0 = warp_global; i0 < rows; i0 += nwarps) {
+    const int64_t i = rows - 1 - i0;
     const int64_t r = i / tc;
     const int64_t row = r * T + t0 + (i - r * tc);
     const uint4* hp = reinterpret_cast<const uint4*>(h + row * H);
