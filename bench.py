@@ -90,15 +90,20 @@ def load_peaks():
 
 
 def kernel_source_hash() -> str:
-    """sha256 over the CUDA sources of the library (file names and bytes, sorted by name)."""
+    """sha256 over the sources of the forward GEMM and norm kernels: their headers and the
+    forward launch code of caat_api.cu (from launch_rowpar up to validate_rowpar)."""
     import hashlib
     h = hashlib.sha256()
     d = os.path.join(ROOT, "partial_activation_sync_caat_b200", "csrc")
-    for f in sorted(os.listdir(d)):
-        if f.endswith((".cu", ".cuh", ".h")):
-            h.update(f.encode())
-            with open(os.path.join(d, f), "rb") as fh:
-                h.update(fh.read())
+    for f in ("ptx.cuh", "rowpar_common.cuh", "rowpar_gemm.cuh", "rowpar_gemm2.cuh", "rownorm.cuh"):
+        h.update(f.encode())
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(fh.read())
+    with open(os.path.join(d, "caat_api.cu"), "rb") as fh:
+        api = fh.read()
+    a = api.find(b"caat_status launch_rowpar(")
+    b = api.find(b"caat_status validate_rowpar(")
+    h.update(api[a:b] if 0 <= a < b else api)
     return h.hexdigest()
 
 
