@@ -191,6 +191,22 @@ CAAT_API caat_status caat_rowpar_forward_host(const caat_rowpar_args* args);
 CAAT_API caat_status caat_rowpar_forward_noalloc(const caat_rowpar_args* args);
 
 /*
+ * Plans: the graph-capture-friendly form of caat_rowpar_forward_ex for calls repeated on the
+ * same buffers (a decode loop, a layer in a captured step).  caat_plan_create validates the
+ * arguments and builds the sync mask once, binding every pointer, size and option of `args`
+ * (which is copied; sync_idx is read before return); caat_plan_execute then only queues the
+ * kernels on `stream` (it allocates nothing and never synchronizes, so it can be captured in
+ * a CUDA graph once the device's first call has been made outside capture).  The buffers
+ * must stay valid for the plan's lifetime.  A plan is host memory owned by the caller
+ * through the handle; executing one plan on two streams at once races on its workspace.
+ * No counterpart in the paper.
+ */
+typedef struct caat_plan caat_plan;
+CAAT_API caat_status caat_plan_create(const caat_rowpar_args* args, caat_plan** plan_out);
+CAAT_API caat_status caat_plan_execute(const caat_plan* plan, caat_stream_t stream);
+CAAT_API caat_status caat_plan_destroy(caat_plan* plan);
+
+/*
  * caat_mlp_forward - the MLP block per rank: column-parallel FC1 with SwiGLU (§3.1 Eq. 6),
  * then the partially synchronized FC2 (App. A.2 Eq. 22), residual add and RMSNorm (Eq. 9).
  *

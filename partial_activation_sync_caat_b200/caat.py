@@ -47,6 +47,7 @@ EXPORTS = [
     "caat_workspace_size", "caat_sync_mask", "caat_get_device_status", "caat_timing_create",
     "caat_timing_destroy", "caat_timing_reset", "caat_timing_read", "caat_status_string",
     "caat_version", "caat_permute_weights", "caat_speedup_model", "caat_rowpar_backward",
+    "caat_plan_create", "caat_plan_execute", "caat_plan_destroy",
 ]
 
 
@@ -120,6 +121,12 @@ def lib() -> ctypes.CDLL:
     L.caat_workspace_size.argtypes = [i64, i64, i64, ctypes.c_int, ctypes.c_int]
     L.caat_workspace_size.restype = sz
     L.caat_sync_mask.argtypes = [i64, dbl, vp, vp, ctypes.POINTER(i64)]
+    L.caat_plan_create.restype = ctypes.c_int
+    L.caat_plan_create.argtypes = [ctypes.POINTER(RowparArgs), ctypes.POINTER(vp)]
+    L.caat_plan_execute.restype = ctypes.c_int
+    L.caat_plan_execute.argtypes = [vp, vp]
+    L.caat_plan_destroy.restype = ctypes.c_int
+    L.caat_plan_destroy.argtypes = [vp]
     L.caat_rowpar_backward.restype = ctypes.c_int
     L.caat_rowpar_backward.argtypes = [ctypes.POINTER(BwdArgs)]
     L.caat_speedup_model.restype = ctypes.c_int
@@ -284,6 +291,49 @@ def caat_rowpar_forward(X, W, residual, gamma, sync_idx, P: int, p: float, out, 
     a.flags = int(flags)
     _check(lib().caat_rowpar_forward_ex(ctypes.byref(a)), "caat_rowpar_forward")
     return out
+
+
+class Plan:
+    """A caat_plan: the row-parallel call with its buffers bound once; execute() only queues
+    the kernels.  The tensors given at creation must outlive the plan (they are kept here)."""
+
+    def __init__(self, X, W, residual, gamma, sync_idx, P: int, p: float, out, *, workspace=None, h_out=None,
+                 eps: float = 1e-5, private_scale: float = 1.0, flags: int = 0):
+        P = int(P)
+        T, K, H = int(X.shape[1]), int(X.shape[2]) * P, int(W.shape[1])
+        if workspace is None:
+            workspace = alloc_workspace(caat_workspace_size(T, K, H, P, CAAT_VARIANT_ROWPAR), X.device)
+        self._keep = (X, W, residual, gamma, out, h_out, workspace)
+        arr, idx_ptr = _sync_idx_host(sync_idx)
+        a = RowparArgs()
+        a.X, a.W = _bf16_dev(X, "X"), _bf16_dev(W, "W")
+        a.residual, a.gamma = _bf16_dev(residual, "residual"), _bf16_dev(gamma, "gamma")
+        a.sync_idx = idx_ptr
+        a.out = _bf16_dev(out, "out")
+        a.h_out = _bf16_dev(h_out, "h_out") if h_out is not None else None
+        a.workspace = _ptr(workspace)
+        a.ws_bytes = workspace.numel() * workspace.element_size()
+        a.stream = None
+        a.timing = None
+        a.T, a.K, a.H = T, K, H
+        a.p, a.eps, a.private_scale, a.P, a.flags = float(p), float(eps), float(private_scale), P, int(flags)
+        h = ctypes.c_void_p(None)
+        _check(lib().caat_plan_create(ctypes.byref(a), ctypes.byref(h)), "caat_plan_create")
+        self.handle = h.value
+
+    def execute(self, stream=None):
+        _check(lib().caat_plan_execute(self.handle, _stream_ptr(stream)), "caat_plan_execute")
+
+    def close(self):
+        if self.handle:
+            lib().caat_plan_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 def caat_rowpar_backward(X, W, h, gamma, dout, sync_idx, P: int, p: float, dX, dW, dgamma, *, dR=None,

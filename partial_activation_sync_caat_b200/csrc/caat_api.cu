@@ -11,6 +11,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <new>
 #include <vector>
 
 #include "caat.h"
@@ -962,6 +963,56 @@ caat_status caat_rowpar_forward_ex(const caat_rowpar_args* a) {
   s = device_info(&dev);
   if (s != CAAT_OK) return s;
   return launch_rowpar(a, mask, dev, static_cast<unsigned int*>(a->workspace));
+}
+
+}  // extern "C"
+
+struct caat_plan {
+  caat_rowpar_args args;
+  std::vector<uint8_t> mask;
+  DeviceInfo* dev = nullptr;
+  int device = 0;
+};
+
+extern "C" {
+
+caat_status caat_plan_create(const caat_rowpar_args* a, caat_plan** plan_out) {
+  if (!plan_out) return CAAT_ERR_INVALID_ARG;
+  *plan_out = nullptr;
+  std::vector<uint8_t> mask;
+  caat_status s = validate_rowpar(a, mask);
+  if (s != CAAT_OK) return s;
+  caat_plan* pl = new (std::nothrow) caat_plan();
+  if (!pl) return CAAT_ERR_INVALID_ARG;
+  pl->args = *a;
+  pl->args.sync_idx = nullptr;  // the mask below replaces it
+  pl->args.timing = nullptr;
+  pl->mask = std::move(mask);
+  if (a->T > 0) {
+    s = device_info(&pl->dev);
+    if (s != CAAT_OK || cudaGetDevice(&pl->device) != cudaSuccess) {
+      delete pl;
+      return s != CAAT_OK ? s : CAAT_ERR_CUDA;
+    }
+  }
+  *plan_out = pl;
+  return CAAT_OK;
+}
+
+caat_status caat_plan_execute(const caat_plan* pl, caat_stream_t stream) {
+  if (!pl) return CAAT_ERR_INVALID_ARG;
+  if (pl->args.T == 0) return CAAT_OK;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return CAAT_ERR_CUDA;
+  if (dev != pl->device) return CAAT_ERR_INVALID_ARG;  // created for another device
+  caat_rowpar_args a = pl->args;
+  a.stream = stream;
+  return launch_rowpar(&a, pl->mask, pl->dev, static_cast<unsigned int*>(a.workspace));
+}
+
+caat_status caat_plan_destroy(caat_plan* pl) {
+  delete pl;
+  return CAAT_OK;
 }
 
 caat_status caat_rowpar_forward_host(const caat_rowpar_args* a) {

@@ -144,3 +144,24 @@ def test_permute_weights_rejects_invalid_arguments_without_device_work(L):
     assert call(Wo=0x100000 + 768 * 768) == C.CAAT_ERR_INVALID_ARG  # overlaps W (W is 768*768*2 bytes)
     bad = np.array([5, 3], dtype=np.int32)
     assert call(H=8, K=16, p=0.25, idx=bad.ctypes.data) == C.CAAT_ERR_INVALID_ARG
+
+
+def test_plan_validation_without_device_work(L):
+    a = C.RowparArgs()
+    a.X, a.W, a.residual, a.gamma, a.out = 0x10000, 0x20000, 0x30000, 0x40000, 0x50000
+    a.workspace, a.ws_bytes = 0x60000, 1 << 20
+    a.T, a.K, a.H, a.P, a.p, a.eps, a.private_scale = 128, 256, 256, 2, 0.5, 1e-5, 1.0
+    h = ctypes.c_void_p(None)
+    a.P = 0
+    assert L.caat_plan_create(ctypes.byref(a), ctypes.byref(h)) == C.CAAT_ERR_INVALID_ARG and h.value is None
+    a.P, a.ws_bytes = 2, 0
+    assert L.caat_plan_create(ctypes.byref(a), ctypes.byref(h)) == C.CAAT_ERR_WORKSPACE and h.value is None
+    assert L.caat_plan_create(None, ctypes.byref(h)) == C.CAAT_ERR_INVALID_ARG
+    assert L.caat_plan_create(ctypes.byref(a), None) == C.CAAT_ERR_INVALID_ARG
+    assert L.caat_plan_execute(None, None) == C.CAAT_ERR_INVALID_ARG
+    assert L.caat_plan_destroy(None) == C.CAAT_OK
+    # an empty call plans and executes as a no-op without a device
+    a.T, a.X, a.W, a.residual, a.gamma, a.out, a.workspace = 0, None, None, None, None, None, None
+    assert L.caat_plan_create(ctypes.byref(a), ctypes.byref(h)) == C.CAAT_OK and h.value
+    assert L.caat_plan_execute(h, None) == C.CAAT_OK
+    assert L.caat_plan_destroy(h) == C.CAAT_OK

@@ -108,3 +108,43 @@ def test_call_captured_in_cuda_graph(T):
         assert C.caat_get_device_status() == 0
         assert torch.equal(out.cpu(), o_ref) and torch.equal(hb.cpu(), h_ref)
     del graph
+
+
+@pytest.mark.parametrize("T,rand", [(1, False), (300, False), (300, True)])
+def test_plan_execute_matches_forward_and_captures(T, rand):
+    """A plan (buffers bound once) gives the forward call's bits, again after its buffers'
+    contents change, and inside a CUDA graph; with a random sync list also on permuted W."""
+    P, K, H, p = 4, 1024, 1032, 0.5
+    d = I.make_rowpar_inputs(T, K, H, P, seed=60 + T, x_std=1.0, w_std=0.05, r_std=1.0, gamma="uniform")
+    idx = I.random_sync_idx(H, O.n_sync(H, p), seed=3) if rand else None
+    g = to_dev(d)
+    flags = 0
+    if rand:
+        Wp = torch.empty_like(g["W"])
+        C.caat_permute_weights(g["W"], Wp, idx, P, p)
+        g["W"], flags = Wp, C.CAAT_FLAG_W_PERMUTED
+    ref_out, ref_h = torch.empty_like(g["R"]), torch.empty_like(g["R"])
+    C.caat_rowpar_forward(g["X"], g["W"], g["R"], g["gamma"], idx, P, p, ref_out, h_out=ref_h, flags=flags)
+    out, hb = torch.empty_like(g["R"]), torch.empty_like(g["R"])
+    plan = C.Plan(g["X"], g["W"], g["R"], g["gamma"], idx, P, p, out, h_out=hb, flags=flags)
+    plan.execute()
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref_out) and torch.equal(hb, ref_h)
+    # new contents in the bound buffers
+    g["X"].copy_(torch.flip(g["X"], dims=[1]))
+    C.caat_rowpar_forward(g["X"], g["W"], g["R"], g["gamma"], idx, P, p, ref_out, h_out=ref_h, flags=flags)
+    plan.execute()
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref_out) and torch.equal(hb, ref_h)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        plan.execute(stream=torch.cuda.current_stream())
+    out.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert C.caat_get_device_status() == 0
+    assert torch.equal(out, ref_out)
+    del graph
+    plan.close()
+    ref = O.rowpar_forward(d["X"].flip(1), d["W"], d["R"], d["gamma"], P, p, idx)
+    assert_out_close(out.cpu(), ref, "plan")
