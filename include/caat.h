@@ -158,7 +158,8 @@ CAAT_API caat_status caat_rowpar_forward_ex(const caat_rowpar_args* args);
  * for asynchronous copies; pageable memory also works, with synchronous staging).
  * args->workspace is a device buffer of caat_workspace_size(T, K, H, P,
  * CAAT_VARIANT_ROWPAR_HOST) bytes that receives device copies of the inputs and outputs.
- * The call is pipelined over chunks of 1024 tokens (token rows are independent): W and gamma
+ * The call is pipelined over chunks of 1024 tokens, the last ones halving down to 256 (token
+ * rows are independent; a small last chunk keeps the final copy back short): W and gamma
  * are copied once, then each chunk's X and residual rows are copied in, its kernels run on
  * args->stream and its out (and h_out) rows are copied back, on two library-owned copy
  * streams (created on the first call on a device) so that both copy directions overlap the

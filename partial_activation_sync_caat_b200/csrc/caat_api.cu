@@ -1053,11 +1053,24 @@ caat_status caat_rowpar_forward_host(const caat_rowpar_args* a) {
       cudaEventRecord(hp->ev_w, hp->s_in) || cudaStreamWaitEvent(st, hp->ev_w, 0))
     return CAAT_ERR_CUDA;
 
-  const int64_t nch = (T + L.Tc - 1) / L.Tc;
+  // Chunks of L.Tc tokens, the last ones halving (to 256): the copy back of the final chunk
+  // is the pipeline's tail, after every upload and kernel.  No chunk is left below 256 tokens
+  // (a remainder that small joins the chunk before it), so every chunk of a multi-chunk call
+  // takes the GEMM path, whose workspace the per-chunk region is sized for.
+  std::vector<int64_t> starts;
+  for (int64_t t0 = 0; t0 < T;) {
+    const int64_t rem = T - t0;
+    int64_t tc = rem >= 2 * L.Tc ? L.Tc : std::max<int64_t>(256, (rem / 2 + 255) / 256 * 256);
+    if (rem - tc < 256) tc = rem;
+    starts.push_back(t0);
+    t0 += tc;
+  }
+  starts.push_back(T);
+  const int64_t nch = static_cast<int64_t>(starts.size()) - 1;
   for (int64_t i = 0; i < nch; ++i) {
     const int b = static_cast<int>(i & 1);
-    const int64_t t0 = i * L.Tc;
-    const int64_t tc = std::min<int64_t>(L.Tc, T - t0);
+    const int64_t t0 = starts[i];
+    const int64_t tc = starts[i + 1] - t0;
     uint8_t* buf = base + L.buf0 + size_t(b) * L.buf_bytes;
     // H2D of the chunk's X and R rows (P strided blocks each)
     if (i >= 2 && cudaStreamWaitEvent(hp->s_in, hp->ev_comp[b], 0)) return CAAT_ERR_CUDA;

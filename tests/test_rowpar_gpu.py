@@ -190,9 +190,10 @@ def test_stall_reports_timeout_and_context_survives(flags):
 
 
 # ------------------------------------------------------------------ host-buffer entry point
-@pytest.mark.parametrize("T", [300, 2500])
+@pytest.mark.parametrize("T", [300, 1060, 2500])
 def test_host_buffer_entry_matches_device_entry(T):
-    """caat_rowpar_forward_host (pipelined over 1024-token chunks: 1 or 3 chunks here) gives
+    """caat_rowpar_forward_host (pipelined over chunks of up to 1024 tokens, the last ones
+    smaller, none below 256: 300 -> one chunk, 1060 -> 768 + 292, 2500 -> 1024 + 768 + 708) gives
     the same bits as the device entry point: rows are independent and every kernel is
     deterministic per row."""
     P, K, H = 4, 1024, 776
