@@ -671,8 +671,17 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
       else
         caat::rownorm_reg_kernel<16><<<rb, caat::K2_THREADS, 0, ns>>>(hdst, o, g, P, T, t0, tc, static_cast<int>(H), a->eps);
     } else {
-      caat::rownorm_kernel<<<blocks, caat::K2_THREADS, 0, ns>>>(hdst, o, g, P, T, t0, tc, static_cast<int>(H),
-                                                                a->eps);
+      // wide rows: one CTA per row (H <= 65536 = 8 x 1024 x 8)
+      const int64_t nb = std::min<int64_t>(rows, int64_t(dev->sm_count) * 8);
+      const int Hi = static_cast<int>(H);
+      if (H <= 8 * 256 * 4)
+        caat::rownorm_block_kernel<256, 4><<<nb, 256, 0, ns>>>(hdst, o, g, P, T, t0, tc, Hi, a->eps);
+      else if (H <= 8 * 512 * 4)
+        caat::rownorm_block_kernel<512, 4><<<nb, 512, 0, ns>>>(hdst, o, g, P, T, t0, tc, Hi, a->eps);
+      else if (H <= 8 * 1024 * 4)
+        caat::rownorm_block_kernel<1024, 4><<<nb, 1024, 0, ns>>>(hdst, o, g, P, T, t0, tc, Hi, a->eps);
+      else
+        caat::rownorm_block_kernel<1024, 8><<<nb, 1024, 0, ns>>>(hdst, o, g, P, T, t0, tc, Hi, a->eps);
     }
     return cudaGetLastError() == cudaSuccess ? CAAT_OK : CAAT_ERR_CUDA;
   };

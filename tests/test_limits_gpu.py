@@ -74,3 +74,16 @@ def test_backward_limits():
                           ("dW", dW, np.stack([(ref["dZt"][m] ** 2).T @ (O._f64(d["X"][m]) ** 2) for m in range(P)]))):
         err = np.abs(O._f64(got.cpu()) - ref[name])
         assert (err <= 8e-3 * np.sqrt(sq) + 4e-3 * np.abs(ref[name]) + 1e-6).all(), name
+
+
+@pytest.mark.parametrize("H", [8192, 12288, 24576])
+def test_wide_rows_norm(H):
+    """H > 4096: the norm runs one CTA per row (256, 512 or 1024 threads) with the row in
+    registers; ragged T, contiguous and listed sync sets."""
+    T, K, P, p = 300, 256, 2, 0.5
+    d = I.make_rowpar_inputs(T, K, H, P, seed=H, x_std=1.0, w_std=0.05, r_std=1.0, gamma="uniform")
+    for idx in (None, I.random_sync_idx(H, O.n_sync(H, p), seed=2)):
+        out, h = run_rowpar(d, P, p, idx)
+        ref = O.rowpar_forward(d["X"], d["W"], d["R"], d["gamma"], P, p, idx, return_all=True)
+        assert_h_close(h, ref["h"], f"h H={H}")
+        assert_out_close(out, ref["out"], f"H={H}")
