@@ -17,6 +17,9 @@
  *     ranks, since norm parameters are synchronized, §4).
  *   - MLP block (§3.1 Eq. 6 with sigma = SwiGLU): Y_m = silu(X_m A_gate,m^T) * (X_m A_up,m^T),
  *     then the layer above with X := Y.
+ *   - Backward of the layer (§4 Eq. 10-13): the norm derivative per rank, then the reduction
+ *     over ranks of the shared channels' gradients, then the gradients of the partial products.
+ *   - Speed-up model of partial synchronization (App. C Eq. 31-35), host only.
  *
  * Conventions for every call below
  *   - bf16 tensors are raw bfloat16 bit patterns (caat_bf16), row-major, last dim contiguous.
@@ -26,8 +29,9 @@
  *   - Every forward call validates all arguments on the host first; an invalid call queues
  *     no work and returns an error code.  No call throws across the ABI.
  *   - Work is queued asynchronously on `stream` (a cudaStream_t; NULL = legacy default).
- *   - Device-side waits are bounded: a wait that runs out (about 1 s) records
- *     CAAT_ERR_TIMEOUT in a device status word, which caat_get_device_status() reads.
+ *   - Device-side waits are bounded: a wait that runs out (2 s; the environment variable
+ *     CAAT_TIMEOUT_MS overrides) records CAAT_ERR_TIMEOUT in a device status word, which
+ *     caat_get_device_status() reads.
  */
 #ifndef CAAT_H_
 #define CAAT_H_
@@ -116,10 +120,15 @@ typedef enum caat_status {
  *   P, p      ranks (1..CAAT_MAX_P) and sync factor p in [0, 1]; n_s = floor(H p) in double.
  *   out       device, bf16 [P, T, H]     normalized output; may alias `residual`.
  *   T, K, H   tokens (>= 0), FFN dim (K % P == 0, (K/P) % 8 == 0), hidden (H % 8 == 0).
- *   workspace device scratch of caat_workspace_size(T, K, H, P, CAAT_VARIANT_ROWPAR) bytes
- *             (about 32 (2 ceil(H/256)) P T bytes: row-block counters and per-row partial
- *             sums of squares of the fused RMSNorm), 256-byte aligned; its contents need not
- *             be initialized and are clobbered.
+ *   workspace device scratch, 256-byte aligned; contents need not be initialized and are
+ *             clobbered.  caat_workspace_size(T, K, H, P, CAAT_VARIANT_ROWPAR) bytes enable
+ *             every path: the fused norm's row-block counters and per-row partial sums of
+ *             squares (about 64 ceil(H/256) P T bytes), the completion flags that give
+ *             column blocks mixing shared and private channels the TMA epilogue (T/8
+ *             ceil(H/256) bytes), the decode path's fp32 partials (4 P T H bytes, T <= 64).
+ *             The separate-norm GEMM path runs with 256 bytes (mixed column blocks then take
+ *             the register epilogue); a smaller workspace than a call needs gives
+ *             CAAT_ERR_WORKSPACE.
  * eps = 1e-5 and private_scale = 1 (use caat_rowpar_forward_ex for other values).
  * Returns CAAT_OK once the work is queued.
  */
