@@ -311,13 +311,21 @@ def run_caat(args):
     if world != args.gpus:
         raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
     torch.cuda.set_device(local)
+    # The library is (re)built by rank 0 before the process group exists, so that a build
+    # (a minute or more of nvcc) never runs into the group's timeout; the other ranks wait
+    # for it (bounded).
+    if rank == 0:
+        B.build()
+    else:
+        t_wait = time.time()
+        while not B.up_to_date():
+            if time.time() - t_wait > 900:
+                raise SystemExit("libcaat.so was not built by rank 0 within 15 minutes")
+            time.sleep(1.0)
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
-    if rank == 0:
-        B.build()
-    if world > 1:
         dist.barrier()
     C.lib()
 
