@@ -46,7 +46,7 @@ def _worker(rank, world, port, out):
 def test_two_gloo_ranks_weak_scaling_helpers():
     world = 2
     port = _free_port()
-    manager = mp.Manager()
+    manager = mp.get_context("spawn").Manager()  # no fork of this (threaded) process
     out = manager.dict()
     mp.start_processes(_worker, args=(world, port, out), nprocs=world, start_method="spawn")
     for rank in range(world):
