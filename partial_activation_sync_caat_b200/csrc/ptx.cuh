@@ -256,6 +256,12 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+// The same two unpacks spelled as byte permutes.  A kernel that unpacks a register-resident row
+// twice (sum of squares, then rescale) uses these for the second pass: with one spelling the
+// compiler keeps the first pass's 2 fp32 values per packed word live across the reduction
+// instead of the packed word, which doubles the row's register footprint and spills.
+__device__ __forceinline__ float bf16lo_p(uint32_t w) { return __uint_as_float(__byte_perm(w, 0u, 0x1044)); }
+__device__ __forceinline__ float bf16hi_p(uint32_t w) { return __uint_as_float(__byte_perm(w, 0u, 0x3244)); }
 
 // ------------------------------------------------------------------------------------------
 // Clusters and CTA pairs (tcgen05 cta_group::2)
