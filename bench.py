@@ -599,12 +599,18 @@ def run_caat(args):
                                                f"({nvlink_gbs} GB/s NVLink per direction / 2 B)",
                                    "speedup_vs_full_sync": round(sp_m, 4), "p_star": round(ps_m, 4)}
     if bwd:
-        names = ["rownorm_bwd_kernel (norm backward + reduction over ranks)", "dgamma_reduce_kernel",
-                 "transpose W", "GEMM dX = dZt W", "transpose dZt", "transpose X", "GEMM dW = dZt^T X"]
+        norm_names = ["rownorm_bwd_kernel (norm backward + reduction over ranks)", "dgamma_reduce_kernel"]
+        if len(kernel_ms) == 4:   # both GEMMs read W, dZt and X MN-major: no transposes
+            names = norm_names + ["GEMM dX = dZt W (W MN-major)", "GEMM dW = dZt^T X (dZt, X MN-major)"]
+            gemm_idx = (2, 3)
+        else:                     # fewer than 129 tokens or channels: K-major operands via transposes
+            names = norm_names + ["transpose W", "GEMM dX = dZt W", "transpose dZt", "transpose X",
+                                  "GEMM dW = dZt^T X"]
+            gemm_idx = (3, 6)
         result["metric"] = "TFLOP/s of the partially-synced row-parallel layer's backward (dX + dW, 4 T K H flop)"
         result["backward_kernels_ms"] = {n: round(x, 4) for n, x in zip(names, kernel_ms)}
-        if len(kernel_ms) >= 7:
-            gx, gw = kernel_ms[3], kernel_ms[6]
+        if len(kernel_ms) > max(gemm_idx):
+            gx, gw = kernel_ms[gemm_idx[0]], kernel_ms[gemm_idx[1]]
             result["roofline"] = {"kernel": "rowpar_gemm_pair_kernel as the batched dX GEMM", "bound": "tensor",
                                   "achieved": round(fc2_flops / gx / 1e9, 1), "peak": peaks["bf16_tflops"],
                                   "peak_source": f"{peak_src} bf16 burst", "unit": "TFLOP/s",

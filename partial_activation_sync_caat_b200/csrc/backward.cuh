@@ -13,8 +13,10 @@
 //   dZt_m[:, c] = sum_q dh_q[:, c]  for c in S     (reduction over ranks, fp32)
 //              = s * dh_m[:, c]    otherwise      (private scale s)
 //   dgamma = sum over ranks and tokens of dout * h * r
-//   dX_m = dZt_m W_m,  dW_m = dZt_m^T X_m          (two batched tcgen05 GEMMs, K-major
-//                                                   operands through transposes below)
+//   dX_m = dZt_m W_m,  dW_m = dZt_m^T X_m          (two batched tcgen05 GEMMs on the CTA-pair
+//                                                   kernel reading W, dZt and X MN-major; the
+//                                                   transposes below serve calls of <= 128
+//                                                   tokens or channels)
 #pragma once
 
 #include "ptx.cuh"

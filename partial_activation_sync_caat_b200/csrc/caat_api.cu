@@ -65,6 +65,10 @@ caat_status device_info(DeviceInfo** out) {
                                caat::K2P_SMEM_BYTES) != cudaSuccess ||
           cudaFuncSetAttribute(caat::rowpar_gemm_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                caat::K2P_SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(caat::rowpar_gemm_pair_kernel<false, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               caat::K2P_SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(caat::rowpar_gemm_pair_kernel<false, 3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               caat::K2P_SMEM_BYTES) != cudaSuccess ||
           cudaFuncSetAttribute(caat::fc1_swiglu_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                caat::K3_SMEM_BYTES) != cudaSuccess ||
           cudaFuncSetAttribute(caat::decode_partials_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -220,6 +224,10 @@ constexpr size_t kCounterBytes = 256;
 // Internal (not in caat.h): run only the GEMM kernel of the row-parallel path, storing the
 // per-rank products without residual or norm -- a batched GEMM C_b = A_b B_b^T (p = 0, P = b).
 constexpr uint32_t kFlagGemmOnly = 0x40000000u;
+// Internal, with kFlagGemmOnly on the CTA-pair kernel: A is stored [b][Kr][M] (M contiguous) /
+// B is stored [b][Kr][N], read MN-major by the tensor cores (no transposed copies).
+constexpr uint32_t kFlagAMn = 0x20000000u;
+constexpr uint32_t kFlagBMn = 0x10000000u;
 
 size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
 
@@ -568,6 +576,8 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
   prm.nslots = prm.nS + prm.nPriv;
   // The CTA-pair kernel (256-token tiles) for all but the smallest token counts.
   const bool pair = !(a->flags & CAAT_FLAG_SINGLE_CTA) && dev->max_pairs > 0 && T > caat::K1_BM;
+  const int major = ((a->flags & kFlagAMn) ? 1 : 0) | ((a->flags & kFlagBMn) ? 2 : 0);
+  if (major != 0 && (!pair || !gemm_only || fused || major == 1)) return CAAT_ERR_UNSUPPORTED;
   const int64_t bm = pair ? 2 * caat::K2P_BM : caat::K1_BM;
   if ((T + bm - 1) / bm * (prm.nS + int64_t(P) * prm.nPriv) > INT32_MAX / 2) return CAAT_ERR_UNSUPPORTED;
   prm.T_pad = static_cast<int>((T + bm - 1) / bm * bm);
@@ -582,9 +592,12 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
   const size_t zero_bytes = merge ? wl.sdone + wl.sdone_bytes : wl.zeroed;
 
   CUtensorMap tmX, tmW, tmR, tmH;
-  caat_status s = make_map_3d(&tmX, a->X, Kp, T, P, caat::K1_BK, caat::K1_BM);
+  // K-major operands: boxes of 64 K x (128 rows); MN-major ones: 64 MN x 64 K rows, two per half
+  caat_status s = (major & 1) ? make_map_3d(&tmX, a->X, T, Kp, P, 64, caat::K2P_BK)
+                              : make_map_3d(&tmX, a->X, Kp, T, P, caat::K1_BK, caat::K1_BM);
   if (s != CAAT_OK) return s;
-  s = make_map_3d(&tmW, a->W, Kp, H, P, caat::K1_BK, pair ? caat::K2P_BN / 2 : caat::K1_BN);
+  s = (major & 2) ? make_map_3d(&tmW, a->W, H, Kp, P, 64, caat::K2P_BK)
+                  : make_map_3d(&tmW, a->W, Kp, H, P, caat::K1_BK, pair ? caat::K2P_BN / 2 : caat::K1_BN);
   if (s != CAAT_OK) return s;
   // residual in / pre-norm h out of the TMA epilogue: 32-row x 64-column boxes
   s = make_map_3d(&tmR, a->residual, H, T, P, 64, 32);
@@ -615,8 +628,10 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
       cfg.attrs = attr;
       cfg.numAttrs = 1;
       const cudaError_t e =
-          fused ? cudaLaunchKernelEx(&cfg, caat::rowpar_gemm_pair_kernel<true>, tmX, tmW, tmR, tmH, prm)
-                : cudaLaunchKernelEx(&cfg, caat::rowpar_gemm_pair_kernel<false>, tmX, tmW, tmR, tmH, prm);
+          fused        ? cudaLaunchKernelEx(&cfg, caat::rowpar_gemm_pair_kernel<true>, tmX, tmW, tmR, tmH, prm)
+          : major == 2 ? cudaLaunchKernelEx(&cfg, caat::rowpar_gemm_pair_kernel<false, 2>, tmX, tmW, tmR, tmH, prm)
+          : major == 3 ? cudaLaunchKernelEx(&cfg, caat::rowpar_gemm_pair_kernel<false, 3>, tmX, tmW, tmR, tmH, prm)
+                       : cudaLaunchKernelEx(&cfg, caat::rowpar_gemm_pair_kernel<false>, tmX, tmW, tmR, tmH, prm);
       if (e != cudaSuccess) return CAAT_ERR_CUDA;
     } else {
       const int grid = static_cast<int>(std::min<int64_t>(dev->sm_count, units));
@@ -779,10 +794,12 @@ caat_status launch_transpose(const void* in, void* out, int64_t nbatch, int64_t 
   return cudaGetLastError() == cudaSuccess ? CAAT_OK : CAAT_ERR_CUDA;
 }
 
-// C_b = A_b B_b^T for b < nb: A [nb, M, Kr], B [nb, N, Kr] (K-major), C [nb, M, N] bf16, through
-// the row-parallel GEMM kernel with every channel private (p = 0) and no residual.
+// C_b = A_b B_b^T for b < nb: A [nb, M, Kr], B [nb, N, Kr] (K-major; with kFlagAMn / kFlagBMn in
+// `major_flags`: A [nb, Kr, M] / B [nb, Kr, N]), C [nb, M, N] bf16, through the row-parallel GEMM
+// kernel with every channel private (p = 0) and no residual.
 caat_status launch_batched_gemm(const void* A, const void* B, void* Cm, int nb, int64_t M, int64_t N, int64_t Kr,
-                                unsigned int* counter, cudaStream_t st, const DeviceInfo* dev, Recorder* rec) {
+                                unsigned int* counter, cudaStream_t st, const DeviceInfo* dev, Recorder* rec,
+                                uint32_t major_flags = 0) {
   caat_rowpar_args g;
   std::memset(&g, 0, sizeof(g));
   g.X = reinterpret_cast<const caat_bf16*>(A);
@@ -801,7 +818,7 @@ caat_status launch_batched_gemm(const void* A, const void* B, void* Cm, int nb, 
   g.eps = 1e-5f;
   g.private_scale = 1.0f;
   g.P = nb;
-  g.flags = CAAT_FLAG_FORCE_GEMM_PATH | kFlagGemmOnly;
+  g.flags = CAAT_FLAG_FORCE_GEMM_PATH | kFlagGemmOnly | major_flags;
   static thread_local std::vector<uint8_t> zero_mask;
   zero_mask.assign(static_cast<size_t>(N), 0);
   return launch_rowpar(&g, zero_mask, dev, counter, rec);
@@ -895,6 +912,16 @@ caat_status caat_rowpar_backward(const caat_rowpar_bwd_args* a) {
                                                                                      static_cast<int>(H));
   if (cudaGetLastError() != cudaSuccess) return CAAT_ERR_CUDA;
   rec.after_kernel(st);
+  if (dev->max_pairs > 0 && T > caat::K1_BM && H > caat::K1_BM) {
+    // Both gradient GEMMs on the CTA-pair kernel with MN-major operands, straight from the
+    // row-major tensors: dX_m = dZt_m W_m (W_m [H][Kp] is B = [Kr=H][N=Kp]); dW_m = dZt_m^T X_m
+    // (dZt_m [T][H] is A = [Kr=T][M=H], X_m [T][Kp] is B = [Kr=T][N=Kp]); the token tail of the
+    // reduction is zero-filled by the tensor maps.
+    s = launch_batched_gemm(ws + L.dzt, a->W, a->dX, P, T, Kp, H, counter, st, dev, &rec, kFlagBMn);
+    if (s != CAAT_OK) return s;
+    return launch_batched_gemm(ws + L.dzt, a->X, a->dW, P, H, Kp, T, counter, st, dev, &rec, kFlagAMn | kFlagBMn);
+  }
+  // Fewer than 129 tokens or channels (the one-CTA kernel, K-major operands only): transposes.
   // dX_m = dZt_m W_m = dZt_m (W_m^T)^T
   s = launch_transpose(a->W, ws + L.wT, P, H, Kp, H, st);
   if (s != CAAT_OK) return s;

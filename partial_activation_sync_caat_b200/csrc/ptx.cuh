@@ -225,12 +225,32 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t smem_addr) {
   return d;
 }
 
+// Shared-memory matrix descriptor of an MN-major operand tile written by TMA with the 128-byte
+// swizzle as 64-element-wide boxes whose rows are K indices: within a box, each K row is 128 B
+// (64 MN elements) and 8 rows form one 1 KiB swizzle atom; the next 64 MN elements sit in the
+// next box.  LBO = distance between MN atoms (one box, 64 K rows x 128 B = 8 KiB), SBO =
+// distance between 8-row K groups (1 KiB).  One K=16 MMA step spans two K groups, so the start
+// address advances by 2 KiB per step.
+__device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>(8192u >> 4) << 16;
+  d |= static_cast<uint64_t>(1024u >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(2u) << 61;
+  return d;
+}
+
 // Instruction descriptor for kind::f16 with bf16 A and B, f32 accumulator, both K-major:
 // c_format [4,6) = 1 (f32), a_format [7,10) = 1 (bf16), b_format [10,13) = 1 (bf16),
 // a/b major bits 15/16 = 0 (K-major), N>>3 at [17,23), M>>4 at [24,29).
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
          (static_cast<uint32_t>(M >> 4) << 24);
+}
+// The same with A (bit 15) and / or B (bit 16) read MN-major.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_major(int M, int N, bool a_mn, bool b_mn) {
+  return idesc_bf16_f32(M, N) | (a_mn ? (1u << 15) : 0u) | (b_mn ? (1u << 16) : 0u);
 }
 
 // ------------------------------------------------------------------------------------------

@@ -17,7 +17,11 @@
 //   * Dynamic scheduling: the leader's producer draws a unit from the global counter and
 //     writes it into both CTAs' broadcast ring.
 // The RMSNorm is fused (rowpar_common.cuh): warps 6-9 of each CTA normalize completed row
-// blocks.  Every wait is bounded; on expiry the device status word is set, all roles leave their
+// blocks.
+// kMajor (GEMM-only use by the backward): bit 0 = A stored MN-major ([K][M], M contiguous),
+// bit 1 = B stored MN-major ([K][N]).  Such an operand half is loaded as two 64-wide boxes of
+// 64 K rows and read through MN-major descriptors, so the gradient GEMMs need no transposes.
+// kMajor = 0 is the forward kernel.  Every wait is bounded; on expiry the device status word is set, all roles leave their
 // loops, copies in flight are given time to land, and both CTAs meet at a final cluster
 // barrier before TMEM is freed.
 #pragma once
@@ -37,7 +41,7 @@ constexpr int K2P_STAGE_BYTES = K2P_A_BYTES + K2P_B_BYTES;
 constexpr int K2P_SMEM_BYTES = 1024 + K2P_STAGES * K2P_STAGE_BYTES + K1_EPI_BYTES + 512;
 constexpr uint64_t K2P_DRAIN_NS = 1000000;      // error path only: let copies in flight land
 
-template <bool kFused>
+template <bool kFused, int kMajor = 0>
 __global__ void __launch_bounds__(K1Threads<kFused>::value, 1)
     rowpar_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                             const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmH,
@@ -133,8 +137,20 @@ __global__ void __launch_bounds__(K1Threads<kFused>::value, 1)
             if (!mbar_wait(&empty[stage], phase ^ 1, tmo, 23)) { ok = false; break; }
             const uint32_t fbar = mapa_shared(smem_u32(&full[stage]), 0);
             if (leader) mbar_arrive_expect_tx(&full[stage], 2 * K2P_STAGE_BYTES);
-            tma_load_3d_pair(sA + stage * K2P_A_BYTES, &tmX, fbar, kb * K2P_BK, xrow, r, pol_x);
-            tma_load_3d_pair(sB + stage * K2P_B_BYTES, &tmW, fbar, kb * K2P_BK, wrow, r, pol_w);
+            if constexpr ((kMajor & 1) != 0) {
+              tma_load_3d_pair(sA + stage * K2P_A_BYTES, &tmX, fbar, xrow, kb * K2P_BK, r, pol_x);
+              tma_load_3d_pair(sA + stage * K2P_A_BYTES + K2P_A_BYTES / 2, &tmX, fbar, xrow + 64, kb * K2P_BK, r,
+                               pol_x);
+            } else {
+              tma_load_3d_pair(sA + stage * K2P_A_BYTES, &tmX, fbar, kb * K2P_BK, xrow, r, pol_x);
+            }
+            if constexpr ((kMajor & 2) != 0) {
+              tma_load_3d_pair(sB + stage * K2P_B_BYTES, &tmW, fbar, wrow, kb * K2P_BK, r, pol_w);
+              tma_load_3d_pair(sB + stage * K2P_B_BYTES + K2P_B_BYTES / 2, &tmW, fbar, wrow + 64, kb * K2P_BK, r,
+                               pol_w);
+            } else {
+              tma_load_3d_pair(sB + stage * K2P_B_BYTES, &tmW, fbar, kb * K2P_BK, wrow, r, pol_w);
+            }
             issued = true;
             if (++stage == K2P_STAGES) { stage = 0; phase ^= 1; }
           }
@@ -145,7 +161,7 @@ __global__ void __launch_bounds__(K1Threads<kFused>::value, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer (leader)
     if (leader && lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(2 * K2P_BM, K2P_BN);
+      const uint32_t idesc = idesc_bf16_f32_major(2 * K2P_BM, K2P_BN, (kMajor & 1) != 0, (kMajor & 2) != 0);
       int stage = 0;
       uint32_t phase = 0;
       int local = 0;
@@ -171,8 +187,9 @@ __global__ void __launch_bounds__(K1Threads<kFused>::value, 1)
           const uint32_t a_addr = smem_u32(sA + stage * K2P_A_BYTES);
           const uint32_t b_addr = smem_u32(sB + stage * K2P_B_BYTES);
           for (int kk = 0; kk < nk16; ++kk) {
-            umma_bf16_pair(dt, sw128_kmajor_desc(a_addr + kk * 32), sw128_kmajor_desc(b_addr + kk * 32), idesc,
-                           (j > 0 || kk > 0) ? 1u : 0u);
+            const uint64_t ad = (kMajor & 1) ? sw128_mnmajor_desc(a_addr + kk * 2048) : sw128_kmajor_desc(a_addr + kk * 32);
+            const uint64_t bd = (kMajor & 2) ? sw128_mnmajor_desc(b_addr + kk * 2048) : sw128_kmajor_desc(b_addr + kk * 32);
+            umma_bf16_pair(dt, ad, bd, idesc, (j > 0 || kk > 0) ? 1u : 0u);
           }
           umma_commit_pair_mc(&empty[stage], 0x3);
           if (++stage == K2P_STAGES) { stage = 0; phase ^= 1; }
