@@ -271,7 +271,10 @@ CAAT_API caat_status caat_mlp_forward_ex(const caat_mlp_args* args);
  *   dW       device bf16 [P, H, K/P]   (out)
  *   dR       device bf16 [P, T, H] or NULL: dL/d(residual) = dL/dh  (out)
  *   dgamma   device fp32 [H]            (out)
- *   workspace caat_workspace_size(T, K, H, P, CAAT_VARIANT_ROWPAR_BWD) bytes, 256-byte aligned
+ *   workspace caat_workspace_size(T, K, H, P, CAAT_VARIANT_ROWPAR_BWD) bytes, 256-byte aligned:
+ *            dZt, per-CTA dgamma partials, and room for transposed copies of W, dZt and X,
+ *            which only calls with T <= 128 or H <= 128 use (larger calls read the three
+ *            tensors in place, MN-major).
  * Requires P <= 16 and H <= 8192.  Outputs must not overlap the inputs.  Asynchronous.
  */
 typedef struct caat_rowpar_bwd_args {
