@@ -297,8 +297,13 @@ typedef struct caat_rowpar_bwd_args {
   float eps;
   float private_scale;
   int32_t P;
-  uint32_t flags;              /* reserved, 0 */
+  uint32_t flags;              /* 0, or CAAT_BWD_FLAG_TRANSPOSED_OPERANDS */
 } caat_rowpar_bwd_args;
+
+/* Test hook: run the gradient GEMMs on transposed K-major copies of W, dZt and X (the path of
+ * calls with T <= 128 or H <= 128) at any size.  The results equal the default path's bit for
+ * bit: same MMA steps on the same values, only the operands' layout in memory differs. */
+#define CAAT_BWD_FLAG_TRANSPOSED_OPERANDS 0x1u
 
 CAAT_API caat_status caat_rowpar_backward(const caat_rowpar_bwd_args* args);
 

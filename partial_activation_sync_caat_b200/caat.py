@@ -27,6 +27,7 @@ CAAT_VARIANT_ROWPAR = 0
 CAAT_VARIANT_MLP = 1
 CAAT_VARIANT_ROWPAR_HOST = 2
 CAAT_VARIANT_ROWPAR_BWD = 4
+CAAT_BWD_FLAG_TRANSPOSED_OPERANDS = 0x1
 
 CAAT_FLAG_FORCE_GEMM_PATH = 0x1
 CAAT_FLAG_FORCE_DECODE_PATH = 0x2
@@ -337,7 +338,8 @@ class Plan:
 
 
 def caat_rowpar_backward(X, W, h, gamma, dout, sync_idx, P: int, p: float, dX, dW, dgamma, *, dR=None,
-                         workspace=None, eps: float = 1e-5, private_scale: float = 1.0, stream=None, timing=None):
+                         workspace=None, eps: float = 1e-5, private_scale: float = 1.0, stream=None, timing=None,
+                         flags: int = 0):
     """Queues the backward of the layer: dX [P,T,K/P], dW [P,H,K/P] (bf16), dgamma [H] (fp32)
     and optionally dR [P,T,H] (bf16), from the forward's inputs, its pre-norm stream h and
     dout = dL/d(out)."""
@@ -366,7 +368,7 @@ def caat_rowpar_backward(X, W, h, gamma, dout, sync_idx, P: int, p: float, dX, d
     a.eps = float(eps)
     a.private_scale = float(private_scale)
     a.P = P
-    a.flags = 0
+    a.flags = int(flags)
     _check(lib().caat_rowpar_backward(ctypes.byref(a)), "caat_rowpar_backward")
 
 

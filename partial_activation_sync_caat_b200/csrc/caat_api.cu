@@ -912,7 +912,7 @@ caat_status caat_rowpar_backward(const caat_rowpar_bwd_args* a) {
                                                                                      static_cast<int>(H));
   if (cudaGetLastError() != cudaSuccess) return CAAT_ERR_CUDA;
   rec.after_kernel(st);
-  if (dev->max_pairs > 0 && T > caat::K1_BM && H > caat::K1_BM) {
+  if (!(a->flags & CAAT_BWD_FLAG_TRANSPOSED_OPERANDS) && dev->max_pairs > 0 && T > caat::K1_BM && H > caat::K1_BM) {
     // Both gradient GEMMs on the CTA-pair kernel with MN-major operands, straight from the
     // row-major tensors: dX_m = dZt_m W_m (W_m [H][Kp] is B = [Kr=H][N=Kp]); dW_m = dZt_m^T X_m
     // (dZt_m [T][H] is A = [Kr=T][M=H], X_m [T][Kp] is B = [Kr=T][N=Kp]); the token tail of the

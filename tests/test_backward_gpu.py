@@ -132,3 +132,24 @@ def test_backward_full_size_fc2_7b_sampled():
     dW_sq = np.stack([(dZt_c[m] ** 2).T @ (Xf[m] ** 2) for m in range(P)])
     _close_gemm(dW[:, torch.as_tensor(chans)], dW_ref, dW_sq, "dW sampled channels")
     _close(dgamma, dg_ref, 1e-3, 1e-3, "dgamma")
+
+
+@pytest.mark.parametrize("T,K,H,P,p,rand", [(300, 2048, 1288, 4, 0.5, False), (600, 1024, 776, 2, 0.0, False),
+                                            (2048, 5632, 2048, 4, 0.5, True)])
+def test_backward_mn_major_equals_transposed_bitwise(T, K, H, P, p, rand):
+    """The gradient GEMMs reading W, dZt and X in place (MN-major) give the same bits as the
+    same GEMMs on transposed K-major copies: identical MMA steps on identical values."""
+    idx = I.random_sync_idx(H, O.n_sync(H, p), seed=T) if rand else None
+    _, g = _setup(T, K, H, P, p, idx, seed=200 + T)
+    outs = []
+    for flags in (0, C.CAAT_BWD_FLAG_TRANSPOSED_OPERANDS):
+        X, W = g["X"], g["W"]
+        dX, dW = torch.empty_like(X), torch.empty_like(W)
+        dR = torch.empty_like(g["R"])
+        dgamma = torch.empty(H, dtype=torch.float32, device="cuda")
+        C.caat_rowpar_backward(X, W, g["h"], g["gamma"], g["dout"], idx, P, p, dX, dW, dgamma, dR=dR, flags=flags)
+        torch.cuda.synchronize()
+        assert C.caat_get_device_status() == 0
+        outs.append((dX, dW, dR, dgamma))
+    for name, a, b in zip(("dX", "dW", "dR", "dgamma"), outs[0], outs[1]):
+        assert torch.equal(a, b), name
