@@ -342,7 +342,8 @@ def caat_rowpar_backward(X, W, h, gamma, dout, sync_idx, P: int, p: float, dX, d
                          flags: int = 0):
     """Queues the backward of the layer: dX [P,T,K/P], dW [P,H,K/P] (bf16), dgamma [H] (fp32)
     and optionally dR [P,T,H] (bf16), from the forward's inputs, its pre-norm stream h and
-    dout = dL/d(out)."""
+    dout = dL/d(out).  flags: 0, or CAAT_BWD_FLAG_TRANSPOSED_OPERANDS (test hook: the gradient
+    GEMMs on transposed K-major copies, bit-identical to the default MN-major reads)."""
     P = int(P)
     T = int(X.shape[1])
     K = int(X.shape[2]) * P
