@@ -33,6 +33,27 @@ def test_header_declares_what_binding_lists():
     assert header_symbols() == sorted(C.EXPORTS)
 
 
+def header_constants():
+    """Every numeric #define and enum value of include/caat.h named CAAT_*."""
+    with open(os.path.join(ROOT, "include", "caat.h")) as f:
+        text = f.read()
+    consts = {}
+    for name, val in re.findall(r"^#define (CAAT_\w+) (0x[0-9a-fA-F]+|\d+)u?\b", text, flags=re.M):
+        consts[name] = int(val, 0)
+    for name, val in re.findall(r"^\s+(CAAT_\w+) = (\d+),?", text, flags=re.M):
+        consts[name] = int(val)
+    return consts
+
+
+def test_binding_constants_match_header():
+    consts = header_constants()
+    assert len(consts) >= 20
+    for name, val in consts.items():
+        if name in ("CAAT_MAX_H", "CAAT_MAX_P", "CAAT_DECODE_MAX_T") and not hasattr(C, name):
+            continue  # limits the binding does not restate
+        assert getattr(C, name) == val, name
+
+
 def test_library_exports_every_declared_symbol(L):
     for name in header_symbols():
         assert hasattr(L, name), name
