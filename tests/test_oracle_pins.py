@@ -280,3 +280,57 @@ def test_pins_catch_planted_mistakes(monkeypatch):
     monkeypatch.setattr(O, "partial_products", wrong_partials)
     res = O.rowpar_forward(X, W, R, np.ones(4), 2, 0.5, return_all=True)
     assert res["Z"][0].tolist() != g["Z1"]
+
+
+# ---------------------------------------------------------------------------------------
+# Helpers: the backward's channel reduce is the adjoint of the forward's; sampled-row
+# evaluation equals the full evaluation restricted to those rows; the pass rule's boundary
+# ---------------------------------------------------------------------------------------
+@pytest.mark.parametrize("P,s", [(1, 1.0), (2, 1.0), (4, 1.5), (8, 0.5)])
+def test_channel_reduce_backward_is_the_adjoint(P, s):
+    rng = np.random.default_rng(P)
+    T, H = 5, 24
+    mask = np.zeros(H, dtype=bool)
+    mask[rng.choice(H, size=H // 3, replace=False)] = True
+    Z = rng.standard_normal((P, T, H))
+    G = rng.standard_normal((P, T, H))
+    lhs = float(np.sum(O.partial_channel_reduce(Z, mask, s) * G))
+    rhs = float(np.sum(Z * O.partial_channel_reduce_backward(G, mask, s)))
+    assert lhs == pytest.approx(rhs, rel=1e-12, abs=1e-12)
+    # and as a matrix: the backward is the transpose of the forward's linear map
+    n = P * T * H
+    F = np.stack([O.partial_channel_reduce(e.reshape(P, T, H), mask, s).ravel() for e in np.eye(n)], axis=1)
+    Bm = np.stack([O.partial_channel_reduce_backward(e.reshape(P, T, H), mask, s).ravel() for e in np.eye(n)],
+                  axis=1)
+    assert np.array_equal(F.T, Bm)
+
+
+def test_sampled_rows_equal_the_full_layer_restricted():
+    T, K, H, P, p = 12, 64, 40, 4, 0.5
+    d = I.make_rowpar_inputs(T, K, H, P, seed=5, x_std=1.0, w_std=0.1, r_std=1.0, gamma="uniform")
+    idx = I.random_sync_idx(H, O.n_sync(H, p), seed=1)
+    rows = np.array([0, 3, 7, 11])
+    full = O.rowpar_forward(d["X"], d["W"], d["R"], d["gamma"], P, p, idx, private_scale=1.5)
+    part = O.rowpar_rows(d["X"], d["W"], d["R"], d["gamma"], P, p, rows, idx, private_scale=1.5)
+    assert np.array_equal(part, full[:, rows, :])
+    m = I.make_mlp_inputs(T, 32, 48, P, seed=6, x_std=1.0, w_std=0.1)
+    full = O.mlp_forward(m["X"], m["A"], m["W2"], m["R"], m["gamma"], P, p)
+    part = O.mlp_rows(m["X"], m["A"], m["W2"], m["R"], m["gamma"], P, p, rows)
+    assert np.array_equal(part, full[:, rows, :])
+
+
+def test_within_tolerance_boundary():
+    ref = np.array([0.0, 1.0, -4.0, 1e-4])
+    bound = 2e-2 + 1e-2 * np.abs(ref)
+    sign = np.array([1.0, 1.0, -1.0, 1.0])
+    # errors just inside atol + rtol |ref| pass; one element just outside fails
+    inside = ref + sign * bound * (1 - 1e-9)
+    ok, max_abs, _ = O.within_tolerance(inside, ref)
+    assert ok and max_abs == pytest.approx(6e-2)
+    for i in range(4):
+        over = inside.copy()
+        over[i] = ref[i] + sign[i] * bound[i] * (1 + 1e-9)
+        assert not O.within_tolerance(over, ref)[0], i
+    # the reported relative error ignores |ref| <= 1e-3
+    _, _, max_rel = O.within_tolerance(ref + 1e-2, ref)
+    assert max_rel == pytest.approx(1e-2)
