@@ -125,10 +125,17 @@ L2_BYTES = 126 * 1024 * 1024
 
 
 def alg_bytes_of(T, K, H, P, mlp=False):
-    """Bytes one step must move at least: X, W, residual in, h and out (bf16)."""
-    if mlp:   # K is the FFN size F: X [P,T,H/P], A [P,2F/P,H], Y, W2 [P,H,F/P], R, out
-        return 2.0 * (T * H + 2 * K * H + 2 * T * K + K * H + 2 * P * T * H)
+    """Bytes one step must move at least (bf16): the inputs read once and the output written
+    once -- X, W, residual and gamma in, out written (h never needs to leave the chip)."""
+    if mlp:   # K is the FFN size F: X [P,T,H], A [P,2F/P,H], Y [P,T,F/P] out and in, W2 [P,H,F/P], R, out
+        return 2.0 * (P * T * H + 2 * K * H + 2 * T * K + K * H + 2 * P * T * H + H)
     return 2.0 * (T * K + H * K + 2 * P * T * H + H)
+
+
+def alg_flops_of(T, K, H, mlp=False):
+    """FLOPs of one step: 2 T K H for the row-parallel GEMM (independent of p); the MLP adds
+    FC1's 2 T H 2F (K = F)."""
+    return 2.0 * T * K * H + (2.0 * T * H * 2 * K if mlp else 0.0)
 
 
 def workload_desc(name, T, K, H, P, p, rand):
@@ -300,6 +307,303 @@ def cpu_baseline(T, K, H, P, p, sync_idx, target_s=10.0, seed=0):
 # ---------------------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------------------
+class Case:
+    """Inputs, workspace and one step (one library call) of a workload on the current GPU."""
+
+    def __init__(self, name, *, tokens=None, p=None, seed=1000, flags=0, no_permute=False, backward=False):
+        import torch
+        from partial_activation_sync_caat_b200 import caat as C
+        from partial_activation_sync_caat_b200 import inputs as I
+        T, K, H, P, p_def, rand = WORKLOADS[name]
+        if tokens:
+            T = tokens
+        p = p if p is not None else p_def
+        self.name, self.T, self.K, self.H, self.P, self.p, self.rand = name, T, K, H, P, p, rand
+        self.mlp = name.startswith("mlp")
+        self.bwd = backward and not self.mlp
+        self.sync_idx = I.random_sync_idx(H, int((H * p) // 1), seed=0) if rand else None
+        self.user_flags = flags
+        self.flags = flags
+        self.flops = alg_flops_of(T, K, H, self.mlp)
+        self.bytes = alg_bytes_of(T, K, H, P, self.mlp)
+        if self.mlp:
+            self.d = I.make_mlp_inputs(T, H, K, P, seed=seed, device="cuda")
+            self.ws = C.alloc_workspace(C.caat_workspace_size(T, K, H, P, C.CAAT_VARIANT_MLP), "cuda")
+        else:
+            self.d = I.make_rowpar_inputs(T, K, H, P, seed=seed, device="cuda")
+            self.ws = C.alloc_workspace(C.caat_workspace_size(T, K, H, P), "cuda")
+        self.out = torch.empty_like(self.d["R"])
+        # A random sync list: W's output channels are permuted once (as at weight load time) so
+        # that the shared channels are contiguous; every step then runs the permuted path.
+        self.permute = rand and not self.mlp and not no_permute and not backward
+        self.permute_ms = None
+        if self.permute:
+            Wp = torch.empty_like(self.d["W"])
+            C.caat_permute_weights(self.d["W"], Wp, self.sync_idx, P, p)       # warm-up
+            torch.cuda.synchronize()
+            pa, pb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            st = torch.cuda.current_stream()
+            pa.record(st)
+            C.caat_permute_weights(self.d["W"], Wp, self.sync_idx, P, p, stream=st)
+            pb.record(st)
+            torch.cuda.synchronize()
+            self.permute_ms = pa.elapsed_time(pb)
+            self.d["W"] = Wp
+            self.flags |= C.CAAT_FLAG_W_PERMUTED
+        if self.bwd:
+            # the layer's backward: the forward's h and a random dout are its inputs
+            d = self.d
+            self.h_saved = torch.empty_like(d["R"])
+            C.caat_rowpar_forward(d["X"], d["W"], d["R"], d["gamma"], self.sync_idx, P, p, self.out, workspace=self.ws,
+                                  h_out=self.h_saved)
+            gen = torch.Generator(device="cuda").manual_seed(seed + 7)
+            self.dout = torch.randn(d["R"].shape, generator=gen, device="cuda").to(torch.bfloat16)
+            self.dX, self.dW, self.dR = torch.empty_like(d["X"]), torch.empty_like(d["W"]), torch.empty_like(d["R"])
+            self.dg = torch.empty(H, dtype=torch.float32, device="cuda")
+            self.ws_b = C.alloc_workspace(C.caat_workspace_size(T, K, H, P, C.CAAT_VARIANT_ROWPAR_BWD), "cuda")
+            self.flops = 4.0 * T * K * H
+        # Workloads whose bytes fit in L2 get an L2 flush before every timed step (see time_case).
+        self.flush = self.bytes < 2 * L2_BYTES and not self.bwd
+
+    def step(self, tm=None, st=None, clear_flags=0):
+        import torch
+        from partial_activation_sync_caat_b200 import caat as C
+        st = torch.cuda.current_stream() if st is None else st
+        d, P, p = self.d, self.P, self.p
+        fl = self.flags & ~clear_flags
+        if self.bwd:
+            C.caat_rowpar_backward(d["X"], d["W"], self.h_saved, d["gamma"], self.dout, self.sync_idx, P, p, self.dX,
+                                   self.dW, self.dg, dR=self.dR, workspace=self.ws_b, stream=st, timing=tm)
+        elif self.mlp:
+            C.caat_mlp_forward(d["X"], d["A"], d["W2"], d["R"], d["gamma"], self.sync_idx, P, p, self.out,
+                               workspace=self.ws, stream=st, timing=tm, flags=fl)
+        else:
+            C.caat_rowpar_forward(d["X"], d["W"], d["R"], d["gamma"], self.sync_idx, P, p, self.out,
+                                  workspace=self.ws, stream=st, timing=tm, flags=fl)
+
+    def launches_per_call(self, n_intervals):
+        """Kernels one call launches (the recorder's intervals, plus the row norm that runs
+        beside the GEMM inside the GEMM's interval)."""
+        if self.bwd:
+            return n_intervals
+        overlapped = n_intervals == (2 if self.mlp else 1)
+        return n_intervals + (1 if overlapped else 0)
+
+
+def time_case(case, steps, warmup, world=1, sample_clocks=False, local=0, soak_ms=500.0):
+    """Times exactly `steps` steps after `warmup` untimed ones: CUDA events on the launching
+    stream, synchronize (and a barrier across ranks) on both sides.  Workloads whose bytes fit
+    in L2 (decode, tiny) get a READ of a buffer 3x the L2 size before every step (a write flush
+    would leave dirty lines whose write-back the next step would pay for); each step is then
+    timed alone, and is one replay of a CUDA graph holding the one library call (the same
+    kernels), so that the host's submission after the flush does not leave the GPU idle inside
+    the timed interval.  Returns (ms_local over all steps, per-call kernel intervals, clocks)."""
+    import torch
+    import torch.distributed as dist
+    from partial_activation_sync_caat_b200 import caat as C
+    stream = torch.cuda.current_stream()
+    timing = C.Timing(capacity=steps + 8)
+    for _ in range(warmup):
+        case.step()
+    torch.cuda.synchronize()
+    if C.caat_get_device_status() != 0:
+        raise SystemExit(f"device status set during warm-up of {case.name}")
+    flush_buf = torch.ones(3 * L2_BYTES // 4, dtype=torch.float32, device="cuda") if case.flush else None
+    graph = None
+    if case.flush:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            case.step(st=torch.cuda.current_stream())
+        graph.replay()
+        torch.cuda.synchronize()
+    sampler = ClockSampler(local) if sample_clocks else None
+    if sampler:
+        sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if case.flush:
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for a_ev, b_ev in evs:
+            flush_buf.sum()
+            a_ev.record(stream)
+            graph.replay()
+            b_ev.record(stream)
+        torch.cuda.synchronize()
+        ms_local = sum(a_ev.elapsed_time(b_ev) for a_ev, b_ev in evs)
+        for _ in range(steps):   # per-kernel split (not part of the timed value)
+            flush_buf.sum()
+            case.step(timing)
+        torch.cuda.synchronize()
+    else:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            case.step(timing)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms_local = e0.elapsed_time(e1)
+    # The timed region is short next to what NVML can sample (tens of ms): keep sampling while
+    # the same step runs back to back for a while more (not timed), on every rank.
+    soak_steps = 0
+    if ms_local < soak_ms:
+        soak_steps = int(min(20000, max(1, (soak_ms - ms_local) / max(ms_local / steps, 1e-3))))
+        for _ in range(soak_steps):
+            if case.flush:
+                graph.replay()
+            else:
+                case.step()
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    if clocks is not None:
+        clocks["window"] = (f"timed region ({ms_local:.1f} ms) + {soak_steps} more steps of the same work run back "
+                            f"to back right after it (not timed)")
+    del flush_buf, graph
+    per_kernel = timing.read()
+    timing.close()
+    return ms_local, per_kernel, clocks
+
+
+def kernel_means(per_kernel):
+    n = max((len(r) for r in per_kernel), default=0)
+    return [statistics.mean(r[j] for r in per_kernel if len(r) > j) for j in range(n)]
+
+
+def sequential_split(case, n):
+    """The same step with the row norm after the GEMM (without CAAT_FLAG_NORM_BESIDE_GEMM),
+    timed per kernel by the library's recorder: what each kernel takes alone (context for the
+    overlapped step; not part of the timed value)."""
+    import torch
+    from partial_activation_sync_caat_b200 import caat as C
+    tm = C.Timing(capacity=n + 2)
+    for _ in range(2):
+        case.step(clear_flags=C.CAAT_FLAG_NORM_BESIDE_GEMM)
+    torch.cuda.synchronize()
+    for _ in range(n):
+        case.step(tm, clear_flags=C.CAAT_FLAG_NORM_BESIDE_GEMM)
+    torch.cuda.synchronize()
+    km = kernel_means(tm.read())
+    tm.close()
+    return km
+
+
+def sub_workloads(args, peaks, peak_src):
+    """The other configurations (rank 0, after the headline run), each timed the same way with
+    its own clock record: ms (or us) per call, throughput and roofline fraction."""
+    import torch
+    res = {}
+    names = ["fc2-1b", "mlp-7b", "attn-out-7b", "decode-1", "decode-8", "decode-64", "tiny"]
+    for name in names:
+        case = Case(name, seed=2000)
+        steps = 20
+        ms_local, per_kernel, clocks = time_case(case, steps, 5, sample_clocks=True, soak_ms=150.0)
+        ms = ms_local / steps
+        km = kernel_means(per_kernel)
+        tflops = case.flops / ms / 1e9
+        gbs = case.bytes / ms / 1e6
+        hbm_bound = case.flops / case.bytes < peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+        e = {"config": workload_desc(name, case.T, case.K, case.H, case.P, case.p, case.rand),
+             "ms_per_call": round(ms, 4), "tflops": round(tflops, 1), "hbm_gbs_algorithmic": round(gbs, 1),
+             "bound": "hbm" if hbm_bound else "tensor",
+             "frac": round(gbs / peaks["hbm_gbs"] if hbm_bound else tflops / peaks["bf16_tflops"], 3),
+             "peak": peaks["hbm_gbs"] if hbm_bound else peaks["bf16_tflops"],
+             "peak_unit": "GB/s" if hbm_bound else "TFLOP/s", "peak_source": peak_src,
+             "kernels_ms": [round(x, 4) for x in km], "l2_flushed": case.flush, "clocks": clocks}
+        if case.T <= 64:
+            e["us_per_call"] = round(ms * 1e3, 2)
+        if case.permute:
+            e["w_permuted_once_ms"] = round(case.permute_ms, 4)
+        res[name] = e
+        del case
+        torch.cuda.empty_cache()
+    return res
+
+
+def run_tp(args):
+    """--tp: the layer over real devices, one tensor-parallel rank per GPU (P = world size):
+    local GEMM step, an NCCL all-reduce (sum, fp32) of the shared channels' partials [T, n_s],
+    finishing step (residual + RMSNorm).  Whole-job TFLOP/s of the one layer (2 T K H over the
+    max-over-ranks step time), plus the bytes each rank's collective reduces."""
+    import datetime
+    import torch
+    import torch.distributed as dist
+    from partial_activation_sync_caat_b200 import build as B
+    from partial_activation_sync_caat_b200 import caat as C
+    from partial_activation_sync_caat_b200 import inputs as I
+    from partial_activation_sync_caat_b200.tp import TPRowParallel, exchanged_bytes
+
+    world, rank, local = rank_env()
+    torch.cuda.set_device(local)
+    if rank == 0:
+        B.build()
+    else:
+        t_wait = time.time()
+        while not B.up_to_date():
+            if time.time() - t_wait > 900:
+                raise SystemExit("libcaat.so was not built by rank 0 within 15 minutes")
+            time.sleep(1.0)
+    if world == 1:   # a one-rank group without torchrun
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        if "MASTER_PORT" not in os.environ:
+            import socket
+            with socket.socket() as sk:
+                sk.bind(("127.0.0.1", 0))
+                os.environ["MASTER_PORT"] = str(sk.getsockname()[1])
+        os.environ.setdefault("RANK", "0")
+        os.environ.setdefault("WORLD_SIZE", "1")
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    C.lib()
+    T, K, H, _, p_def, _ = WORKLOADS["fc2-7b"]
+    if args.tokens:
+        T = args.tokens
+    p = args.p if args.p is not None else p_def
+    P = world
+    if K % P or (K // P) % 8:
+        raise SystemExit(f"K={K} does not split over {P} ranks")
+    # every rank draws the whole layer's inputs from one seed on its GPU and keeps its slice
+    d = I.make_rowpar_inputs(T, K, H, P, seed=0, device="cuda")
+    X, W, R = d["X"][rank].contiguous(), d["W"][rank].contiguous(), d["R"][rank].contiguous()
+    del d["X"], d["W"], d["R"]
+    layer = TPRowParallel(H, p)
+    zs, h = layer.buffers(T, "cuda")
+    out = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
+    ws = C.alloc_workspace(256, "cuda")
+
+    def step():
+        layer.forward(X, W, R, d["gamma"], out, zs=zs, h=h, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    dist.barrier()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(a.elapsed_time(b)) / args.steps
+    status = C.caat_get_device_status()
+    dist.barrier()
+    dist.destroy_process_group()
+    if rank != 0:
+        return
+    flops = 2.0 * T * K * H
+    print(json.dumps({
+        "metric": "TFLOP/s of the partially-synced row-parallel FC2 over real devices (one TP rank per GPU)",
+        "value": round(flops / ms / 1e9, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"fc2-7b over {P} devices: T={T} H={H} K={K} (K/P={K // P} per rank) p={p}",
+                   "parallelism": f"tp{P}"},
+        "exchange": {"collective": "NCCL all-reduce (sum) of the shared channels' fp32 partials",
+                     "bytes_per_rank": exchanged_bytes(T, H, p), "full_all_reduce_bytes": 4 * T * H},
+        "gpu_launches": 2 * args.steps, "device_status": status}))
+
+
 def run_caat(args):
     import torch
     import torch.distributed as dist
@@ -329,163 +633,40 @@ def run_caat(args):
         dist.barrier()
     C.lib()
 
-    T, K, H, P, p_def, rand = WORKLOADS[args.workload]
-    if args.tokens:
-        T = args.tokens
-    p = args.p if args.p is not None else p_def
-    ns = int((H * p) // 1)
-    sync_idx = I.random_sync_idx(H, ns, seed=0) if rand else None
-    mlp = args.workload.startswith("mlp")
+    case = Case(args.workload, tokens=args.tokens, p=args.p, seed=rank_seed(rank), flags=args.flags,
+                no_permute=args.no_permute, backward=args.backward)
+    T, K, H, P, p, rand, mlp, bwd = case.T, case.K, case.H, case.P, case.p, case.rand, case.mlp, case.bwd
+    sync_idx, flops = case.sync_idx, case.flops
     stream = torch.cuda.current_stream()
-    timing = C.Timing(capacity=args.steps + 8)
-    if mlp:
-        d = I.make_mlp_inputs(T, H, K, P, seed=rank_seed(rank), device="cuda")
-        ws = C.alloc_workspace(C.caat_workspace_size(T, K, H, P, C.CAAT_VARIANT_MLP), "cuda")
-        flops = 2.0 * T * H * 2 * K + 2.0 * T * K * H
-    else:
-        d = I.make_rowpar_inputs(T, K, H, P, seed=rank_seed(rank), device="cuda")
-        ws = C.alloc_workspace(C.caat_workspace_size(T, K, H, P), "cuda")
-        flops = 2.0 * T * K * H
-    out = torch.empty_like(d["R"])
-    # A random sync list: W's output channels are permuted once (as at weight load time) so
-    # that the shared channels are contiguous; every step then runs the permuted path.
-    user_flags = args.flags
-    permute = rand and not mlp and not args.no_permute and not args.backward
-    permute_ms = None
-    if permute:
-        Wp = torch.empty_like(d["W"])
-        C.caat_permute_weights(d["W"], Wp, sync_idx, P, p)       # warm-up
-        torch.cuda.synchronize()
-        pa, pb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        pa.record(stream)
-        C.caat_permute_weights(d["W"], Wp, sync_idx, P, p, stream=stream)
-        pb.record(stream)
-        torch.cuda.synchronize()
-        permute_ms = pa.elapsed_time(pb)
-        d["W"] = Wp
-        args.flags |= C.CAAT_FLAG_W_PERMUTED
 
-    bwd = args.backward and not mlp
-    if bwd:
-        # the layer's backward: the forward's h and a random dout are its inputs
-        permute = False
-        h_saved = torch.empty_like(d["R"])
-        C.caat_rowpar_forward(d["X"], d["W"], d["R"], d["gamma"], sync_idx, P, p, out, workspace=ws, h_out=h_saved)
-        gen = torch.Generator(device="cuda").manual_seed(rank_seed(rank) + 7)
-        dout = torch.randn(d["R"].shape, generator=gen, device="cuda").to(torch.bfloat16)
-        dX_b, dW_b, dR_b = torch.empty_like(d["X"]), torch.empty_like(d["W"]), torch.empty_like(d["R"])
-        dg_b = torch.empty(H, dtype=torch.float32, device="cuda")
-        ws_b = C.alloc_workspace(C.caat_workspace_size(T, K, H, P, C.CAAT_VARIANT_ROWPAR_BWD), "cuda")
-        flops = 4.0 * T * K * H
-
-    def step(tm=None, st=None):
-        st = stream if st is None else st
-        if bwd:
-            C.caat_rowpar_backward(d["X"], d["W"], h_saved, d["gamma"], dout, sync_idx, P, p, dX_b, dW_b, dg_b,
-                                   dR=dR_b, workspace=ws_b, stream=st, timing=tm)
-            return
-        if mlp:
-            C.caat_mlp_forward(d["X"], d["A"], d["W2"], d["R"], d["gamma"], sync_idx, P, p, out, workspace=ws,
-                               stream=st, timing=tm, flags=args.flags)
-        else:
-            C.caat_rowpar_forward(d["X"], d["W"], d["R"], d["gamma"], sync_idx, P, p, out, workspace=ws,
-                                  stream=st, timing=tm, flags=args.flags)
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    if C.caat_get_device_status() != 0:
-        raise SystemExit("device status set during warm-up")
-
-    # Workloads whose bytes fit in L2 (decode: W is 90 MB) get an L2 flush before every timed
-    # step: a READ of a buffer 3x the L2 size (a write flush would leave dirty lines whose
-    # write-back the next step would pay for).  Each step is then timed alone with CUDA events
-    # and the flush stays outside the timed intervals.  The step is one call of the library
-    # captured in a CUDA graph (the same kernels, launched from the graph), so that the
-    # host's submission of a call after the flush does not leave the GPU idle inside the
-    # timed interval; the per-kernel split comes from separate flushed calls with the timer.
-    step_bytes = alg_bytes_of(T, K, H, P, mlp)
-    flush = step_bytes < 2 * L2_BYTES
-    flush_buf = torch.ones(3 * L2_BYTES // 4, dtype=torch.float32, device="cuda") if flush else None
-    graph = None
-    if flush:
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
-            step(st=torch.cuda.current_stream())
-        graph.replay()
-        torch.cuda.synchronize()
-    sampler = ClockSampler(local) if rank == 0 else None
-    if sampler:
-        sampler.start()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    if flush:
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(args.steps)]
-        for a_ev, b_ev in evs:
-            flush_buf.sum()
-            a_ev.record(stream)
-            graph.replay()
-            b_ev.record(stream)
-        torch.cuda.synchronize()
-        ms_local = sum(a_ev.elapsed_time(b_ev) for a_ev, b_ev in evs)
-        for _ in range(args.steps):   # per-kernel split (not part of the timed value)
-            flush_buf.sum()
-            step(timing)
-        torch.cuda.synchronize()
-    else:
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
-            step(timing)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        ms_local = e0.elapsed_time(e1)
-    # The timed region is short next to what NVML can sample (tens of ms): keep sampling while
-    # the same step runs back to back for about half a second more (not timed), on every rank.
-    soak_steps = 0
-    if ms_local < 500.0:
-        soak_steps = int(min(20000, max(1, (500.0 - ms_local) / max(ms_local / args.steps, 1e-3))))
-        for _ in range(soak_steps):
-            if flush:
-                graph.replay()
-            else:
-                step()
-        torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    clocks = sampler.stop() if sampler else None
-    if clocks is not None:
-        clocks["window"] = (f"timed region ({ms_local:.1f} ms) + {soak_steps} more steps of the same work run back "
-                            f"to back right after it (not timed)")
+    ms_local, per_kernel, clocks = time_case(case, args.steps, args.warmup, world, sample_clocks=(rank == 0),
+                                             local=local)
     ms = max_over_ranks(ms_local)
-    del flush_buf, graph
-    per_kernel = timing.read()
-    n_kernels = max((len(r) for r in per_kernel), default=1)
-    kernel_ms = [statistics.mean(r[j] for r in per_kernel if len(r) > j) for j in range(n_kernels)]
-    # index of the row-parallel GEMM kernel in the per-call kernel list (FC1 comes first in the MLP)
-    kg = 1 if mlp else 0
-    k1 = [r[kg] for r in per_kernel if len(r) > kg]
-    k2 = [r[kg + 1] for r in per_kernel if len(r) > kg + 1]
+    kernel_ms = kernel_means(per_kernel)
+    n_intervals = len(kernel_ms)
+    launches = case.launches_per_call(n_intervals) * args.steps
     status = C.caat_get_device_status()
+    # the row norm ran beside the GEMM: one recorded interval holds both kernels
+    overlapped = (not bwd) and not case.permute and n_intervals == (2 if mlp else 1)
+    split = sequential_split(case, max(5, args.steps // 2)) if overlapped else None
 
     # optional p sweep (same shapes, fewer steps), rank 0 only
     sweep = None
-    if args.sweep and rank == 0 and not mlp and not permute and not bwd:   # W permuted for one (p, S) only
+    if args.sweep and rank == 0 and not mlp and not case.permute and not bwd:   # W permuted for one (p, S) only
         sweep = {}
+        d, out, ws = case.d, case.out, case.ws
         for ps in (0.0, 0.25, 0.5, 0.75, 1.0):
             idx_s = I.random_sync_idx(H, int((H * ps) // 1), seed=0) if rand else None
             for _ in range(2):
                 C.caat_rowpar_forward(d["X"], d["W"], d["R"], d["gamma"], idx_s, P, ps, out, workspace=ws,
-                                      flags=args.flags)
+                                      flags=case.flags)
             torch.cuda.synchronize()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             n = max(3, args.steps // 2)
             a.record()
             for _ in range(n):
                 C.caat_rowpar_forward(d["X"], d["W"], d["R"], d["gamma"], idx_s, P, ps, out, workspace=ws,
-                                      flags=args.flags)
+                                      flags=case.flags)
             b.record()
             torch.cuda.synchronize()
             t_ms = a.elapsed_time(b) / n
@@ -494,11 +675,12 @@ def run_caat(args):
     # end to end through the host-buffer entry point (pinned host tensors, copies timed)
     e2e = None
     if not args.no_e2e and not mlp and not bwd:
+        d = case.d
         hX, hW, hR, hg = (d[k].cpu().pin_memory() for k in ("X", "W", "R", "gamma"))
         hout = torch.empty(hR.shape, dtype=torch.bfloat16).pin_memory()
         wsh = C.alloc_workspace(C.caat_workspace_size(T, K, H, P, C.CAAT_VARIANT_ROWPAR_HOST), "cuda")
         for _ in range(2):
-            C.caat_rowpar_forward_host(hX, hW, hR, hg, sync_idx, P, p, hout, wsh, stream=stream, flags=args.flags)
+            C.caat_rowpar_forward_host(hX, hW, hR, hg, sync_idx, P, p, hout, wsh, stream=stream, flags=case.flags)
         torch.cuda.synchronize()
         n_e2e = max(3, min(args.steps, 10))
         if world > 1:
@@ -506,7 +688,7 @@ def run_caat(args):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         for _ in range(n_e2e):
-            C.caat_rowpar_forward_host(hX, hW, hR, hg, sync_idx, P, p, hout, wsh, stream=stream, flags=args.flags)
+            C.caat_rowpar_forward_host(hX, hW, hR, hg, sync_idx, P, p, hout, wsh, stream=stream, flags=case.flags)
         b.record(stream)
         torch.cuda.synchronize()
         e_ms = max_over_ranks(a.elapsed_time(b) / n_e2e)
@@ -525,16 +707,28 @@ def run_caat(args):
         return
 
     peaks, peak_src = load_peaks()
-    default_case = not args.tokens and args.p is None and not user_flags  # the recorded ncu case
+    default_case = not args.tokens and args.p is None and not args.flags  # the recorded ncu case
     ms_step = ms / args.steps
     value = whole_job_tflops(flops, world, ms_step)
-    k1_ms = statistics.mean(k1) if k1 else float("nan")
-    k2_ms = statistics.mean(k2) if k2 else None
     fc2_flops = 2.0 * T * K * H
+    kg = 1 if mlp else 0           # index of the row-parallel GEMM's interval (FC1 comes first in the MLP)
+    k1_ms = kernel_ms[kg] if len(kernel_ms) > kg else float("nan")
+    k2_ms = kernel_ms[kg + 1] if len(kernel_ms) > kg + 1 else None
     k1_tflops = fc2_flops / k1_ms / 1e9
     norm_bytes = 2.0 * P * T * H * 2
-    k2_gbs = norm_bytes / k2_ms / 1e6 if k2_ms else None
     alg_bytes = alg_bytes_of(T, K, H, P)
+    if overlapped:
+        t_g, t_n = recorded_traffic(args.workload, "gemm"), recorded_traffic(args.workload, "norm_overlapped")
+        traffic = (t_g + t_n) if (default_case and t_g is not None and t_n is not None) else None
+        kname = ("rowpar_gemm_pair_kernel (tcgen05 cta_group::2 GEMM + partial channel-reduce + residual) with "
+                 "rownorm_consumer_kernel (RMSNorm on the SMs the GEMM leaves free) beside it: one overlapped "
+                 "interval")
+        algo = "2*T*K*H flops per call of the overlapped GEMM + norm"
+    else:
+        traffic = recorded_traffic(args.workload, "gemm") if default_case else None
+        kname = ("rowpar_gemm_pair_kernel (tcgen05 cta_group::2 GEMM + partial channel-reduce "
+                 "+ residual" + (")" if k2_ms else " + fused RMSNorm)"))
+        algo = "2*T*K*H flops per launch"
     result = {
         "metric": "TFLOP/s & tokens/s of partially-synced row-parallel FC2 (7B shape), % bf16 peak",
         "value": round(value, 2),
@@ -551,26 +745,35 @@ def run_caat(args):
         "config": {"workload": workload_desc(args.workload, T, K, H, P, p, rand), "T": T, "H": H, "K": K,
                    "P": P, "p": p, "parallelism": f"{world} independent GPU(s), P={P} emulated TP ranks each",
                    "l2": ("step bytes (%.1f MB) fit in L2: read-flush of a %d MB buffer before every step, "
-                          "outside the per-step event intervals" % (step_bytes / 1e6, 3 * L2_BYTES // 2**20)
-                          if flush else
-                          "inputs larger than L2 (%.2f GB touched per step); no flush" % (step_bytes / 1e9))},
+                          "outside the per-step event intervals" % (case.bytes / 1e6, 3 * L2_BYTES // 2**20)
+                          if case.flush else
+                          "inputs larger than L2 (%.2f GB touched per step); no flush" % (case.bytes / 1e9))},
         "tokens_per_s": round(world * T / (ms_step / 1e3), 1),
-        "pct_bf16_peak": {"measured_burst": round(100 * value / world / peaks["bf16_tflops"], 1),
+        "pct_bf16_peak": {f"{peak_src}_burst": round(100 * value / world / peaks["bf16_tflops"], 1),
                           "datasheet_2250": round(100 * value / world / 2250.0, 1)},
-        "roofline": {"kernel": "rowpar_gemm_pair_kernel (tcgen05 cta_group::2 GEMM + partial channel-reduce "
-                               "+ residual" + (")" if k2_ms else " + fused RMSNorm)"),
-                     "bound": "tensor", "achieved": round(k1_tflops, 1), "peak": peaks["bf16_tflops"],
+        "roofline": {"kernel": kname, "bound": "tensor", "achieved": round(k1_tflops, 1), "peak": peaks["bf16_tflops"],
                      "peak_source": f"{peak_src} bf16 burst", "unit": "TFLOP/s",
                      "frac": round(k1_tflops / peaks["bf16_tflops"], 3),
                      "frac_vs_sustained": round(k1_tflops / peaks["bf16_tflops_sustained"], 3),
-                     "traffic": recorded_traffic(args.workload, "gemm") if default_case else None,
-                     "launch_ms": round(k1_ms, 4),
-                     "algorithmic": "2*T*K*H flops per launch"},
-        "gpu_launches": n_kernels * args.steps,
+                     "traffic": traffic, "launch_ms": round(k1_ms, 4), "algorithmic": algo},
+        "gpu_launches": launches,
         "device_status": status,
         "clocks": clocks,
     }
     result["kernels_ms"] = [round(x, 4) for x in kernel_ms]
+    if split is not None:
+        sg = split[kg] if len(split) > kg else None
+        sn = split[kg + 1] if len(split) > kg + 1 else None
+        result["sequential_split"] = {
+            "about": "the same call with the norm after the GEMM (no CAAT_FLAG_NORM_BESIDE_GEMM), per-kernel CUDA "
+                     "events; not the timed value",
+            "gemm_ms": round(sg, 4) if sg else None, "norm_ms": round(sn, 4) if sn else None,
+            "gemm_tflops": round(fc2_flops / sg / 1e9, 1) if sg else None,
+            "gemm_frac": round(fc2_flops / sg / 1e9 / peaks["bf16_tflops"], 3) if sg else None,
+            "norm_gbs": round(norm_bytes / sn / 1e6, 1) if sn else None,
+            "norm_frac": round(norm_bytes / sn / 1e6 / peaks["hbm_gbs"], 3) if sn else None,
+            "gemm_traffic": recorded_traffic(args.workload, "gemm") if default_case else None,
+            "norm_traffic": recorded_traffic(args.workload, "norm") if default_case else None}
     if mlp:
         result["metric"] = "TFLOP/s of the partially-synced MLP block (FC1+SwiGLU+FC2+residual+RMSNorm, 7B shape)"
         result["fc1_kernel"] = {"kernel": "fc1_swiglu_pair_kernel", "launch_ms": round(kernel_ms[0], 4),
@@ -578,25 +781,28 @@ def run_caat(args):
     if T <= 64:
         result["decode"] = {"us_per_call": round(ms_step * 1e3, 2), "hbm_gbs": round(alg_bytes / ms_step / 1e6, 1),
                             "frac_of_measured_hbm": round(alg_bytes / ms_step / 1e6 / peaks["hbm_gbs"], 3)}
-    if k2_ms:
+    if k2_ms and not overlapped:
         result["norm_kernel"] = {"kernel": "rownorm_reg_kernel" if H <= 4096 else "rownorm_kernel", "bound": "hbm",
-                                 "achieved": round(k2_gbs, 1),
+                                 "achieved": round(norm_bytes / k2_ms / 1e6, 1),
                                  "traffic": recorded_traffic(args.workload, "norm") if default_case else None,
-                                 "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(k2_gbs / peaks["hbm_gbs"], 3),
+                                 "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                 "frac": round(norm_bytes / k2_ms / 1e6 / peaks["hbm_gbs"], 3),
                                  "launch_ms": round(k2_ms, 4), "algorithmic": "2*P*T*H*2 bytes (read h, write out)"}
     if args.flags:
         result["config"]["flags"] = hex(args.flags)
     if not mlp:
-        # the paper's speed-up model (App. C Eq. 34-35) for this shape, fed with this pool's
-        # measured numbers: bf16 GEMM burst and the NVLink peer copy per direction (770 GB/s,
-        # bf16 activations on the wire): C = operations per exchanged activation
+        # the paper's speed-up model (App. C Eq. 34-35) for this shape: C = operations per exchanged
+        # activation from the bf16 GEMM rate and an NVLink rate per direction (bf16 activations on
+        # the wire).  The NVLink figure is an assumed constant (this pool's peer-copy figure from
+        # its documentation), not measured by this run: every run here has one GPU.
         nvlink_gbs = 770.0
         c_ratio = peaks["bf16_tflops"] * 1e12 / (nvlink_gbs * 1e9 / 2.0)
         sp_m, ps_m = C.caat_speedup_model(H, T, P, p, c_ratio)
         result["speedup_model"] = {"source": "App. C Eq. 34-35", "h": H, "s": T, "r": P, "p": p,
                                    "C_ops_per_activation": round(c_ratio, 1),
                                    "C_inputs": f"{peaks['bf16_tflops']} TFLOP/s {peak_src} bf16 / "
-                                               f"({nvlink_gbs} GB/s NVLink per direction / 2 B)",
+                                               f"({nvlink_gbs} GB/s NVLink per direction, assumed, not measured "
+                                               f"here / 2 B)",
                                    "speedup_vs_full_sync": round(sp_m, 4), "p_star": round(ps_m, 4)}
     if bwd:
         norm_names = ["rownorm_bwd_kernel (norm backward + reduction over ranks)", "dgamma_reduce_kernel"]
@@ -618,13 +824,17 @@ def run_caat(args):
                                   "traffic": None, "launch_ms": round(gx, 4), "algorithmic": "2*T*K*H flops",
                                   "dW_gemm_tflops": round(fc2_flops / gw / 1e9, 1)}
         result.pop("norm_kernel", None)
-    if permute:
+    if case.permute:
         result["w_permuted"] = {"api": "caat_permute_weights, once before the steps (weights are static)",
-                                "once_ms": round(permute_ms, 4)}
+                                "once_ms": round(case.permute_ms, 4)}
     if sweep is not None:
         result["p_sweep"] = sweep
     if e2e is not None:
         result["e2e"] = e2e
+    del case
+    torch.cuda.empty_cache()
+    if world == 1 and not args.no_workloads and args.workload == "fc2-7b" and not args.tokens and not bwd:
+        result["workloads"] = sub_workloads(args, peaks, peak_src)
     if not args.no_cpu_baseline and not bwd:
         result["cpu_baseline"] = cpu_baseline(T, K, H, P, p, sync_idx, target_s=args.cpu_seconds)
     print(json.dumps(result))
@@ -693,7 +903,12 @@ def main():
     ap.add_argument("--sweep", action="store_true", help="also time p in {0,.25,.5,.75,1}")
     ap.add_argument("--backward", action="store_true",
                     help="time the layer's backward (caat_rowpar_backward) instead of the forward")
+    ap.add_argument("--tp", action="store_true",
+                    help="the layer over real devices: one tensor-parallel rank per GPU (P = --gpus), NCCL "
+                         "all-reduce of the shared channels")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the per-workload records of the other configurations (fc2-7b default run)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-rows", type=int, default=64)
@@ -702,6 +917,8 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.tp:
+        run_tp(args)
     else:
         run_caat(args)
 

@@ -102,6 +102,13 @@ typedef enum caat_status {
                                             residual, else out, which must then not alias
                                             residual); not with CAAT_FLAG_FUSED_NORM; the
                                             GEMM path needs H <= 4096. */
+#define CAAT_FLAG_NORM_BESIDE_GEMM 0x200u /* CTA-pair GEMM path, H <= 4096, separate norm: start the
+                                            row norm while the GEMM runs, on SMs the GEMM leaves
+                                            free; it normalizes each 128-token block of a rank as
+                                            soon as the GEMM has stored all of it (the GEMM counts
+                                            its finished tiles per block in the workspace).  Needs
+                                            the workspace caat_workspace_size reports; same bits
+                                            as the default (norm after the GEMM) */
 #define CAAT_FLAG_TEST_STALL 0x100u      /* test hook: the GEMM kernel's MMA warp never signals
                                             its accumulator, so every consumer wait runs out
                                             and the call reports CAAT_ERR_TIMEOUT through
@@ -186,13 +193,21 @@ CAAT_API caat_status caat_rowpar_forward_host(const caat_rowpar_args* args);
  * deployment convenience of this library.
  *
  * Arguments as caat_rowpar_forward_ex, except that args->workspace and args->ws_bytes are
- * ignored.  The scratch the kernels need (the work-unit counter of the GEMM kernel) lives in
- * a fixed device array inside the library, CAAT_NOALLOC_SCRATCH_BYTES bytes per GPU, held by
- * every GPU that loads the library until the process exits.  A call whose scratch need
- * exceeds that size returns CAAT_ERR_WORKSPACE and queues nothing.
+ * ignored.  The scratch the kernels need lives in a fixed device array inside the library,
+ * CAAT_NOALLOC_SCRATCH_BYTES bytes per GPU, held by every GPU that loads the library until the
+ * process exits.  It holds whatever workspace the path the call takes uses, when that fits:
+ * the GEMM kernel's work-unit counter (always), the row-block counters and job list of the
+ * norm that runs beside the GEMM (8 bytes per 128 tokens per rank), the completion flags of
+ * column blocks that mix shared and private channels (T/8 ceil(H/256) bytes), the fused
+ * norm's counters and partials, and the decode path's fp32 partials (4 P T H bytes).
+ *   - A fused norm (CAAT_FLAG_FUSED_NORM) whose partials do not fit runs as the separate norm;
+ *     a decode-sized call whose partials do not fit takes the GEMM path; the optional parts
+ *     (job list, flags) are simply not used when they do not fit.  A call that still needs
+ *     more than the array (a forced decode path that does not fit) returns
+ *     CAAT_ERR_WORKSPACE and queues nothing.
  *   - Calls no cudaMalloc, cudaFree or other allocating routine.
- *   - The first call on a device looks up the array's device address (once per device, with
- *     that device current); make that first call before any stream capture.
+ *   - The first call on a device looks up the array's device address (once per device and
+ *     context, with that device current); make that first call before any stream capture.
  *   - Every call shares the one array and clears the part that must start at zero; calls
  *     whose work overlaps on the GPU (other streams, other host threads) race on it and must
  *     be serialized by the caller.
@@ -306,6 +321,54 @@ typedef struct caat_rowpar_bwd_args {
 #define CAAT_BWD_FLAG_TRANSPOSED_OPERANDS 0x1u
 
 CAAT_API caat_status caat_rowpar_backward(const caat_rowpar_bwd_args* args);
+
+/*
+ * The layer over real devices, one tensor-parallel rank per GPU (App. A.2 Eq. 22; §3: only the
+ * first floor(h p) channels are synchronized; App. D: the exchange moves p times the bytes of
+ * a full all-reduce).  Each rank r runs, on its own GPU:
+ *   1. caat_rowpar_tp_local: its partial product X_r W_r^T (tcgen05 GEMM); the shared channels
+ *      c < n_s = floor(H p) are written to zs as fp32 partials, the private channels are
+ *      finished into h (private_scale * partial + residual, bf16);
+ *   2. the caller's collective: zs summed over the ranks in place (e.g. an NCCL all-reduce,
+ *      sum, fp32, of T * n_s elements); every rank then holds the same sums (Eq. 22);
+ *   3. caat_rowpar_tp_finish: h[:, c] = bf16(zs[:, c] + residual[:, c]) for c < n_s (so h is the
+ *      complete pre-norm residual stream), then out = RMSNorm(h) * gamma (§4 Eq. 9).
+ * S is the first n_s channels (the paper's definition); n_s % 8 == 0 and H <= 4096 are
+ * required (CAAT_ERR_UNSUPPORTED otherwise).  The single-device entry points above emulate the
+ * same layer with the exchange folded into the tensor-core accumulation.
+ *
+ *   X         device bf16 [T, K_r]   this rank's input slice (local)
+ *   W         device bf16 [H, K_r]   this rank's weight block (local)
+ *   residual  device bf16 [T, H]     this rank's residual (local, finish)
+ *   gamma     device bf16 [H]        RMSNorm weight (finish)
+ *   zs        device fp32 [T, n_s]   local: out (this rank's partial); finish: in (the sum over
+ *                                    ranks); NULL allowed when n_s == 0
+ *   h         device bf16 [T, H]     local: out (private channels); finish: in/out (complete h)
+ *   out       device bf16 [T, H]     finish: out; may alias h
+ *   workspace local: 256 device bytes, 256-byte aligned (finish: unused)
+ * Both calls are asynchronous on `stream`.  Outputs must not overlap other inputs.
+ */
+typedef struct caat_tp_args {
+  const caat_bf16* X;
+  const caat_bf16* W;
+  const caat_bf16* residual;
+  const caat_bf16* gamma;
+  float* zs;
+  caat_bf16* h;
+  caat_bf16* out;
+  void* workspace;
+  size_t ws_bytes;
+  caat_stream_t stream;
+  caat_timing* timing;
+  int64_t T, K_r, H;
+  double p;
+  float eps;
+  float private_scale;
+  uint32_t flags;              /* 0 */
+} caat_tp_args;
+
+CAAT_API caat_status caat_rowpar_tp_local(const caat_tp_args* args);
+CAAT_API caat_status caat_rowpar_tp_finish(const caat_tp_args* args);
 
 /*
  * caat_permute_weights - reorders the output channels (rows) of W for a sync set: with

@@ -38,6 +38,7 @@ CAAT_FLAG_OVERLAP_NORM = 0x20
 CAAT_FLAG_ORDER_GROUPED = 0x40
 CAAT_FLAG_W_PERMUTED = 0x80
 CAAT_FLAG_TEST_STALL = 0x100
+CAAT_FLAG_NORM_BESIDE_GEMM = 0x200
 
 CAAT_NOALLOC_SCRATCH_BYTES = 1048576
 
@@ -48,7 +49,8 @@ EXPORTS = [
     "caat_workspace_size", "caat_sync_mask", "caat_get_device_status", "caat_timing_create",
     "caat_timing_destroy", "caat_timing_reset", "caat_timing_read", "caat_status_string",
     "caat_version", "caat_permute_weights", "caat_speedup_model", "caat_rowpar_backward",
-    "caat_plan_create", "caat_plan_execute", "caat_plan_destroy",
+    "caat_plan_create", "caat_plan_execute", "caat_plan_destroy", "caat_rowpar_tp_local",
+    "caat_rowpar_tp_finish",
 ]
 
 
@@ -79,6 +81,17 @@ class BwdArgs(ctypes.Structure):
         ("timing", ctypes.c_void_p), ("T", ctypes.c_int64), ("K", ctypes.c_int64), ("H", ctypes.c_int64),
         ("p", ctypes.c_double), ("eps", ctypes.c_float), ("private_scale", ctypes.c_float),
         ("P", ctypes.c_int32), ("flags", ctypes.c_uint32),
+    ]
+
+
+class TpArgs(ctypes.Structure):
+    _fields_ = [
+        ("X", ctypes.c_void_p), ("W", ctypes.c_void_p), ("residual", ctypes.c_void_p),
+        ("gamma", ctypes.c_void_p), ("zs", ctypes.c_void_p), ("h", ctypes.c_void_p), ("out", ctypes.c_void_p),
+        ("workspace", ctypes.c_void_p), ("ws_bytes", ctypes.c_size_t), ("stream", ctypes.c_void_p),
+        ("timing", ctypes.c_void_p), ("T", ctypes.c_int64), ("K_r", ctypes.c_int64), ("H", ctypes.c_int64),
+        ("p", ctypes.c_double), ("eps", ctypes.c_float), ("private_scale", ctypes.c_float),
+        ("flags", ctypes.c_uint32),
     ]
 
 
@@ -128,6 +141,10 @@ def lib() -> ctypes.CDLL:
     L.caat_plan_execute.argtypes = [vp, vp]
     L.caat_plan_destroy.restype = ctypes.c_int
     L.caat_plan_destroy.argtypes = [vp]
+    L.caat_rowpar_tp_local.argtypes = [ctypes.POINTER(TpArgs)]
+    L.caat_rowpar_tp_local.restype = ctypes.c_int
+    L.caat_rowpar_tp_finish.argtypes = [ctypes.POINTER(TpArgs)]
+    L.caat_rowpar_tp_finish.restype = ctypes.c_int
     L.caat_rowpar_backward.restype = ctypes.c_int
     L.caat_rowpar_backward.argtypes = [ctypes.POINTER(BwdArgs)]
     L.caat_speedup_model.restype = ctypes.c_int
@@ -335,6 +352,62 @@ class Plan:
             self.close()
         except Exception:
             pass
+
+
+def _f32_dev(t, name):
+    import torch
+    if t.dtype != torch.float32:
+        raise TypeError(f"{name} must be float32")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    return _ptr(t)
+
+
+def _tp_args(T, K_r, H, p, eps, private_scale, stream, timing):
+    a = TpArgs()
+    a.T, a.K_r, a.H = int(T), int(K_r), int(H)
+    a.p = float(p)
+    a.eps = float(eps)
+    a.private_scale = float(private_scale)
+    a.stream = _stream_ptr(stream)
+    a.timing = timing.handle if timing is not None else None
+    a.flags = 0
+    return a
+
+
+def caat_rowpar_tp_local(X, W, residual, p: float, zs, h, *, workspace=None, private_scale: float = 1.0,
+                         stream=None, timing=None):
+    """Local step of one rank of the layer over real devices: X [T,K_r], W [H,K_r], residual
+    [T,H] (bf16, this rank's); writes zs [T, floor(H p)] (fp32, this rank's partial of the shared
+    channels) and the private channels of h [T,H] (bf16)."""
+    T, K_r = int(X.shape[0]), int(X.shape[1])
+    H = int(W.shape[0])
+    if workspace is None:
+        workspace = alloc_workspace(256, X.device)
+    a = _tp_args(T, K_r, H, p, 1e-5, private_scale, stream, timing)
+    a.X = _bf16_dev(X, "X")
+    a.W = _bf16_dev(W, "W")
+    a.residual = _bf16_dev(residual, "residual")
+    a.zs = _f32_dev(zs, "zs") if zs is not None and zs.numel() else None
+    a.h = _bf16_dev(h, "h")
+    a.workspace = _ptr(workspace)
+    a.ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().caat_rowpar_tp_local(ctypes.byref(a)), "caat_rowpar_tp_local")
+    return zs, h
+
+
+def caat_rowpar_tp_finish(zs, residual, h, gamma, p: float, out, *, eps: float = 1e-5, stream=None, timing=None):
+    """Finishing step after the exchange: zs [T, floor(H p)] holds the sum over the ranks;
+    writes the shared channels of h [T,H] and out [T,H] = RMSNorm(h) * gamma."""
+    T, H = int(h.shape[0]), int(h.shape[1])
+    a = _tp_args(T, 0, H, p, eps, 1.0, stream, timing)
+    a.residual = _bf16_dev(residual, "residual")
+    a.gamma = _bf16_dev(gamma, "gamma")
+    a.zs = _f32_dev(zs, "zs") if zs is not None and zs.numel() else None
+    a.h = _bf16_dev(h, "h")
+    a.out = _bf16_dev(out, "out")
+    _check(lib().caat_rowpar_tp_finish(ctypes.byref(a)), "caat_rowpar_tp_finish")
+    return out
 
 
 def caat_rowpar_backward(X, W, h, gamma, dout, sync_idx, P: int, p: float, dX, dW, dgamma, *, dR=None,

@@ -23,6 +23,7 @@
 #include "decode.cuh"
 #include "permuted.cuh"
 #include "rownorm.cuh"
+#include "tp.cuh"
 
 namespace {
 
@@ -31,10 +32,32 @@ using caat::RowparParams;
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;  // bounded device waits: 2 s
 
 // ---------------------------------------------------------------------------------------
-// Device info and one-time kernel attributes (per device)
+// The current CUDA context (driver entry point fetched through the runtime).  Per-device state
+// below (kernel attributes, streams, the no-alloc scratch address) is tied to the context it
+// was made in: after a device reset the next call finds a new context and sets it up again.
+// ---------------------------------------------------------------------------------------
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+CUcontext current_context() {
+  static CtxGetCurrentFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<CtxGetCurrentFn>(nullptr);
+    return reinterpret_cast<CtxGetCurrentFn>(p);
+  }();
+  CUcontext c = nullptr;
+  if (fn && fn(&c) != CUDA_SUCCESS) c = nullptr;
+  return c;
+}
+
+// ---------------------------------------------------------------------------------------
+// Device info and one-time kernel attributes (per device and context)
 // ---------------------------------------------------------------------------------------
 struct DeviceInfo {
   bool init = false;
+  CUcontext ctx = nullptr;
   bool supported = false;
   int sm_count = 0;
   int max_pairs = 0;  // co-resident 2-CTA clusters of the pair GEMM kernel
@@ -49,7 +72,10 @@ caat_status device_info(DeviceInfo** out) {
   if (dev < 0 || dev >= 64) return CAAT_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lk(g_mu);
   DeviceInfo& d = g_dev[dev];
+  const CUcontext ctx = current_context();
+  if (d.init && d.ctx != ctx) d = DeviceInfo();  // a new context (device reset): set up again
   if (!d.init) {
+    d.ctx = ctx;
     int major = 0, minor = 0, sms = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return CAAT_ERR_CUDA;
     if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return CAAT_ERR_CUDA;
@@ -80,7 +106,13 @@ caat_status device_info(DeviceInfo** out) {
           cudaFuncSetAttribute(caat::rownorm_gather_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(caat::gather_smem_bytes(2048))) != cudaSuccess ||
           cudaFuncSetAttribute(caat::rownorm_gather_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(caat::gather_smem_bytes(4096))) != cudaSuccess)
+                               static_cast<int>(caat::gather_smem_bytes(4096))) != cudaSuccess ||
+          cudaFuncSetAttribute(caat::rownorm_consumer_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               caat::K2C_SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(caat::rownorm_consumer_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               caat::K2C_SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(caat::rownorm_consumer_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               caat::K2C_SMEM_BYTES) != cudaSuccess)
         return CAAT_ERR_CUDA;
       cudaLaunchConfig_t cfg = {};
       cudaLaunchAttribute attr[1];
@@ -113,6 +145,54 @@ int group_m_setting() {
     const char* e = std::getenv("CAAT_GROUP_M");
     const int g = (e && *e) ? std::atoi(e) : 0;
     return g > 0 ? g : 8;
+  }();
+  return v;
+}
+
+// Upper bounds on the GEMM kernel's CTA pairs and the row norm's blocks (tuning; 0 = none).
+int env_cap(const char* name) {
+  const char* e = std::getenv(name);
+  const int v = (e && *e) ? std::atoi(e) : 0;
+  return v > 0 ? v : 0;
+}
+int gemm_pairs_cap() {
+  static int v = env_cap("CAAT_GEMM_PAIRS");
+  return v;
+}
+int norm_blocks_cap() {
+  static int v = env_cap("CAAT_NORM_BLOCKS");
+  return v;
+}
+// SMs the GEMM kernel leaves to the row norm running beside it (tuning; CAAT_NORM_SMS).
+int norm_sms_setting() {
+  static int v = [] {
+    const char* e = std::getenv("CAAT_NORM_SMS");
+    return (e && *e) ? std::max(0, std::atoi(e)) : 16;
+  }();
+  return v;
+}
+// Unit order and stagger distance of the GEMM when the row norm runs beside it (tuning;
+// CAAT_ORDER, CAAT_STAGGER).
+int consumer_order_setting() {
+  static int v = [] {
+    const char* e = std::getenv("CAAT_ORDER");
+    const int o = (e && *e) ? std::atoi(e) : 0;
+    return (o >= 0 && o <= 3) ? o : 0;
+  }();
+  return v;
+}
+bool order_env_set() {
+  static bool v = [] {
+    const char* e = std::getenv("CAAT_ORDER");
+    return e && *e;
+  }();
+  return v;
+}
+int stagger_setting() {
+  static int v = [] {
+    const char* e = std::getenv("CAAT_STAGGER");
+    const int d = (e && *e) ? std::atoi(e) : 6;
+    return d >= 0 ? d : 6;
   }();
   return v;
 }
@@ -158,6 +238,21 @@ caat_status make_map_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_
   const cuuint32_t box[3] = {b0, b1, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? CAAT_OK : CAAT_ERR_CUDA;
+}
+
+// 3-D fp32 tensor [d2][d1][d0] (d0 contiguous), box {b0, b1, 1}, 128-byte swizzle.
+caat_status make_map_3d_f32(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0,
+                            uint32_t b1) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return CAAT_ERR_CUDA;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {d0 * 4, d0 * d1 * 4};
+  const cuuint32_t box[3] = {b0, b1, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? CAAT_OK : CAAT_ERR_CUDA;
@@ -234,13 +329,14 @@ size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
 // Workspace of the row-parallel layer.  Fused norm: [counters (256 B) | rb_count[n_rb] |
 // job_slots[n_rb] | ss_part[P][T_pad][nslots_max] floats]; the counter region (first `zeroed`
 // bytes) is cleared on the stream before every launch; ss_part needs no clearing (every slot
-// of every valid row is written once).  Separate norm: [counters (256 B) | sdone], where the
-// optional sdone flags ([T_pad/32][n-blocks] u32, cleared before the launch when used) let
-// the CTA-pair kernel give mixed column blocks the TMA epilogue; with a workspace of only
-// the 256 B (`min_total`) those blocks take the register epilogue.  Sized for the larger of
-// the two GEMM kernels' row blocking.
+// of every valid row is written once).  Separate norm: [counters (256 B) | rb_count[n_rb] |
+// sdone]: the tile counters (cleared before the launch when used) let the row norm run beside
+// the GEMM; the optional sdone flags ([T_pad/32][n-blocks] u32, cleared before the launch when
+// used) let the CTA-pair kernel give mixed column blocks the TMA epilogue.  With a workspace of
+// only the 256 B (`min_total`) the norm runs after the GEMM and mixed blocks take the register
+// epilogue.  Sized for the larger of the two GEMM kernels' row blocking.
 struct RowparWs {
-  size_t rb_count, job_slots, ss_part, zeroed, total, min_total, sdone, sdone_bytes;
+  size_t rb_count, job_slots, ss_part, zeroed, total, min_total, sdone, sdone_bytes, consumer_total;
   int64_t T_pad, n_rb, nslots_max;
 };
 
@@ -257,8 +353,12 @@ RowparWs rowpar_ws_layout(int64_t T, int64_t H, int P, bool fused) {
     L.total = L.ss_part + align256(size_t(P) * L.T_pad * L.nslots_max * 4);
     L.min_total = L.total;
   } else {
+    // [counters | rb_count | sdone]: the per-(128-row block, rank) tile counters let the row
+    // norm run beside the GEMM (a workspace that ends before sdone still allows it).
+    L.rb_count = kCounterBytes;
     L.zeroed = kCounterBytes;
-    L.sdone = kCounterBytes;
+    L.consumer_total = L.rb_count + size_t(L.n_rb) * 4;
+    L.sdone = align256(L.consumer_total);
     L.sdone_bytes = size_t(L.T_pad / 32) * size_t((H + 255) / 256) * 4;
     L.total = L.sdone + align256(L.sdone_bytes);
     L.min_total = kCounterBytes;
@@ -284,14 +384,27 @@ size_t decode_workspace(int64_t T, int64_t H, int P) {
   return kCounterBytes + align256(size_t(decode_splits(T)) * P * T * H * 4);
 }
 
-// Workspace a call needs at least (`fused`: with the fused norm), or, with full = true, the size
-// that also enables every fast path (the value caat_workspace_size reports).
-size_t rowpar_workspace(int64_t T, int64_t K, int64_t H, int P, bool fused = true, bool full = true) {
+// Whether a call with these shapes and flags runs the decode (weight-streaming) kernels.
+bool takes_decode_path(int64_t T, int P, int64_t H, uint32_t flags) {
+  if (!decode_eligible(T, P, H)) return false;
+  if (flags & CAAT_FLAG_FORCE_DECODE_PATH) return true;
+  return !(flags & (CAAT_FLAG_FORCE_GEMM_PATH | CAAT_FLAG_FUSED_NORM | CAAT_FLAG_TEST_STALL));
+}
+
+// The size that enables every path and fast path of a call of this shape (the value
+// caat_workspace_size reports).
+size_t rowpar_workspace(int64_t T, int64_t K, int64_t H, int P) {
   (void)K;
-  size_t n = full ? std::max(rowpar_ws_layout(T, H, P, true).total, rowpar_ws_layout(T, H, P, false).total)
-                  : rowpar_ws_layout(T, H, P, fused).min_total;
+  size_t n = std::max(rowpar_ws_layout(T, H, P, true).total, rowpar_ws_layout(T, H, P, false).total);
   if (decode_eligible(T, P, H)) n = std::max(n, decode_workspace(T, H, P));
   return n;
+}
+
+// The workspace a call with these flags needs at least: the decode path's partials if it takes
+// that path, else the GEMM path's minimum (the fused norm's partials, or the 256-byte counters).
+size_t rowpar_workspace_min(int64_t T, int64_t H, int P, uint32_t flags) {
+  if (takes_decode_path(T, P, H, flags)) return decode_workspace(T, H, P);
+  return rowpar_ws_layout(T, H, P, (flags & CAAT_FLAG_FUSED_NORM) != 0).min_total;
 }
 
 // Device staging of caat_rowpar_forward_host.  Token rows are independent through the whole
@@ -329,6 +442,7 @@ constexpr int64_t kNormChunk = 2048;  // tokens per GEMM launch when the norm is
 // kernel computes the next chunk (created once per device).
 struct NormSide {
   bool init = false;
+  CUcontext ctx = nullptr;
   cudaStream_t s = nullptr;
   cudaEvent_t ev_gemm = nullptr, ev_done = nullptr;
 };
@@ -340,7 +454,10 @@ caat_status norm_side(NormSide** out) {
   if (dev < 0 || dev >= 64) return CAAT_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lk(g_mu);
   NormSide& ns = g_side[dev];
+  const CUcontext ctx = current_context();
+  if (ns.init && ns.ctx != ctx) ns = NormSide();  // handles of a context that no longer exists
   if (!ns.init) {
+    ns.ctx = ctx;
     if (cudaStreamCreateWithFlags(&ns.s, cudaStreamNonBlocking) != cudaSuccess ||
         cudaEventCreateWithFlags(&ns.ev_gemm, cudaEventDisableTiming) != cudaSuccess ||
         cudaEventCreateWithFlags(&ns.ev_done, cudaEventDisableTiming) != cudaSuccess)
@@ -354,6 +471,7 @@ caat_status norm_side(NormSide** out) {
 // Copy streams and events of the host-buffer pipeline (created once per device).
 struct HostPipe {
   bool init = false;
+  CUcontext ctx = nullptr;
   cudaStream_t s_in = nullptr, s_out = nullptr;
   cudaEvent_t ev_start = nullptr, ev_w = nullptr, ev_in[2] = {}, ev_comp[2] = {}, ev_out[2] = {};
 };
@@ -365,7 +483,10 @@ caat_status host_pipe(HostPipe** out) {
   if (dev < 0 || dev >= 64) return CAAT_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lk(g_mu);
   HostPipe& hp = g_pipe[dev];
+  const CUcontext ctx = current_context();
+  if (hp.init && hp.ctx != ctx) hp = HostPipe();  // handles of a context that no longer exists
   if (!hp.init) {
+    hp.ctx = ctx;
     if (cudaStreamCreateWithFlags(&hp.s_in, cudaStreamNonBlocking) != cudaSuccess ||
         cudaStreamCreateWithFlags(&hp.s_out, cudaStreamNonBlocking) != cudaSuccess)
       return CAAT_ERR_CUDA;
@@ -387,7 +508,8 @@ struct MlpWs {
 MlpWs mlp_ws_layout(int64_t T, int64_t H, int64_t F, int P, bool fused) {
   MlpWs L{};
   L.rowpar = kCounterBytes;
-  L.y = L.rowpar + align256(rowpar_workspace(T, F, H, P, fused));
+  (void)fused;
+  L.y = L.rowpar + align256(rowpar_workspace(T, F, H, P));
   L.total = L.y + align256(size_t(P) * T * (F / P) * 2);
   return L;
 }
@@ -497,12 +619,18 @@ caat_status launch_decode(const caat_rowpar_args* a, const std::vector<uint8_t>&
   return CAAT_OK;
 }
 
+// The split-output local step of one rank of a multi-device layer (caat_rowpar_tp_local):
+// the fp32 partial of the first n_s channels goes to zs [T, n_s], the other channels are
+// finished into h.
+struct TpSplit {
+  float* zs;
+  int64_t n_s;
+};
+
 caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>& mask, const DeviceInfo* dev,
-                          unsigned int* counter, Recorder* outer = nullptr) {
+                          unsigned int* counter, Recorder* outer = nullptr, const TpSplit* split = nullptr) {
   // Decode-sized calls stream W once through the dedicated path.
-  const bool decode = decode_eligible(a->T, a->P, a->H) && !(a->flags & CAAT_FLAG_FORCE_GEMM_PATH) &&
-                      !(a->flags & CAAT_FLAG_FUSED_NORM) && !(a->flags & CAAT_FLAG_TEST_STALL);
-  if (decode || ((a->flags & CAAT_FLAG_FORCE_DECODE_PATH) && decode_eligible(a->T, a->P, a->H)))
+  if (!split && takes_decode_path(a->T, a->P, a->H, a->flags))
     return launch_decode(a, mask, dev, reinterpret_cast<uint8_t*>(counter), outer);
   const int P = a->P;
   const int64_t T = a->T, H = a->H, Kp = a->K / P;
@@ -549,6 +677,26 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
   // order); otherwise shared tiles first, then private tiles rank by rank.
   prm.order = (a->flags & CAAT_FLAG_ORDER_ROWBLOCK) ? 1 : ((fused || (a->flags & CAAT_FLAG_ORDER_GROUPED)) ? 2 : 0);
   prm.group_m = group_m_setting();
+  // The row norm beside the GEMM (CTA-pair kernel, separate norm, rows of at most 4096
+  // channels): the GEMM publishes each completed (128-row block, rank), and the norm kernel,
+  // launched as its programmatic dependent, normalizes published rows on the SMs the GEMM
+  // leaves free, while the GEMM computes the others.
+  const bool pair_possible =
+      dev->max_pairs > 0 && (split != nullptr || (!(a->flags & CAAT_FLAG_SINGLE_CTA) && T > caat::K1_BM));
+  const bool consumer = pair_possible && !split && !fused && !permuted && !gemm_only && H <= 4096 &&
+                        (a->flags & CAAT_FLAG_NORM_BESIDE_GEMM) && !(a->flags & CAAT_FLAG_OVERLAP_NORM) &&
+                        a->ws_bytes >= wl.consumer_total;
+  prm.publish = fused ? 1 : (consumer ? 2 : 0);
+  if (consumer) {
+    prm.rb_count = reinterpret_cast<unsigned int*>(wsb + wl.rb_count);
+    if (!(a->flags & (CAAT_FLAG_ORDER_ROWBLOCK | CAAT_FLAG_ORDER_GROUPED))) {
+      prm.order = consumer_order_setting();
+      if (prm.order == 3) prm.group_m = stagger_setting();
+    }
+  } else if (!fused && !(a->flags & (CAAT_FLAG_ORDER_ROWBLOCK | CAAT_FLAG_ORDER_GROUPED)) && order_env_set()) {
+    prm.order = consumer_order_setting();  // tuning: the same tile orders with the norm after the GEMM
+    if (prm.order == 3) prm.group_m = stagger_setting();
+  }
   prm.eps = a->eps;
   prm.T = static_cast<int>(T);
   prm.H = static_cast<int>(H);
@@ -575,7 +723,7 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
     if ((*tmask)[c]) prm.mask_bits[c >> 5] |= 1u << (c & 31);
   prm.nslots = prm.nS + prm.nPriv;
   // The CTA-pair kernel (256-token tiles) for all but the smallest token counts.
-  const bool pair = !(a->flags & CAAT_FLAG_SINGLE_CTA) && dev->max_pairs > 0 && T > caat::K1_BM;
+  const bool pair = pair_possible;
   const int major = ((a->flags & kFlagAMn) ? 1 : 0) | ((a->flags & kFlagBMn) ? 2 : 0);
   if (major != 0 && (!pair || !gemm_only || fused || major == 1)) return CAAT_ERR_UNSUPPORTED;
   const int64_t bm = pair ? 2 * caat::K2P_BM : caat::K1_BM;
@@ -589,9 +737,12 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
   const bool merge = pair && !fused && any_mixed && a->ws_bytes >= wl.total;
   prm.merge_mixed = merge ? 1 : 0;
   prm.sdone = merge ? reinterpret_cast<unsigned int*>(wsb + wl.sdone) : nullptr;
-  const size_t zero_bytes = merge ? wl.sdone + wl.sdone_bytes : wl.zeroed;
+  const size_t zero_bytes = merge ? wl.sdone + wl.sdone_bytes : (consumer ? wl.consumer_total : wl.zeroed);
 
-  CUtensorMap tmX, tmW, tmR, tmH;
+  prm.zs_mode = split ? 1 : 0;
+  prm.zs_ns = split ? static_cast<int>(split->n_s) : 0;
+  if (split && (!pair || fused || permuted || gemm_only)) return CAAT_ERR_UNSUPPORTED;
+  CUtensorMap tmX, tmW, tmR, tmH, tmZ;
   // K-major operands: boxes of 64 K x (128 rows); MN-major ones: 64 MN x 64 K rows, two per half
   caat_status s = (major & 1) ? make_map_3d(&tmX, a->X, T, Kp, P, 64, caat::K2P_BK)
                               : make_map_3d(&tmX, a->X, Kp, T, P, caat::K1_BK, caat::K1_BM);
@@ -604,6 +755,12 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
   if (s != CAAT_OK) return s;
   s = make_map_3d(&tmH, hdst, H, T, P, 64, 32);
   if (s != CAAT_OK) return s;
+  // the split output's fp32 shared-channel partials: 32-row x 32-column boxes
+  tmZ = tmH;
+  if (split && split->n_s > 0) {
+    s = make_map_3d_f32(&tmZ, split->zs, static_cast<uint64_t>(split->n_s), T, 1, 32, 32);
+    if (s != CAAT_OK) return s;
+  }
 
   // One GEMM launch over the token rows [t0, t0 + tc) (t0 a multiple of the tile height).
   auto gemm = [&](int64_t t0, int64_t tc) -> caat_status {
@@ -614,7 +771,9 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
     prm.n_units = static_cast<int>(units);
     if (cudaMemsetAsync(counter, 0, zero_bytes, st) != cudaSuccess) return CAAT_ERR_CUDA;
     if (pair) {
-      const int pairs = static_cast<int>(std::min<int64_t>(dev->max_pairs, units));
+      int pairs = static_cast<int>(std::min<int64_t>(dev->max_pairs, units));
+      if (consumer) pairs = std::max(1, std::min(pairs, dev->max_pairs - (norm_sms_setting() + 1) / 2));
+      if (gemm_pairs_cap() > 0) pairs = std::min(pairs, gemm_pairs_cap());
       cudaLaunchConfig_t cfg = {};
       cudaLaunchAttribute attr[1];
       attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -628,10 +787,12 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
       cfg.attrs = attr;
       cfg.numAttrs = 1;
       const cudaError_t e =
-          fused        ? cudaLaunchKernelEx(&cfg, caat::rowpar_gemm_pair_kernel<true>, tmX, tmW, tmR, tmH, prm)
-          : major == 2 ? cudaLaunchKernelEx(&cfg, caat::rowpar_gemm_pair_kernel<false, 2>, tmX, tmW, tmR, tmH, prm)
-          : major == 3 ? cudaLaunchKernelEx(&cfg, caat::rowpar_gemm_pair_kernel<false, 3>, tmX, tmW, tmR, tmH, prm)
-                       : cudaLaunchKernelEx(&cfg, caat::rowpar_gemm_pair_kernel<false>, tmX, tmW, tmR, tmH, prm);
+          fused ? cudaLaunchKernelEx(&cfg, caat::rowpar_gemm_pair_kernel<true>, tmX, tmW, tmR, tmH, tmZ, prm)
+          : major == 2
+              ? cudaLaunchKernelEx(&cfg, caat::rowpar_gemm_pair_kernel<false, 2>, tmX, tmW, tmR, tmH, tmZ, prm)
+          : major == 3
+              ? cudaLaunchKernelEx(&cfg, caat::rowpar_gemm_pair_kernel<false, 3>, tmX, tmW, tmR, tmH, tmZ, prm)
+              : cudaLaunchKernelEx(&cfg, caat::rowpar_gemm_pair_kernel<false>, tmX, tmW, tmR, tmH, tmZ, prm);
       if (e != cudaSuccess) return CAAT_ERR_CUDA;
     } else {
       const int grid = static_cast<int>(std::min<int64_t>(dev->sm_count, units));
@@ -678,7 +839,8 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
     const int64_t blocks = std::min<int64_t>((rows + warps_per_block - 1) / warps_per_block, max_blocks);
     if (H <= 4096) {
       // row held in registers: VPL 128-bit vectors per lane
-      const int64_t rb = std::min<int64_t>((rows + warps_per_block - 1) / warps_per_block, int64_t(dev->sm_count) * 2);
+      int64_t rb = std::min<int64_t>((rows + warps_per_block - 1) / warps_per_block, int64_t(dev->sm_count) * 2);
+      if (norm_blocks_cap() > 0) rb = std::min<int64_t>(rb, norm_blocks_cap());
       if (H <= 1024)
         caat::rownorm_reg_kernel<4><<<rb, caat::K2_THREADS, 0, ns>>>(hdst, o, g, P, T, t0, tc, static_cast<int>(H), a->eps);
       else if (H <= 2048)
@@ -704,13 +866,58 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
   Recorder own;
   Recorder& rec = outer ? *outer : own;
   if (!outer) rec.begin(a->timing, st);
-  const bool overlap =
-      !fused && !permuted && !gemm_only && (a->flags & CAAT_FLAG_OVERLAP_NORM) && T >= 2 * kNormChunk;
+  if (consumer) {
+    // GEMM, then the row norm as its programmatic dependent (no event between the two: the
+    // recorder's one interval covers both kernels).
+    s = gemm(0, T);
+    if (s != CAAT_OK) return s;
+    const int64_t pieces = int64_t(prm.n_rb) * (caat::K2C_ROWS_PER_JOB / caat::K2C_ROWS_PER_PIECE);
+    const int64_t warps_per_block = caat::K2C_THREADS / 32;
+    const int64_t nb = std::max<int64_t>(
+        1, std::min<int64_t>((pieces + warps_per_block - 1) / warps_per_block, int64_t(dev->sm_count)));
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3(static_cast<unsigned>(nb), 1, 1);
+    cfg.blockDim = dim3(caat::K2C_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = caat::K2C_SMEM_BYTES;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const __nv_bfloat16* hc = hdst;
+    const unsigned int* rbc = prm.rb_count;
+    // a (128-row block, rank) is complete after every tile of its row, from each epilogue warp
+    const unsigned int target = static_cast<unsigned int>((prm.nS + prm.nPriv) * 4);
+    const int n_m128 = prm.T_pad / 128;
+    const int order = prm.order == 0 ? 0 : 1;
+    const unsigned int* prog = counter;     // the GEMM's unit counter: its progress
+    unsigned int* pc = counter + 32;        // piece counter, on its own 128-byte line
+    const uint64_t tmo = prm.timeout_ns;
+    const int64_t Tl = T;
+    const int Hi = static_cast<int>(H);
+    const float ep = a->eps;
+    cudaError_t e;
+    if (H <= 1024)
+      e = cudaLaunchKernelEx(&cfg, caat::rownorm_consumer_kernel<4>, hc, o, g, P, Tl, Hi, ep, rbc, target, n_m128,
+                             order, prog, pc, tmo);
+    else if (H <= 2048)
+      e = cudaLaunchKernelEx(&cfg, caat::rownorm_consumer_kernel<8>, hc, o, g, P, Tl, Hi, ep, rbc, target, n_m128,
+                             order, prog, pc, tmo);
+    else
+      e = cudaLaunchKernelEx(&cfg, caat::rownorm_consumer_kernel<16>, hc, o, g, P, Tl, Hi, ep, rbc, target, n_m128,
+                             order, prog, pc, tmo);
+    if (e != cudaSuccess) return CAAT_ERR_CUDA;
+    rec.after_kernel(st);
+    return CAAT_OK;
+  }
+  const bool overlap = !fused && !permuted && !gemm_only && !split && (a->flags & CAAT_FLAG_OVERLAP_NORM) &&
+                       T >= 2 * kNormChunk;
   if (!overlap) {
     s = gemm(0, T);
     if (s != CAAT_OK) return s;
     rec.after_kernel(st);
-    if (fused || gemm_only) return CAAT_OK;
+    if (fused || gemm_only || split) return CAAT_OK;
     s = norm(0, T, st, int64_t(dev->sm_count) * 4);
     if (s != CAAT_OK) return s;
     rec.after_kernel(st);
@@ -748,7 +955,7 @@ caat_status validate_rowpar(const caat_rowpar_args* a, std::vector<uint8_t>& mas
   if (!aligned16(a->X) || !aligned16(a->W) || !aligned16(a->residual) || !aligned16(a->gamma) ||
       !aligned16(a->out) || (a->h_out && !aligned16(a->h_out)))
     return CAAT_ERR_UNSUPPORTED;
-  const size_t need = rowpar_workspace(a->T, a->K, a->H, a->P, (a->flags & CAAT_FLAG_FUSED_NORM) != 0, false);
+  const size_t need = rowpar_workspace_min(a->T, a->H, a->P, a->flags);
   if (need > 0) {
     if (!a->workspace || a->ws_bytes < need || (reinterpret_cast<uintptr_t>(a->workspace) & 255u))
       return CAAT_ERR_WORKSPACE;
@@ -1154,17 +1361,122 @@ caat_status caat_rowpar_forward_host(const caat_rowpar_args* a) {
 }  // extern "C"
 
 // ---------------------------------------------------------------------------------------
+// The layer over real devices, one tensor-parallel rank per GPU
+// ---------------------------------------------------------------------------------------
+namespace {
+
+// `local`: the local step's arguments (K_r is checked only there).
+caat_status validate_tp(const caat_tp_args* a, int64_t* n_s_out, bool local) {
+  if (!a) return CAAT_ERR_INVALID_ARG;
+  if (a->T < 0 || (local && a->K_r <= 0) || a->H <= 0 || !(a->p >= 0.0 && a->p <= 1.0)) return CAAT_ERR_INVALID_ARG;
+  if (!(a->eps >= 0.f) || !std::isfinite(a->eps) || !std::isfinite(a->private_scale)) return CAAT_ERR_INVALID_ARG;
+  if ((local && (a->K_r % 8 != 0 || a->K_r > (int64_t(1) << 30))) || a->H % 8 != 0 || a->H > 4096 ||
+      a->T > (int64_t(1) << 30))
+    return CAAT_ERR_UNSUPPORTED;
+  const int64_t ns = n_sync_of(a->H, a->p);
+  if (ns % 8 != 0) return CAAT_ERR_UNSUPPORTED;
+  *n_s_out = ns;
+  return CAAT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+caat_status caat_rowpar_tp_local(const caat_tp_args* a) {
+  int64_t ns = 0;
+  caat_status s = validate_tp(a, &ns, true);
+  if (s != CAAT_OK) return s;
+  if (a->T == 0) return CAAT_OK;
+  if (!a->X || !a->W || !a->residual || !a->h || (ns > 0 && !a->zs)) return CAAT_ERR_INVALID_ARG;
+  if (!aligned16(a->X) || !aligned16(a->W) || !aligned16(a->residual) || !aligned16(a->h) ||
+      (ns > 0 && !aligned16(a->zs)))
+    return CAAT_ERR_UNSUPPORTED;
+  if (!a->workspace || a->ws_bytes < kCounterBytes || (reinterpret_cast<uintptr_t>(a->workspace) & 255u))
+    return CAAT_ERR_WORKSPACE;
+  DeviceInfo* dev = nullptr;
+  s = device_info(&dev);
+  if (s != CAAT_OK) return s;
+  if (dev->max_pairs <= 0) return CAAT_ERR_UNSUPPORTED;
+  // One rank, every channel a private tile; the split epilogue decides per 64-channel chunk.
+  caat_rowpar_args r;
+  std::memset(&r, 0, sizeof(r));
+  r.X = a->X;
+  r.W = a->W;
+  r.residual = a->residual;
+  r.gamma = a->residual;  // unused by the split mode
+  r.out = a->h;
+  r.h_out = a->h;
+  r.workspace = a->workspace;
+  r.ws_bytes = kCounterBytes;
+  r.stream = a->stream;
+  r.timing = a->timing;
+  r.T = a->T;
+  r.K = a->K_r;
+  r.H = a->H;
+  r.p = 0.0;
+  r.eps = a->eps;
+  r.private_scale = a->private_scale;
+  r.P = 1;
+  r.flags = CAAT_FLAG_FORCE_GEMM_PATH;
+  static thread_local std::vector<uint8_t> zero_mask;
+  zero_mask.assign(static_cast<size_t>(a->H), 0);
+  const TpSplit split{a->zs, ns};
+  return launch_rowpar(&r, zero_mask, dev, static_cast<unsigned int*>(a->workspace), nullptr, &split);
+}
+
+caat_status caat_rowpar_tp_finish(const caat_tp_args* a) {
+  int64_t ns = 0;
+  caat_status s = validate_tp(a, &ns, false);
+  if (s != CAAT_OK) return s;
+  if (a->T == 0) return CAAT_OK;
+  if (!a->residual || !a->gamma || !a->h || !a->out || (ns > 0 && !a->zs)) return CAAT_ERR_INVALID_ARG;
+  if (!aligned16(a->residual) || !aligned16(a->gamma) || !aligned16(a->h) || !aligned16(a->out) ||
+      (ns > 0 && !aligned16(a->zs)))
+    return CAAT_ERR_UNSUPPORTED;
+  DeviceInfo* dev = nullptr;
+  s = device_info(&dev);
+  if (s != CAAT_OK) return s;
+  Recorder rec;
+  rec.begin(a->timing, a->stream);
+  const int64_t warps = caat::KT_FIN_THREADS / 32;
+  const int64_t nb = std::max<int64_t>(1, std::min<int64_t>((a->T + warps - 1) / warps, int64_t(dev->sm_count) * 4));
+  const float* z = a->zs;
+  const __nv_bfloat16* R = reinterpret_cast<const __nv_bfloat16*>(a->residual);
+  __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(a->h);
+  __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(a->out);
+  const __nv_bfloat16* g = reinterpret_cast<const __nv_bfloat16*>(a->gamma);
+  const int Hi = static_cast<int>(a->H), nsi = static_cast<int>(ns);
+  cudaStream_t st = a->stream;
+  if (a->H <= 1024)
+    caat::tp_finish_kernel<4><<<nb, caat::KT_FIN_THREADS, 0, st>>>(z, R, h, o, g, a->T, Hi, nsi, a->eps);
+  else if (a->H <= 2048)
+    caat::tp_finish_kernel<8><<<nb, caat::KT_FIN_THREADS, 0, st>>>(z, R, h, o, g, a->T, Hi, nsi, a->eps);
+  else
+    caat::tp_finish_kernel<16><<<nb, caat::KT_FIN_THREADS, 0, st>>>(z, R, h, o, g, a->T, Hi, nsi, a->eps);
+  if (cudaGetLastError() != cudaSuccess) return CAAT_ERR_CUDA;
+  rec.after_kernel(st);
+  return CAAT_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------------------
 // Entry point without any device allocation: the scratch is a fixed device array.
 // ---------------------------------------------------------------------------------------
 namespace {
 
-// Scratch of caat_rowpar_forward_noalloc (the work-unit counter of the GEMM kernel), shared
-// by every call of that entry point on a device.  In host code `g_noalloc_scratch` is only a
-// host-side stand-in for the symbol: the kernels get its device address, looked up once per
-// device with cudaGetSymbolAddress.
+// Scratch of caat_rowpar_forward_noalloc, shared by every call of that entry point on a
+// device: whatever workspace the path a call takes needs (the GEMM's unit counter, the
+// row-block counters and job list of the norm running beside the GEMM, the mixed-block flags,
+// the fused norm's counters and partials, the decode path's fp32 partials), when it fits.  In
+// host code `g_noalloc_scratch` is only a host-side stand-in for the symbol: the kernels get its
+// device address, looked up with cudaGetSymbolAddress once per device (and again if the
+// device's context was replaced, e.g. after a device reset).
 static __device__ __align__(256) unsigned char g_noalloc_scratch[CAAT_NOALLOC_SCRATCH_BYTES];
 
 void* g_noalloc_ptr[64];
+CUcontext g_noalloc_ctx[64];
 bool g_noalloc_ready[64];
 
 caat_status noalloc_scratch(void** out) {
@@ -1172,10 +1484,12 @@ caat_status noalloc_scratch(void** out) {
   if (cudaGetDevice(&dev) != cudaSuccess) return CAAT_ERR_CUDA;
   if (dev < 0 || dev >= 64) return CAAT_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_noalloc_ready[dev]) {
+  const CUcontext ctx = current_context();
+  if (!g_noalloc_ready[dev] || g_noalloc_ctx[dev] != ctx) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return CAAT_ERR_CUDA;
     g_noalloc_ptr[dev] = p;
+    g_noalloc_ctx[dev] = ctx;
     g_noalloc_ready[dev] = true;
   }
   *out = g_noalloc_ptr[dev];
@@ -1200,11 +1514,14 @@ caat_status caat_rowpar_forward_noalloc(const caat_rowpar_args* a) {
   // The fused RMSNorm needs scratch that grows with T; when it does not fit the built-in
   // array, the norm runs as the separate row kernel, which needs only the unit counter.
   if ((d.flags & CAAT_FLAG_FUSED_NORM) &&
-      rowpar_workspace(d.T, d.K, d.H, d.P, true, false) > CAAT_NOALLOC_SCRATCH_BYTES)
+      rowpar_workspace_min(d.T, d.H, d.P, d.flags) > CAAT_NOALLOC_SCRATCH_BYTES)
     d.flags &= ~CAAT_FLAG_FUSED_NORM;
-  if (rowpar_workspace(d.T, d.K, d.H, d.P, (d.flags & CAAT_FLAG_FUSED_NORM) != 0, false) >
-      CAAT_NOALLOC_SCRATCH_BYTES)
-    return CAAT_ERR_WORKSPACE;
+  // Likewise the decode path's fp32 partials (4 P T H bytes): a decode-sized call whose partials
+  // do not fit takes the GEMM path (unless the caller forces the decode path).
+  if (takes_decode_path(d.T, d.P, d.H, d.flags) && !(d.flags & CAAT_FLAG_FORCE_DECODE_PATH) &&
+      decode_workspace(d.T, d.H, d.P) > CAAT_NOALLOC_SCRATCH_BYTES)
+    d.flags |= CAAT_FLAG_FORCE_GEMM_PATH;
+  if (rowpar_workspace_min(d.T, d.H, d.P, d.flags) > CAAT_NOALLOC_SCRATCH_BYTES) return CAAT_ERR_WORKSPACE;
   void* scratch = nullptr;
   s = noalloc_scratch(&scratch);
   if (s != CAAT_OK) return s;

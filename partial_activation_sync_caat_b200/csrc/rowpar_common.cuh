@@ -59,6 +59,9 @@ struct RowparParams {
   unsigned int* sdone;         // [T_pad/32][n-blocks] shared unit of a mixed block stored, zero at launch
   int merge_mixed;             // 1: mixed blocks use the TMA epilogue (see k1_epilogue_tma)
   int no_residual;             // 1: store Z (no residual add) -- channel-permuted path, see rownorm.cuh
+  int zs_mode;                 // 1: split output of one rank of a multi-device layer (tp.cuh):
+                               // channels c < zs_ns go to Zs as the fp32 partial, the others to h
+  int zs_ns;                   // shared channels (zs_mode)
   int T, H, Kp, P;             // T: token rows of the tensors (the row stride of rank blocks)
   int t_begin, t_end;          // token rows this launch processes: [t_begin, t_end)
   int n_mblk;                  // row blocks of the kernel's tile height over [t_begin, t_end)
@@ -67,10 +70,17 @@ struct RowparParams {
   int nS, nPriv;               // n-blocks that have a shared unit / private units
   int n_units;
   int fuse_norm;               // 1: normalizer warps produce `Out`; 0: h only
+  int publish;                 // 1 (fused norm): count each tile into its (128-row block, rank)
+                               // counter and publish completed row blocks to the job list;
+                               // 2 (row-norm kernel beside this one): each epilogue warp adds 1 to
+                               // the counters of its tile's (128-row block, rank)s once the tile's
+                               // stores are complete (checked when the warp's next tile starts)
   int order;                   // unit order: 0 shared units first, then private rank-major;
                                // 1 row-block-major (each row block's units together);
-                               // 2 grouped: order 0 within groups of group_m row blocks
-  int group_m;                 // row blocks per group (order 2)
+                               // 2 grouped: order 0 within groups of group_m row blocks;
+                               // 3 staggered: row block s's shared units, then row block
+                               //   (s - group_m)'s private units, for s = 0, 1, ...
+  int group_m;                 // row blocks per group (order 2) / stagger distance (order 3)
   int n_rb;                    // (128-row block, rank) pairs = n_m128 * P
   int T_pad;                   // n_m128 * 128
   int nslots;                  // nS + nPriv partial slots per row
@@ -91,6 +101,49 @@ struct K1Unit {
 
 __device__ __forceinline__ K1Unit k1_decode(int u, const RowparParams& prm) {
   K1Unit un;
+  if (prm.order == 3) {
+    // Staggered: step s holds the shared units of row block s (if s < n_mblk), then the
+    // private units of row block s - D (rank-major, n fastest).  Row blocks complete at an even
+    // rate over the whole kernel (a row block is complete with its private units), and every
+    // step mixes long shared and short private units.  D >= 0 keeps each mixed block's shared
+    // unit ahead of its private units.
+    const int D = min(prm.group_m, prm.n_mblk);
+    const int np = prm.P * prm.nPriv;
+    const int per = prm.nS + np;
+    const int head = D * prm.nS;
+    const int n_mid = prm.n_mblk - D;
+    int m, v;  // v < 0: shared unit -v - 1; v >= 0: private unit v
+    if (u < head) {
+      m = u / prm.nS;
+      v = -(u - m * prm.nS) - 1;
+    } else if (u - head < n_mid * per) {
+      const int s = (u - head) / per;
+      const int w = (u - head) - s * per;
+      if (w < prm.nS) {
+        m = D + s;
+        v = -w - 1;
+      } else {
+        m = s;
+        v = w - prm.nS;
+      }
+    } else {
+      const int w = u - head - n_mid * per;
+      m = n_mid + w / np;
+      v = w - (m - n_mid) * np;
+    }
+    un.m = m;
+    if (v < 0) {
+      un.slot = -v - 1;
+      un.n = prm.slist[un.slot];
+      un.rank = -1;
+    } else {
+      un.rank = v / prm.nPriv;
+      const int pi = v - un.rank * prm.nPriv;
+      un.n = prm.plist[pi];
+      un.slot = prm.nS + pi;
+    }
+    return un;
+  }
   if (prm.order == 2) {
     // Grouped: for each group of group_m row blocks, its shared units (row block major),
     // then its private units rank by rank.  Row blocks of a group complete together, while
@@ -385,6 +438,13 @@ __device__ __forceinline__ bool k1_epilogue_tma(uint32_t trow, const RowparParam
       }
       __syncwarp();
     }
+    if (prm.publish == 1) {  // the row blocks are published after this tile: complete its stores
+      if (lane == 0) {
+        bulk_wait_group0();
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+      }
+      __syncwarp();
+    }
     return true;
   }
   const int nch = min(4, (prm.H - n0 + 63) / 64);
@@ -421,7 +481,14 @@ __device__ __forceinline__ bool k1_epilogue_tma(uint32_t trow, const RowparParam
         bulk_commit_group();
       }
     }
-    if (lane == 0) bulk_wait_group_read0();
+    if (lane == 0) {
+      if (prm.publish == 1) {
+        bulk_wait_group0();
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+      } else {
+        bulk_wait_group_read0();
+      }
+    }
     __syncwarp();
     return true;
   }
@@ -489,7 +556,7 @@ __device__ __forceinline__ bool k1_epilogue_tma(uint32_t trow, const RowparParam
     }
   }
   if (lane == 0) {
-    if (prm.fuse_norm) {
+    if (prm.publish == 1) {
       // The normalizers of other CTAs read this tile's h: complete the stores and order
       // them (async proxy) before the generic-proxy signal that follows.
       bulk_wait_group0();
@@ -498,6 +565,83 @@ __device__ __forceinline__ bool k1_epilogue_tma(uint32_t trow, const RowparParam
       bulk_wait_group_read0();
     }
   }
+  __syncwarp();
+  return true;
+}
+
+// Epilogue of one tile of the split-output mode (one tensor-parallel rank per device, every
+// unit private): for each 64-column chunk of the warp's 32 rows, the columns below zs_ns (the
+// shared channels, exchanged between devices) are stored as the fp32 partial to Zs [T, zs_ns]
+// (two 32-column boxes, clipped at zs_ns by the tensor map), and a chunk reaching beyond zs_ns
+// gets its private columns finished as in the plain epilogue (private scale, residual, bf16)
+// and stored to h.  A chunk straddling zs_ns also stores its first columns to h with private
+// arithmetic; the finishing kernel overwrites them with the exchanged values.  Returns false
+// if a wait ran out.
+__device__ __forceinline__ bool k1_epilogue_split(uint32_t trow, const RowparParams& prm, const void* tmR,
+                                                  const void* tmH, const void* tmZ, int row0, int n0, int rank,
+                                                  uint8_t* bufs, uint64_t* rbar, uint32_t& phase, int lane,
+                                                  uint64_t pol_r, uint64_t pol_h) {
+  const int nch = min(4, (prm.H - n0 + 63) / 64);
+  const float scale = prm.private_scale;
+  for (int c = 0; c < nch; ++c) {
+    const int col = n0 + 64 * c;
+    const bool has_shared = col < prm.zs_ns;
+    const bool has_private = col + 64 > prm.zs_ns;
+    if (has_private && lane == 0) {  // the residual box, while the accumulator is read
+      bulk_wait_group_read0();       // earlier stores from the buffers are done reading them
+      mbar_arrive_expect_tx(&rbar[0], K1_EPI_BOX_BYTES);
+      tma_load_3d(bufs, tmR, &rbar[0], col, row0, rank, pol_r);
+    }
+    uint32_t v[64];
+    __syncwarp();
+    tmem_ld_32x32b_x32(trow + 64 * c, *reinterpret_cast<uint32_t(*)[32]>(v));
+    tmem_ld_32x32b_x32(trow + 64 * c + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+    tmem_wait_ld();
+    if (has_shared) {
+      // fp32 boxes of 32 rows x 32 columns (128-byte rows, 128-byte swizzle) in buffer 1
+      for (int hf = 0; hf < 2; ++hf) {
+        if (col + 32 * hf >= prm.zs_ns) break;  // warp-uniform
+        if (lane == 0) bulk_wait_group_read0();
+        __syncwarp();
+        uint8_t* rowp = bufs + K1_EPI_BOX_BYTES + lane * 128;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          *reinterpret_cast<uint4*>(rowp + ((j ^ (lane & 7)) << 4)) =
+              make_uint4(v[32 * hf + 4 * j], v[32 * hf + 4 * j + 1], v[32 * hf + 4 * j + 2], v[32 * hf + 4 * j + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(tmZ, bufs + K1_EPI_BOX_BYTES, col + 32 * hf, row0, 0, pol_h);
+          bulk_commit_group();
+        }
+      }
+    }
+    if (has_private) {
+      const bool ok = mbar_wait(&rbar[0], phase & 1u, prm.timeout_ns, 34);
+      phase ^= 1u;
+      if (!__all_sync(0xFFFFFFFFu, ok)) return false;
+      uint8_t* rowp = bufs + lane * 128;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        uint4* ptr = reinterpret_cast<uint4*>(rowp + ((j ^ (lane & 7)) << 4));
+        const uint4 rr = *ptr;
+        const uint32_t rw[4] = {rr.x, rr.y, rr.z, rr.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          o[e] = pack_bf16x2(__uint_as_float(v[8 * j + 2 * e]) * scale + bf16lo(rw[e]),
+                             __uint_as_float(v[8 * j + 2 * e + 1]) * scale + bf16hi(rw[e]));
+        *ptr = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_3d(tmH, bufs, col, row0, rank, pol_h);
+        bulk_commit_group();
+      }
+    }
+  }
+  if (lane == 0) bulk_wait_group_read0();
   __syncwarp();
   return true;
 }
@@ -543,9 +687,28 @@ __device__ __forceinline__ bool k1_wait_sdone(const RowparParams& prm, const uns
 // and then does the counting, so a warp that has left its loop on an error cannot block
 // the others.  Four barriers: a warp can be at most two tiles ahead of another (the TMEM
 // double buffer), so no warp arrives twice on a barrier before its phase completes.
+// Publication of one finished tile for the row-norm kernel running beside the GEMM (publish
+// mode 2), by one epilogue warp: complete the warp's box stores of the tile, order them (async
+// proxy, then a gpu-scope fence) before the counter updates, and add 1 to the counter of each
+// (128-row block, rank) the tile belongs to (every rank for a shared tile).  Called one tile
+// late, when the warp starts its next tile (or leaves), so the stores have had a mainloop's
+// time to complete and the wait rarely stalls.  Fire-and-forget reductions: no round trip.
+__device__ __forceinline__ void k1_publish_counts(const RowparParams& prm, int m128, int rank) {
+  if ((threadIdx.x & 31) == 0) {
+    bulk_wait_group0();
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    __threadfence();
+    const int r0 = rank < 0 ? 0 : rank;
+    const int r1 = rank < 0 ? prm.P : rank + 1;
+    unsigned int* c = prm.rb_count + static_cast<size_t>(m128) * prm.P;
+    for (int r = r0; r < r1; ++r) asm volatile("red.relaxed.gpu.global.add.u32 [%0], 1;" ::"l"(c + r) : "memory");
+  }
+  __syncwarp();
+}
+
 __device__ __forceinline__ void k1_signal_tile(const RowparParams& prm, uint64_t* sig, int tile_idx, int m128,
                                                int rank) {
-  if (!prm.fuse_norm) return;
+  if (prm.publish != 1) return;
   __threadfence();
   __syncwarp();
   const int lane = threadIdx.x & 31;

@@ -45,7 +45,7 @@ template <bool kFused, int kMajor = 0>
 __global__ void __launch_bounds__(K1Threads<kFused>::value, 1)
     rowpar_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                             const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmH,
-                            const __grid_constant__ RowparParams prm) {
+                            const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ RowparParams prm) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sA = smem;
@@ -90,6 +90,7 @@ __global__ void __launch_bounds__(K1Threads<kFused>::value, 1)
     tma_prefetch_desc(&tmW);
     tma_prefetch_desc(&tmR);
     tma_prefetch_desc(&tmH);
+    if (prm.zs_mode) tma_prefetch_desc(&tmZ);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_holder, K1_TMEM_COLS);
@@ -98,6 +99,9 @@ __global__ void __launch_bounds__(K1Threads<kFused>::value, 1)
   tc_fence_before();
   cluster_sync();  // barriers of both CTAs initialized, TMEM allocated, before any remote access
   tc_fence_after();
+  // A row-norm kernel launched as a programmatic dependent may start now, on the SMs this
+  // grid leaves free: it waits on the row-block job list, never on this grid's completion.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const uint32_t tmem_base = *tmem_holder;
   const uint64_t tmo = prm.timeout_ns;
   const uint32_t peer = cta ^ 1u;
@@ -212,10 +216,12 @@ __global__ void __launch_bounds__(K1Threads<kFused>::value, 1)
     uint64_t* my_rbar = rbar + (warp - 2) * K1_EPI_NBUF;
     uint32_t rphase = 0;
     const uint64_t pol_r = policy_evict_first();
-    // h is read back by the fused norm (from L2); otherwise streamed out, behind X and W
-    const uint64_t pol_h = kFused ? policy_evict_normal() : policy_evict_first();
+    // h is read back soon by the norm (fused, or the row-norm kernel beside this one), maybe
+    // still from L2; otherwise streamed out, behind X and W
+    const uint64_t pol_h = prm.publish ? policy_evict_normal() : policy_evict_first();
     const uint32_t tempty_leader[2] = {mapa_shared(smem_u32(&tempty[0]), 0), mapa_shared(smem_u32(&tempty[1]), 0)};
     int local = 0;
+    int pend_m128 = -1, pend_rank = 0;  // publish mode 2: the tile still to be counted
     for (int i = 0;; ++i) {
       const int slot = i % K1_SCHED;
       const uint32_t sph = (i / K1_SCHED) & 1;
@@ -239,12 +245,21 @@ __global__ void __launch_bounds__(K1Threads<kFused>::value, 1)
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
       if (!ok) break;
       tc_fence_after();
+      if (pend_m128 >= 0) {  // the previous tile's stores have had this tile's mainloop to land
+        k1_publish_counts(prm, pend_m128, pend_rank);
+        pend_m128 = -1;
+      }
       const uint32_t trow = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * K2P_BN);
       const int row = prm.t_begin + un.m * (2 * K2P_BM) + static_cast<int>(cta) * K2P_BM + q * 32 + lane;
       const int n0 = un.n * K2P_BN;
       const bool mixed = prm.ncls[un.n] == 2;
       const bool merge = mixed && !kFused && prm.merge_mixed;
-      if (!mixed || merge) {
+      if (prm.zs_mode) {
+        const int row0 = prm.t_begin + un.m * (2 * K2P_BM) + static_cast<int>(cta) * K2P_BM + q * 32;
+        if (!k1_epilogue_split(trow, prm, &tmR, &tmH, &tmZ, row0, n0, un.rank, my_bufs, my_rbar, rphase, lane,
+                               pol_r, pol_h))
+          break;
+      } else if (!mixed || merge) {
         const int row0 = prm.t_begin + un.m * (2 * K2P_BM) + static_cast<int>(cta) * K2P_BM + q * 32;
         // flag of this warp's 32 rows in column block n: [row group][n-block]
         unsigned int* flag =
@@ -264,9 +279,15 @@ __global__ void __launch_bounds__(K1Threads<kFused>::value, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty_leader[buf]);
-      k1_signal_tile(prm, sig, local, 2 * un.m + static_cast<int>(cta), un.rank);
+      if (prm.publish == 2) {
+        pend_m128 = 2 * un.m + static_cast<int>(cta);
+        pend_rank = un.rank;
+      } else {
+        k1_signal_tile(prm, sig, local, 2 * un.m + static_cast<int>(cta), un.rank);
+      }
       ++local;
     }
+    if (pend_m128 >= 0) k1_publish_counts(prm, pend_m128, pend_rank);
   }
 
   tc_fence_before();

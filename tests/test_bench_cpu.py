@@ -14,6 +14,23 @@ def test_algorithmic_bytes_of_the_fc2_7b_step():
     assert abs(bench.alg_bytes_of(T, K, H, P) / 1e6 - 1344.3) < 0.1
 
 
+def test_algorithmic_bytes_of_the_mlp_block():
+    # X [P,T,H] + A [P,2F/P,H] + Y [P,T,F/P] written and read + W2 [P,H,F/P] + residual + out + gamma
+    T, F, H, P = 4096, 11008, 4096, 8
+    x = P * T * H
+    a = P * (2 * F // P) * H
+    y = P * T * (F // P)
+    w2 = P * H * (F // P)
+    r = out = P * T * H
+    assert bench.alg_bytes_of(T, F, H, P, mlp=True) == 2.0 * (x + a + 2 * y + w2 + r + out + H)
+
+
+def test_algorithmic_flops():
+    T, K, H = 8192, 11008, 4096
+    assert bench.alg_flops_of(T, K, H) == 2.0 * T * K * H
+    assert abs(bench.alg_flops_of(4096, 11008, 4096, mlp=True) / 1e9 - 1108.1) < 0.1
+
+
 def test_traffic_record_follows_the_sources(monkeypatch, tmp_path):
     rec = {"source_sha256": "abc", "workloads": {"fc2-7b": {"gemm": {"read_bytes": 10, "write_bytes": 5}}}}
     (tmp_path / "profiles").mkdir()
