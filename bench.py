@@ -392,7 +392,8 @@ class Case:
 
 def time_case(case, steps, warmup, world=1, sample_clocks=False, local=0, soak_ms=500.0):
     """Times exactly `steps` steps after `warmup` untimed ones: CUDA events on the launching
-    stream, synchronize (and a barrier across ranks) on both sides.  Workloads whose bytes fit
+    stream, synchronize (and a barrier across ranks) on both sides; the per-kernel split comes
+    from `steps` more calls with the library's event recorder, after the timed region.  Workloads whose bytes fit
     in L2 (decode, tiny) get a READ of a buffer 3x the L2 size before every step (a write flush
     would leave dirty lines whose write-back the next step would pay for); each step is then
     timed alone, and is one replay of a CUDA graph holding the one library call (the same
@@ -439,10 +440,13 @@ def time_case(case, steps, warmup, world=1, sample_clocks=False, local=0, soak_m
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(steps):
-            case.step(timing)
+            case.step()
         e1.record(stream)
         torch.cuda.synchronize()
         ms_local = e0.elapsed_time(e1)
+        for _ in range(steps):   # per-kernel split: the library's events around each kernel (an
+            case.step(timing)    # event between two kernels holds the second back), not timed
+        torch.cuda.synchronize()
     # The timed region is short next to what NVML can sample (tens of ms): keep sampling while
     # the same step runs back to back for a while more (not timed), on every rank.
     soak_steps = 0

@@ -187,8 +187,12 @@ __global__ void __launch_bounds__(KB_THREADS, 1) rownorm_bwd_kernel(const __grid
 }
 
 // KB1s: the same as KB1 with the token's h and dout staged in shared memory (cp.async, P H 4
-// bytes), so that each is read from memory once and passes 2 and 3 read shared memory.  One
-// 8-channel vector of every rank per thread (H <= 8 * KB_THREADS).
+// bytes), so that each is read from memory once.  One 8-channel vector of every rank per thread
+// (H <= 8 * KB_THREADS); each thread stages and reads back only its own vectors, so the staging
+// needs no block barrier.  Pass 2 leaves in the h slot the private channels' bf16 result
+// s * dh, so pass 3 only selects; as soon as pass 2 is done with a token's dout, the next
+// token's dout is requested into its slot (and its h after pass 3), so those loads overlap the
+// stores of dZt.
 __global__ void __launch_bounds__(KB_THREADS, 1) rownorm_bwd_smem_kernel(const __grid_constant__ BwdParams prm) {
   extern __shared__ __align__(16) uint8_t kb_smem[];
   __shared__ float red[2 * KB_MAXP][KB_THREADS / 32];
@@ -198,7 +202,7 @@ __global__ void __launch_bounds__(KB_THREADS, 1) rownorm_bwd_smem_kernel(const _
   const int nvec = H >> 3;
   const float inv_h = 1.0f / static_cast<float>(H);
   const size_t rstride = static_cast<size_t>(prm.T) * H;
-  uint4* sh = reinterpret_cast<uint4*>(kb_smem);                    // [P][nvec] h
+  uint4* sh = reinterpret_cast<uint4*>(kb_smem);                    // [P][nvec] h, then s dh
   uint4* sd = sh + static_cast<size_t>(P) * nvec;                  // [P][nvec] dout
   const int v = threadIdx.x;
   const bool active = v < nvec;
@@ -209,18 +213,23 @@ __global__ void __launch_bounds__(KB_THREADS, 1) rownorm_bwd_smem_kernel(const _
   for (int e = 0; e < 8; ++e) dg[e] = 0.f;
   const uint32_t bits = active ? (prm.mask_bits[c >> 5] >> (c & 31)) & 0xFFu : 0u;
 
+  auto stage = [&](uint4* dst, const __nv_bfloat16* src, int64_t t) {
+    if (!active) return;
+    const size_t toff = static_cast<size_t>(t) * H + c;
+    for (int m = 0; m < P; ++m)
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst + m * nvec + v)),
+                   "l"(src + m * rstride + toff) : "memory");
+  };
+  if (blockIdx.x < prm.T) {
+    stage(sh, prm.h, blockIdx.x);
+    stage(sd, prm.dout, blockIdx.x);
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+
   for (int64_t t = blockIdx.x; t < prm.T; t += gridDim.x) {
     const size_t toff = static_cast<size_t>(t) * H + c;
-    if (active) {
-      for (int m = 0; m < P; ++m) {
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(sh + m * nvec + v)),
-                     "l"(prm.h + m * rstride + toff) : "memory");
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(sd + m * nvec + v)),
-                     "l"(prm.dout + m * rstride + toff) : "memory");
-      }
-    }
-    asm volatile("cp.async.commit_group;" ::: "memory");
-    asm volatile("cp.async.wait_group 0;" ::: "memory");  // each thread reads back only its own vectors
+    const int64_t tn = t + gridDim.x;  // this CTA's next token
+    asm volatile("cp.async.wait_group 0;" ::: "memory");  // this token's h and dout (own vectors)
     for (int m = 0; m < P; ++m) {
       float a = 0.f, b = 0.f;
       if (active) {
@@ -255,12 +264,13 @@ __global__ void __launch_bounds__(KB_THREADS, 1) rownorm_bwd_smem_kernel(const _
       s_k[threadIdx.x] = r * r * r * b * inv_h;
     }
     __syncthreads();
-    if (active) {
-      float S[8];
+    float S[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) S[e] = 0.f;
+    for (int e = 0; e < 8; ++e) S[e] = 0.f;
+    if (active) {
+      // pass 2: dh per rank -> dR, the shared sum S, dgamma; the h slot gets bf16(s dh)
       for (int m = 0; m < P; ++m) {
-        float hf[8], df[8], dh[8];
+        float hf[8], df[8], dh[8], zp[8];
         unpack8(sh[m * nvec + v], hf);
         unpack8(sd[m * nvec + v], df);
         const float r = s_r[m], kk = s_k[m];
@@ -269,22 +279,30 @@ __global__ void __launch_bounds__(KB_THREADS, 1) rownorm_bwd_smem_kernel(const _
           dh[e] = r * df[e] * gam[e] - hf[e] * kk;
           S[e] += dh[e];
           dg[e] = fmaf(df[e], hf[e] * r, dg[e]);
+          zp[e] = prm.private_scale * dh[e];
         }
         if (prm.dR != nullptr) *reinterpret_cast<uint4*>(prm.dR + m * rstride + toff) = pack8(dh);
+        sh[m * nvec + v] = pack8(zp);
       }
+    }
+    if (tn < prm.T) stage(sd, prm.dout, tn);  // dout of this token is no longer needed
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    if (active) {
+      // pass 3: dZt per rank (shared channels: S, private: s dh)
       for (int m = 0; m < P; ++m) {
-        float hf[8], df[8], z[8];
-        unpack8(sh[m * nvec + v], hf);
-        unpack8(sd[m * nvec + v], df);
-        const float r = s_r[m], kk = s_k[m];
+        float z[8];
+        unpack8(sh[m * nvec + v], z);
 #pragma unroll
         for (int e = 0; e < 8; ++e)
-          z[e] = ((bits >> e) & 1u) ? S[e] : prm.private_scale * (r * df[e] * gam[e] - hf[e] * kk);
+          if ((bits >> e) & 1u) z[e] = S[e];
         *reinterpret_cast<uint4*>(prm.dZt + m * rstride + toff) = pack8(z);
       }
     }
-    __syncthreads();  // red / s_r / s_k (and this thread's staging slots) are reused next token
+    if (tn < prm.T) stage(sh, prm.h, tn);  // the h slots were read back by this thread only
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    __syncthreads();  // red / s_r / s_k are reused next token
   }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
   if (active) {
     float4* dst = reinterpret_cast<float4*>(prm.dg_part + static_cast<size_t>(blockIdx.x) * H + c);
     dst[0] = make_float4(dg[0], dg[1], dg[2], dg[3]);

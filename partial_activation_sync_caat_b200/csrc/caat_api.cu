@@ -366,22 +366,15 @@ RowparWs rowpar_ws_layout(int64_t T, int64_t H, int P, bool fused) {
   return L;
 }
 
-// Decode path (T <= CAAT_DECODE_MAX_T, P <= 16): K splits of the weight-streaming kernel.
-// One split: the stream of W runs at the same speed with 1, 4 or 8 splits (its time is W
-// bytes plus a fixed launch-to-first-byte cost), and every extra split is one more partial
-// for the reduce kernel to gather.
-int decode_splits(int64_t T) {
-  (void)T;
-  return 1;
-}
-
+// Decode path (T <= CAAT_DECODE_MAX_T, P <= 16): the weight-streaming kernel splits the stream
+// of (unit, k-block) items evenly over its CTAs; a unit cut in two leaves two fp32 partials.
 bool decode_eligible(int64_t T, int P, int64_t H) {
   return T >= 1 && T <= CAAT_DECODE_MAX_T && P <= caat::K4_MAXP && H <= 4 * caat::K4B_THREADS * caat::K4B_VEC;
 }
 
-// Decode workspace: [256 B | Zp fp32 [splits][P][T][H]].
+// Decode workspace: [256 B | Zp fp32 [2 slots][P][T][H]].
 size_t decode_workspace(int64_t T, int64_t H, int P) {
-  return kCounterBytes + align256(size_t(decode_splits(T)) * P * T * H * 4);
+  return kCounterBytes + align256(size_t(2) * P * T * H * 4);
 }
 
 // Whether a call with these shapes and flags runs the decode (weight-streaming) kernels.
@@ -560,29 +553,47 @@ caat_status launch_decode(const caat_rowpar_args* a, const std::vector<uint8_t>&
   const int P = a->P;
   const int64_t T = a->T, H = a->H, Kp = a->K / P;
   cudaStream_t st = a->stream;
+  caat::DecodeGemmParams gp{};
+  gp.Zp = reinterpret_cast<float*>(ws + kCounterBytes);
+  gp.T = static_cast<int>(T);
+  gp.Tpad = static_cast<int>((T + 15) / 16 * 16);
+  gp.H = static_cast<int>(H);
+  gp.P = P;
+  gp.n_cb = static_cast<int>((H + caat::K4_BM - 1) / caat::K4_BM);
+  gp.kblk = static_cast<int>((Kp + caat::K4_BK - 1) / caat::K4_BK);
+  const int64_t tail = Kp - int64_t(gp.kblk - 1) * caat::K4_BK;
+  gp.last_k16 = static_cast<int>((tail + 15) / 16);
+  const int64_t units = int64_t(P) * gp.n_cb;
+  const int64_t items = units * gp.kblk;
+  if (items > INT32_MAX / 2) return CAAT_ERR_UNSUPPORTED;
+  gp.n_items = static_cast<int>(items);
+  gp.stages = caat::k4_stages(gp.Tpad);
+  gp.timeout_ns = timeout_ns();
+  // No more CTAs than units: every CTA then streams at least one unit's worth of items, so a
+  // unit is cut at most once (two partials).
+  const int grid = static_cast<int>(std::min<int64_t>(dev->sm_count, units));
+
   static thread_local caat::DecodeParams prm;
   std::memset(&prm, 0, sizeof(prm));
-  prm.Zp = reinterpret_cast<float*>(ws + kCounterBytes);
+  prm.Zp = gp.Zp;
   prm.R = reinterpret_cast<const __nv_bfloat16*>(a->residual);
   prm.Hout = reinterpret_cast<__nv_bfloat16*>(a->h_out ? a->h_out : a->out);
   prm.Out = reinterpret_cast<__nv_bfloat16*>(a->out);
   prm.gamma = reinterpret_cast<const __nv_bfloat16*>(a->gamma);
   prm.T = static_cast<int>(T);
-  prm.Tpad = static_cast<int>((T + 15) / 16 * 16);
   prm.H = static_cast<int>(H);
-  prm.Kp = static_cast<int>(Kp);
   prm.P = P;
-  prm.n_cb = static_cast<int>((H + caat::K4_BM - 1) / caat::K4_BM);
-  prm.kblk = static_cast<int>((Kp + caat::K4_BK - 1) / caat::K4_BK);
-  prm.splits = std::min(decode_splits(T), prm.kblk);
-  prm.kb_per_split = (prm.kblk + prm.splits - 1) / prm.splits;
-  prm.splits = (prm.kblk + prm.kb_per_split - 1) / prm.kb_per_split;
-  const int64_t tail = Kp - int64_t(prm.kblk - 1) * caat::K4_BK;
-  prm.last_k16 = static_cast<int>((tail + 15) / 16);
-  prm.n_units = P * prm.n_cb * prm.splits;
+  prm.n_cb = gp.n_cb;
+  prm.kblk = gp.kblk;
+  // units cut between two streaming CTAs (their first and last k-block have different owners)
+  if (units > int64_t(caat::K4_MAXP) * 64) return CAAT_ERR_UNSUPPORTED;
+  for (int64_t u = 0; u < units; ++u) {
+    const int64_t first = u * gp.kblk;
+    if (caat::k4_cta_of(first, items, grid) != caat::k4_cta_of(first + gp.kblk - 1, items, grid))
+      prm.split_bits[u >> 5] |= 1u << (u & 31);
+  }
   prm.private_scale = a->private_scale;
   prm.eps = a->eps;
-  prm.timeout_ns = timeout_ns();
   prm.permuted = (a->flags & CAAT_FLAG_W_PERMUTED) ? 1 : 0;
   for (int64_t c = 0; c < H; ++c)
     if (mask[c]) {
@@ -593,13 +604,12 @@ caat_status launch_decode(const caat_rowpar_args* a, const std::vector<uint8_t>&
   CUtensorMap tmW, tmX;
   caat_status s = make_map_3d(&tmW, a->W, Kp, H, P, caat::K4_BK, caat::K4_BM);
   if (s != CAAT_OK) return s;
-  s = make_map_3d(&tmX, a->X, Kp, T, P, caat::K4_BK, static_cast<uint32_t>(prm.Tpad));
+  s = make_map_3d(&tmX, a->X, Kp, T, P, caat::K4_BK, static_cast<uint32_t>(gp.Tpad));
   if (s != CAAT_OK) return s;
   Recorder own;
   Recorder& rec = outer ? *outer : own;
   if (!outer) rec.begin(a->timing, st);
-  const int grid = std::min(dev->sm_count, prm.n_units);
-  caat::decode_partials_kernel<<<grid, caat::K4_THREADS, caat::K4_SMEM_BYTES, st>>>(tmW, tmX, prm);
+  caat::decode_partials_kernel<<<grid, caat::K4_THREADS, caat::K4_SMEM_BYTES, st>>>(tmW, tmX, gp);
   if (cudaGetLastError() != cudaSuccess) return CAAT_ERR_CUDA;
   rec.after_kernel(st);
   // The reduce kernel is a programmatic dependent of the partials kernel: its launch overlaps
@@ -841,12 +851,28 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
       // row held in registers: VPL 128-bit vectors per lane
       int64_t rb = std::min<int64_t>((rows + warps_per_block - 1) / warps_per_block, int64_t(dev->sm_count) * 2);
       if (norm_blocks_cap() > 0) rb = std::min<int64_t>(rb, norm_blocks_cap());
+      // Right after the GEMM on the same stream: a programmatic dependent launch, so that the
+      // norm's launch overlaps the GEMM's tail (the kernel waits for the GEMM grid itself).
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[0].val.programmaticStreamSerializationAllowed = 1;
+      cfg.gridDim = dim3(static_cast<unsigned>(rb), 1, 1);
+      cfg.blockDim = dim3(caat::K2_THREADS, 1, 1);
+      cfg.stream = ns;
+      cfg.attrs = attr;
+      cfg.numAttrs = (ns == st && pair) ? 1 : 0;
+      const __nv_bfloat16* hc = hdst;
+      const int Hi = static_cast<int>(H);
+      const float ep = a->eps;
+      cudaError_t e;
       if (H <= 1024)
-        caat::rownorm_reg_kernel<4><<<rb, caat::K2_THREADS, 0, ns>>>(hdst, o, g, P, T, t0, tc, static_cast<int>(H), a->eps);
+        e = cudaLaunchKernelEx(&cfg, caat::rownorm_reg_kernel<4>, hc, o, g, P, T, t0, tc, Hi, ep);
       else if (H <= 2048)
-        caat::rownorm_reg_kernel<8><<<rb, caat::K2_THREADS, 0, ns>>>(hdst, o, g, P, T, t0, tc, static_cast<int>(H), a->eps);
+        e = cudaLaunchKernelEx(&cfg, caat::rownorm_reg_kernel<8>, hc, o, g, P, T, t0, tc, Hi, ep);
       else
-        caat::rownorm_reg_kernel<16><<<rb, caat::K2_THREADS, 0, ns>>>(hdst, o, g, P, T, t0, tc, static_cast<int>(H), a->eps);
+        e = cudaLaunchKernelEx(&cfg, caat::rownorm_reg_kernel<16>, hc, o, g, P, T, t0, tc, Hi, ep);
+      if (e != cudaSuccess) return CAAT_ERR_CUDA;
     } else {
       // wide rows: one CTA per row (H <= 65536 = 8 x 1024 x 8)
       const int64_t nb = std::min<int64_t>(rows, int64_t(dev->sm_count) * 8);

@@ -7,15 +7,21 @@
 // private scale (§4 Eq. 14-15), residual add and RMSNorm (§4 Eq. 9); §3.2 describes running
 // all tensor-parallel ranks on one device ("logical devices").
 //
-// K4a decode_partials_kernel: every (rank, 128-channel block, K split) is one unit; a
-//     persistent CTA streams W_m's 128 x (K/P)/splits slice with TMA and computes the swapped
-//     product D[c, t] = W_m[c,:] . X_m[t,:] with tcgen05.mma (M = 128 channels, N = T padded to
-//     a multiple of 16, fp32 in TMEM), then writes the fp32 partial Zp[split][m][t][c].  The
-//     tokens are the N side, so W (the only large operand) is read exactly once.
-// K4b decode_reduce_norm_kernel: one CTA per (rank m, token t) row.  It sums the K splits
-//     of rank m's partial, forms the shared channels' cross-rank sum (ranks and splits in
-//     order, fp32), applies the private scale, adds the residual, stores h (bf16), reduces the
-//     sum of squares of the stored h over the CTA and rescales the row held in registers:
+// K4a decode_partials_kernel: the work is the sequence of items (unit, k-block), a unit being
+//     (rank m, 128-channel block), k-blocks fastest.  Persistent CTA i takes the contiguous items
+//     [floor(i N / G), floor((i + 1) N / G)) (stream-K: every CTA streams the same number of W
+//     bytes, within one k-block).  It streams its W slices with TMA through a ring whose depth
+//     follows the token count (the X tile of a stage is T padded to 16 rows), and computes the
+//     swapped product D[c, t] = W_m[c,:] . X_m[t,:] with tcgen05.mma (M = 128 channels, N = T
+//     padded, fp32 in TMEM).  Each run of a CTA's items inside one unit (a segment) is one
+//     accumulation, written as an fp32 partial to Zp[slot][m][t][c]: slot 0 for the segment
+//     that starts the unit, slot 1 for the one that ends a unit split between two CTAs (the
+//     grid never exceeds the unit count, so a unit has at most two segments).  The tokens are
+//     the N side, so W (the only large operand) is read exactly once.
+// K4b decode_reduce_norm_kernel: one CTA per (rank m, token t) row.  It adds the two slots of
+//     a split unit, forms the shared channels' cross-rank sum (ranks in order, fp32), applies
+//     the private scale, adds the residual, stores h (bf16), reduces the sum of squares of the
+//     stored h over the CTA and rescales the row held in registers:
 //     out = h / sqrt(sum/H + eps) * gamma.
 #pragma once
 
@@ -27,49 +33,69 @@ namespace caat {
 
 constexpr int K4_BM = 128;                 // channels per unit
 constexpr int K4_BK = 64;
-constexpr int K4_STAGES = 8;
 constexpr int K4_MAXN = 64;                // max padded token count
-constexpr int K4_A_BYTES = K4_BM * K4_BK * 2;       // 16 KiB of W
-constexpr int K4_B_BYTES = K4_MAXN * K4_BK * 2;     // up to 8 KiB of X
-constexpr int K4_STAGE_BYTES = K4_A_BYTES + K4_B_BYTES;
+constexpr int K4_A_BYTES = K4_BM * K4_BK * 2;       // 16 KiB of W per stage
+constexpr int K4_RING_BYTES = 229376;      // stages of (W tile + X tile)
+constexpr int K4_MAX_STAGES = 12;
 constexpr int K4_THREADS = 192;
-constexpr int K4_SMEM_BYTES = 1024 + K4_STAGES * K4_STAGE_BYTES + 256;
+constexpr int K4_SMEM_BYTES = 1024 + K4_RING_BYTES + 512;
 constexpr int K4_TMEM_COLS = 128;          // two accumulators of up to 64 columns
 constexpr int K4_MAXP = 16;                // ranks supported by the reduce kernel
 constexpr int K4B_THREADS = 1024;
 constexpr int K4B_VEC = 2;                 // 4-channel groups per thread: H <= 4 * 1024 * 2 = 8192
 
+// Ring depth for a padded token count: stages of 16 KiB of W + Tpad x 128 B of X.
+__host__ __device__ constexpr int k4_stages(int Tpad) {
+  return (K4_RING_BYTES / (K4_A_BYTES + Tpad * 128)) < K4_MAX_STAGES ? (K4_RING_BYTES / (K4_A_BYTES + Tpad * 128))
+                                                                       : K4_MAX_STAGES;
+}
+
+// The streaming kernel's parameters (no channel mask: a small parameter block).
+struct DecodeGemmParams {
+  float* Zp;                  // [2][P][T][H] fp32 partials (slot 1: second segments of split units)
+  int T, Tpad, H, P;
+  int n_cb;                   // ceil(H / 128)
+  int kblk;                   // ceil(Kp / 64)
+  int last_k16;               // 16-wide steps in the last k-block of a rank
+  int n_items;                // P * n_cb * kblk
+  int stages;                 // ring depth
+  uint64_t timeout_ns;
+};
+
+// The reduce kernel's parameters.
 struct DecodeParams {
-  float* Zp;                  // [splits][P][T][H] fp32 partials
+  const float* Zp;            // [2][P][T][H]
   const __nv_bfloat16* R;     // residual [P, T, H]
   __nv_bfloat16* Hout;        // h [P, T, H]
   __nv_bfloat16* Out;         // out [P, T, H]
   const __nv_bfloat16* gamma;
-  int T, Tpad, H, Kp, P;
-  int n_cb;                   // ceil(H / 128)
-  int splits;                 // K splits
-  int kb_per_split;           // k-blocks (64) per split
-  int kblk;                   // ceil(Kp / 64)
-  int last_k16;               // 16-wide steps in the last k-block of a rank
-  int n_units;                // P * n_cb * splits
+  int T, H, P;
+  int n_cb, kblk;
   float private_scale, eps;
-  uint64_t timeout_ns;
   int permuted;               // 1: W's rows are channel-permuted (permuted.cuh): Zp columns are permuted
   int n_s;                    // shared channels (the permuted path's prefix length)
   uint32_t mask_bits[K1_MASK_WORDS];
+  uint32_t split_bits[K4_MAXP * 64 / 32];  // bit u: unit u = m * n_cb + cb has a second partial
 };
+
+// CTA of the streaming kernel that owns item x: the largest i with floor(i N / G) <= x.
+__host__ __device__ __forceinline__ int64_t k4_cta_of(int64_t x, int64_t N, int64_t G) {
+  return ((x + 1) * G + N - 1) / N - 1;
+}
 
 __global__ void __launch_bounds__(K4_THREADS, 1)
     decode_partials_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
-                           const __grid_constant__ DecodeParams prm) {
+                           const __grid_constant__ DecodeGemmParams prm) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  uint8_t* sA = smem;
-  uint8_t* sB = smem + K4_STAGES * K4_A_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + K4_STAGES * K4_STAGE_BYTES);
-  uint64_t* full = bars;
-  uint64_t* empty = full + K4_STAGES;
-  uint64_t* tfull = empty + K4_STAGES;
+  const int S = prm.stages;
+  const uint32_t b_bytes = static_cast<uint32_t>(prm.Tpad) * K4_BK * 2;
+  uint8_t* sA = smem;                               // [S] W tiles (16 KiB, 1024-aligned)
+  uint8_t* sB = smem + S * K4_A_BYTES;              // [S] X tiles (Tpad x 128 B, 1024-aligned)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + K4_RING_BYTES);
+  uint64_t* full = bars;                            // [K4_MAX_STAGES]
+  uint64_t* empty = full + K4_MAX_STAGES;           // [K4_MAX_STAGES]
+  uint64_t* tfull = empty + K4_MAX_STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* mma_done = tempty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
@@ -77,7 +103,7 @@ __global__ void __launch_bounds__(K4_THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < K4_STAGES; ++s) {
+    for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -101,8 +127,10 @@ __global__ void __launch_bounds__(K4_THREADS, 1)
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const uint32_t tmem_base = *tmem_holder;
   const uint64_t tmo = prm.timeout_ns;
-  const int per_rank = prm.n_cb * prm.splits;
-  const uint32_t b_bytes = static_cast<uint32_t>(prm.Tpad) * K4_BK * 2;
+  const int64_t N = prm.n_items, G = gridDim.x;
+  const int item0 = static_cast<int>(static_cast<int64_t>(blockIdx.x) * N / G);
+  const int item1 = static_cast<int>((static_cast<int64_t>(blockIdx.x) + 1) * N / G);
+  const int kblk = prm.kblk;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -111,21 +139,17 @@ __global__ void __launch_bounds__(K4_THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true, issued = false;
-      for (int u = blockIdx.x; u < prm.n_units && ok; u += gridDim.x) {
-        const int r = u / per_rank;
-        const int rem = u - r * per_rank;
-        const int cb = rem / prm.splits;
-        const int sp = rem - cb * prm.splits;
-        const int kb0 = sp * prm.kb_per_split;
-        const int kb1 = min(prm.kblk, kb0 + prm.kb_per_split);
-        for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1, tmo, 61)) { ok = false; break; }
-          mbar_arrive_expect_tx(&full[stage], K4_A_BYTES + b_bytes);
-          tma_load_3d(sA + stage * K4_A_BYTES, &tmW, &full[stage], kb * K4_BK, cb * K4_BM, r, pol_w);
-          tma_load_3d(sB + stage * K4_B_BYTES, &tmX, &full[stage], kb * K4_BK, 0, r, pol_x);
-          issued = true;
-          if (++stage == K4_STAGES) { stage = 0; phase ^= 1; }
-        }
+      for (int it = item0; it < item1; ++it) {
+        const int u = it / kblk;
+        const int kb = it - u * kblk;
+        const int r = u / prm.n_cb;
+        const int cb = u - r * prm.n_cb;
+        if (!mbar_wait(&empty[stage], phase ^ 1, tmo, 61)) { ok = false; break; }
+        mbar_arrive_expect_tx(&full[stage], K4_A_BYTES + b_bytes);
+        tma_load_3d(sA + stage * K4_A_BYTES, &tmW, &full[stage], kb * K4_BK, cb * K4_BM, r, pol_w);
+        tma_load_3d(sB + stage * b_bytes, &tmX, &full[stage], kb * K4_BK, 0, r, pol_x);
+        issued = true;
+        if (++stage == S) { stage = 0; phase ^= 1; }
       }
       if (!ok && issued) spin_ns(1000000);
     }
@@ -136,30 +160,30 @@ __global__ void __launch_bounds__(K4_THREADS, 1)
       uint32_t phase = 0;
       int local = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < prm.n_units && ok; u += gridDim.x) {
-        const int rem = u % per_rank;
-        const int sp = rem % prm.splits;
-        const int kb0 = sp * prm.kb_per_split;
-        const int kb1 = min(prm.kblk, kb0 + prm.kb_per_split);
+      for (int seg = item0; seg < item1 && ok;) {
+        const int u = seg / kblk;
+        const int seg_end = min(item1, (u + 1) * kblk);
         const int buf = local & 1;
         const uint32_t bph = (local >> 1) & 1;
         if (!mbar_wait(&tempty[buf], bph ^ 1, tmo, 62)) { ok = false; break; }
         tc_fence_after();
         const uint32_t dt = tmem_base + static_cast<uint32_t>(buf * K4_MAXN);
-        for (int kb = kb0; kb < kb1; ++kb) {
+        for (int it = seg; it < seg_end; ++it) {
           if (!mbar_wait(&full[stage], phase, tmo, 63)) { ok = false; break; }
-          const int nk16 = (kb == prm.kblk - 1) ? prm.last_k16 : (K4_BK / 16);
+          const int kb = it - u * kblk;
+          const int nk16 = (kb == kblk - 1) ? prm.last_k16 : (K4_BK / 16);
           const uint32_t a_addr = smem_u32(sA + stage * K4_A_BYTES);
-          const uint32_t b_addr = smem_u32(sB + stage * K4_B_BYTES);
+          const uint32_t b_addr = smem_u32(sB + stage * b_bytes);
           for (int kk = 0; kk < nk16; ++kk)
             umma_bf16(dt, sw128_kmajor_desc(a_addr + kk * 32), sw128_kmajor_desc(b_addr + kk * 32), idesc,
-                      (kb > kb0 || kk > 0) ? 1u : 0u);
+                      (it > seg || kk > 0) ? 1u : 0u);
           umma_commit(&empty[stage]);
-          if (++stage == K4_STAGES) { stage = 0; phase ^= 1; }
+          if (++stage == S) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
         umma_commit(&tfull[buf]);
         ++local;
+        seg = seg_end;
       }
       umma_commit(mma_done);
       mbar_wait(mma_done, 0, tmo, 64);
@@ -167,11 +191,12 @@ __global__ void __launch_bounds__(K4_THREADS, 1)
   } else {
     const int q = warp & 3;
     int local = 0;
-    for (int u = blockIdx.x; u < prm.n_units; u += gridDim.x) {
-      const int r = u / per_rank;
-      const int rem = u - r * per_rank;
-      const int cb = rem / prm.splits;
-      const int sp = rem - cb * prm.splits;
+    for (int seg = item0; seg < item1;) {
+      const int u = seg / kblk;
+      const int seg_end = min(item1, (u + 1) * kblk);
+      const int r = u / prm.n_cb;
+      const int cb = u - r * prm.n_cb;
+      const int slot = (seg == u * kblk) ? 0 : 1;  // the unit's first or second segment
       const int buf = local & 1;
       const uint32_t bph = (local >> 1) & 1;
       int ok = 1;
@@ -190,12 +215,13 @@ __global__ void __launch_bounds__(K4_THREADS, 1)
       if (lane == 0) mbar_arrive(&tempty[buf]);
       const int c = cb * K4_BM + q * 32 + lane;
       if (c < prm.H) {
-        float* zp = prm.Zp + ((static_cast<size_t>(sp) * prm.P + r) * prm.T) * prm.H + c;
+        float* zp = prm.Zp + ((static_cast<size_t>(slot) * prm.P + r) * prm.T) * prm.H + c;
 #pragma unroll
         for (int t = 0; t < K4_MAXN; ++t)
           if (t < prm.T) zp[static_cast<size_t>(t) * prm.H] = __uint_as_float(v[t]);
       }
       ++local;
+      seg = seg_end;
     }
   }
   tc_fence_before();
@@ -207,9 +233,15 @@ __global__ void __launch_bounds__(K4_THREADS, 1)
 // K4b: one CTA per (rank m, token t) row, 4 channels per thread and pass.  All loads a thread
 // needs for its 4 channels go out before any is used: the residual, and the fp32 partials of
 // every rank (the shared channels' cross-rank sum, in rank order 0..P-1; rank m's own partial
-// for the private ones), in batches of 8 ranks.  The stored h stays in registers for the
-// rescale after the block's sum-of-squares reduction.  Launched as a programmatic dependent
-// of K4a: the launch overlaps K4a's tail and griddepcontrol.wait orders the reads.
+// for the private ones), in batches of 8 ranks; a unit split between two streaming CTAs adds
+// its second slot.  The stored h stays in registers for the rescale after the block's
+// sum-of-squares reduction.  Launched as a programmatic dependent of K4a: the launch overlaps
+// K4a's tail and griddepcontrol.wait orders the reads.
+__device__ __forceinline__ bool k4_split(const DecodeParams& prm, int m, int cb) {
+  const int u = m * prm.n_cb + cb;
+  return (prm.split_bits[u >> 5] >> (u & 31)) & 1u;
+}
+
 __global__ void __launch_bounds__(K4B_THREADS, 1)
     decode_reduce_norm_kernel(const __grid_constant__ DecodeParams prm) {
   __shared__ float red[K4B_THREADS / 32];
@@ -220,7 +252,8 @@ __global__ void __launch_bounds__(K4B_THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int nq = prm.H >> 2;  // 4-channel groups
   const size_t rowoff = (static_cast<size_t>(r) * prm.T + t) * prm.H;
-  const size_t zstride = static_cast<size_t>(prm.T) * prm.H;  // between ranks (one K split)
+  const size_t zstride = static_cast<size_t>(prm.T) * prm.H;   // between ranks
+  const size_t slot1 = static_cast<size_t>(prm.P) * zstride;    // between the two slots
   const float* zrow = prm.Zp + static_cast<size_t>(t) * prm.H;
   __shared__ uint32_t s_mask[K1_MASK_WORDS];
   __shared__ int s_pre[K1_MASK_WORDS + 1];
@@ -245,44 +278,55 @@ __global__ void __launch_bounds__(K4B_THREADS, 1)
       for (int e = 0; e < 4; ++e) {
         const int pe = perm_pos(c + e, prm.n_s, s_mask, s_pre);
         const bool shared_e = (bits >> e) & 1u;
-        for (int sp = 0; sp < prm.splits; ++sp) {
-          const float* zb = zrow + static_cast<size_t>(sp) * prm.P * zstride + pe;
-          for (int m0 = 0; m0 < prm.P; m0 += 8) {
-            float z[8];
+        const int cbe = pe / K4_BM;
+        for (int m0 = 0; m0 < prm.P; m0 += 8) {
+          float z[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const int m = m0 + j;
-              z[j] = (m < prm.P && (shared_e || m == r)) ? __ldcg(zb + m * zstride) : 0.f;
+          for (int j = 0; j < 8; ++j) {
+            const int m = m0 + j;
+            z[j] = 0.f;
+            if (m < prm.P && (shared_e || m == r)) {
+              z[j] = __ldcg(zrow + m * zstride + pe);
+              if (k4_split(prm, m, cbe)) z[j] += __ldcg(zrow + slot1 + m * zstride + pe);
             }
+          }
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              S[e] += z[j];
-              if (m0 + j == r) own[e] += z[j];
-            }
+          for (int j = 0; j < 8; ++j) {
+            S[e] += z[j];
+            if (m0 + j == r) own[e] += z[j];
           }
         }
       }
     } else if (bits != 0u) {
-      for (int m0 = 0; m0 < prm.P; m0 += 8) {
-        for (int sp = 0; sp < prm.splits; ++sp) {
-          const float* zb = zrow + (static_cast<size_t>(sp) * prm.P + m0) * zstride + c;
-          float4 z[8];
+      const int cb = c / K4_BM;
+      for (int m0 = 0; m0 < prm.P; m0 += 4) {
+        const float* zb = zrow + static_cast<size_t>(m0) * zstride + c;
+        float4 z[4], w[4];
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            z[j] = (m0 + j < prm.P) ? __ldcg(reinterpret_cast<const float4*>(zb + j * zstride))
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = 0; j < 4; ++j) {
+          const bool in = m0 + j < prm.P;
+          z[j] = in ? __ldcg(reinterpret_cast<const float4*>(zb + j * zstride)) : make_float4(0.f, 0.f, 0.f, 0.f);
+          w[j] = (in && k4_split(prm, m0 + j, cb)) ? __ldcg(reinterpret_cast<const float4*>(zb + slot1 + j * zstride))
+                                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            S[0] += z[j].x; S[1] += z[j].y; S[2] += z[j].z; S[3] += z[j].w;
-            if (m0 + j == r) { own[0] += z[j].x; own[1] += z[j].y; own[2] += z[j].z; own[3] += z[j].w; }
-          }
+        for (int j = 0; j < 4; ++j) {
+          z[j].x += w[j].x; z[j].y += w[j].y; z[j].z += w[j].z; z[j].w += w[j].w;
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          S[0] += z[j].x; S[1] += z[j].y; S[2] += z[j].z; S[3] += z[j].w;
+          if (m0 + j == r) { own[0] += z[j].x; own[1] += z[j].y; own[2] += z[j].z; own[3] += z[j].w; }
         }
       }
     } else {
-      for (int sp = 0; sp < prm.splits; ++sp) {
-        const float4 w = __ldcg(reinterpret_cast<const float4*>(zrow + (static_cast<size_t>(sp) * prm.P + r) * zstride + c));
-        own[0] += w.x; own[1] += w.y; own[2] += w.z; own[3] += w.w;
+      const float* zb = zrow + static_cast<size_t>(r) * zstride + c;
+      float4 w = __ldcg(reinterpret_cast<const float4*>(zb));
+      if (k4_split(prm, r, c / K4_BM)) {
+        const float4 w2 = __ldcg(reinterpret_cast<const float4*>(zb + slot1));
+        w.x += w2.x; w.y += w2.y; w.z += w2.z; w.w += w2.w;
       }
+      own[0] = w.x; own[1] = w.y; own[2] = w.z; own[3] = w.w;
     }
     const uint32_t rw[2] = {rv.x, rv.y};
     uint32_t o[2];

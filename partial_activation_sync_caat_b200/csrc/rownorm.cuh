@@ -30,6 +30,10 @@ __global__ void __launch_bounds__(K2_THREADS, 2)
   const int nvec = H >> 3;
   const float inv_h = 1.0f / static_cast<float>(H);
   const uint4* g4 = reinterpret_cast<const uint4*>(gamma);
+  // Launched as a programmatic dependent of the GEMM kernel (its launch and block setup overlap
+  // the GEMM's tail): wait until the GEMM grid has completed and its h is visible.  A no-op
+  // when launched normally.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   // Rows in reverse order: the rows the GEMM wrote last (rank P-1's) may still be in L2.
   for (int64_t i0 = warp_global; i0 < rows; i0 += nwarps) {

@@ -73,7 +73,7 @@ def _backward(g, P, p, idx, private_scale=1.0, eps=1e-5, with_dR=True):
 @pytest.mark.parametrize("T,K,H,P,p,rand", [
     (1, 1024, 776, 4, 0.5, False), (37, 1024, 776, 4, 0.3, True), (300, 2048, 1288, 4, 0.5, False),
     (600, 1024, 776, 2, 0.0, False), (257, 1024, 520, 8, 1.0, False), (130, 512, 1032, 16, 0.5, True),
-    # H % 16 == 0: the 2-CTA cluster norm backward (fewer tokens than clusters in the first)
+    # H % 16 == 0 and few tokens (fewer tokens than CTAs in the first)
     (5, 1024, 1024, 4, 0.5, True), (300, 2048, 2048, 8, 0.25, False), (200, 512, 1024, 16, 0.5, False)])
 def test_backward_matches_oracle(T, K, H, P, p, rand):
     idx = I.random_sync_idx(H, O.n_sync(H, p), seed=T) if rand else None
