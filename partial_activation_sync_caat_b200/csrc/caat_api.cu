@@ -91,6 +91,8 @@ caat_status device_info(DeviceInfo** out) {
                                caat::K2P_SMEM_BYTES) != cudaSuccess ||
           cudaFuncSetAttribute(caat::rowpar_gemm_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                caat::K2P_SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(caat::rowpar_gemm_pair_kernel<false, 0, caat::K2P_STAGES_EPI, caat::K2P_EPI_NBUF_EPI>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, caat::K2P_SMEM_BYTES) != cudaSuccess ||
           cudaFuncSetAttribute(caat::rowpar_gemm_pair_kernel<false, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                caat::K2P_SMEM_BYTES) != cudaSuccess ||
           cudaFuncSetAttribute(caat::rowpar_gemm_pair_kernel<false, 3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -796,8 +798,14 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
       cfg.stream = st;
       cfg.attrs = attr;
       cfg.numAttrs = 1;
+      // units short in K (few k-blocks per rank): the split with more epilogue buffers
+      const bool epi_heavy = !fused && major == 0 && prm.kblk_per_rank <= 12;
       const cudaError_t e =
           fused ? cudaLaunchKernelEx(&cfg, caat::rowpar_gemm_pair_kernel<true>, tmX, tmW, tmR, tmH, tmZ, prm)
+          : epi_heavy
+              ? cudaLaunchKernelEx(
+                    &cfg, caat::rowpar_gemm_pair_kernel<false, 0, caat::K2P_STAGES_EPI, caat::K2P_EPI_NBUF_EPI>, tmX,
+                    tmW, tmR, tmH, tmZ, prm)
           : major == 2
               ? cudaLaunchKernelEx(&cfg, caat::rowpar_gemm_pair_kernel<false, 2>, tmX, tmW, tmR, tmH, tmZ, prm)
           : major == 3
@@ -851,28 +859,12 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
       // row held in registers: VPL 128-bit vectors per lane
       int64_t rb = std::min<int64_t>((rows + warps_per_block - 1) / warps_per_block, int64_t(dev->sm_count) * 2);
       if (norm_blocks_cap() > 0) rb = std::min<int64_t>(rb, norm_blocks_cap());
-      // Right after the GEMM on the same stream: a programmatic dependent launch, so that the
-      // norm's launch overlaps the GEMM's tail (the kernel waits for the GEMM grid itself).
-      cudaLaunchConfig_t cfg = {};
-      cudaLaunchAttribute attr[1];
-      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-      attr[0].val.programmaticStreamSerializationAllowed = 1;
-      cfg.gridDim = dim3(static_cast<unsigned>(rb), 1, 1);
-      cfg.blockDim = dim3(caat::K2_THREADS, 1, 1);
-      cfg.stream = ns;
-      cfg.attrs = attr;
-      cfg.numAttrs = (ns == st && pair) ? 1 : 0;
-      const __nv_bfloat16* hc = hdst;
-      const int Hi = static_cast<int>(H);
-      const float ep = a->eps;
-      cudaError_t e;
       if (H <= 1024)
-        e = cudaLaunchKernelEx(&cfg, caat::rownorm_reg_kernel<4>, hc, o, g, P, T, t0, tc, Hi, ep);
+        caat::rownorm_reg_kernel<4><<<rb, caat::K2_THREADS, 0, ns>>>(hdst, o, g, P, T, t0, tc, static_cast<int>(H), a->eps);
       else if (H <= 2048)
-        e = cudaLaunchKernelEx(&cfg, caat::rownorm_reg_kernel<8>, hc, o, g, P, T, t0, tc, Hi, ep);
+        caat::rownorm_reg_kernel<8><<<rb, caat::K2_THREADS, 0, ns>>>(hdst, o, g, P, T, t0, tc, static_cast<int>(H), a->eps);
       else
-        e = cudaLaunchKernelEx(&cfg, caat::rownorm_reg_kernel<16>, hc, o, g, P, T, t0, tc, Hi, ep);
-      if (e != cudaSuccess) return CAAT_ERR_CUDA;
+        caat::rownorm_reg_kernel<16><<<rb, caat::K2_THREADS, 0, ns>>>(hdst, o, g, P, T, t0, tc, static_cast<int>(H), a->eps);
     } else {
       // wide rows: one CTA per row (H <= 65536 = 8 x 1024 x 8)
       const int64_t nb = std::min<int64_t>(rows, int64_t(dev->sm_count) * 8);

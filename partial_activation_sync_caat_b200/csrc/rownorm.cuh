@@ -30,10 +30,6 @@ __global__ void __launch_bounds__(K2_THREADS, 2)
   const int nvec = H >> 3;
   const float inv_h = 1.0f / static_cast<float>(H);
   const uint4* g4 = reinterpret_cast<const uint4*>(gamma);
-  // Launched as a programmatic dependent of the GEMM kernel (its launch and block setup overlap
-  // the GEMM's tail): wait until the GEMM grid has completed and its h is visible.  A no-op
-  // when launched normally.
-  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   // Rows in reverse order: the rows the GEMM wrote last (rank P-1's) may still be in L2.
   for (int64_t i0 = warp_global; i0 < rows; i0 += nwarps) {
@@ -99,6 +95,7 @@ __global__ void __launch_bounds__(K2_THREADS, 2)
 //     counter, `progress`; the GEMM as a whole may run longer than the timeout), or when another
 //     wait set the status word.
 //   * h and out may alias.
+//   * With target 0 it is the plain bulk-copy row norm of every row (launched after the GEMM).
 constexpr int K2C_THREADS = 256;
 constexpr int K2C_ROWS_PER_JOB = 128;
 constexpr int K2C_ROWS_PER_PIECE = 8;
@@ -198,7 +195,8 @@ __global__ void __launch_bounds__(K2C_THREADS, 1)
         }
         const unsigned int* cnt = rb_count + static_cast<size_t>(jm) * P + jr;
         uint32_t v = 0;
-        if (lane == 0) v = ld_acquire_u32(cnt) >= target ? 1u : 0u;
+        // target 0: launched after the GEMM has finished (stream order), nothing to wait for
+        if (lane == 0) v = (target == 0u || ld_acquire_u32(cnt) >= target) ? 1u : 0u;
         v = __shfl_sync(0xFFFFFFFFu, v, 0);
         if (v == 0u && issued > consumed) break;  // not complete yet: work on the rows in flight
         if (v == 0u) {

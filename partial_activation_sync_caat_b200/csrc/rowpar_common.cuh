@@ -35,7 +35,7 @@ struct K1Threads {
 
 // TMA epilogue of pure column blocks: per epilogue warp, K1_EPI_NBUF shared-memory buffers of
 // one 32-row x 64-column bf16 box (128-byte rows, 128-byte swizzle).
-constexpr int K1_EPI_NBUF = 2;  // the no-residual epilogue's buffer reuse relies on 2 (wait_group.read 1)
+constexpr int K1_EPI_NBUF = 2;
 constexpr int K1_EPI_BOX_BYTES = 32 * 64 * 2;
 constexpr int K1_EPI_BYTES = 4 * K1_EPI_NBUF * K1_EPI_BOX_BYTES;  // per CTA
 constexpr int K1_NORM_WARP0 = 6;                 // first normalizer warp (fused RMSNorm)
@@ -381,11 +381,12 @@ __device__ __forceinline__ void k1_epilogue_shared(uint32_t trow, const RowparPa
 // the private scale for private units), rounds to bf16 in place, and the box is stored to h
 // by TMA.  Full 128-byte lines move in bulk; rows beyond T and columns beyond H are
 // zero-filled on load and clipped on store by the tensor maps.  Items are pipelined over
-// K1_EPI_NBUF buffers.  Returns false if a wait ran out.
+// NBUF buffers (K1_EPI_NBUF by default).  Returns false if a wait ran out.
 // Mixed column blocks (merge = true, private units only): the shared unit of the block has
 // already stored full boxes of h whose shared columns are final; the private unit loads that
 // h box together with the residual box, keeps the shared columns, writes its private columns
 // and stores the full box again (single-buffered).
+template <int NBUF = K1_EPI_NBUF>
 __device__ __forceinline__ bool k1_epilogue_tma(uint32_t trow, const RowparParams& prm, const void* tmR,
                                                 const void* tmH, int row0, int n0, int rank, int slot, uint8_t* bufs,
                                                 uint64_t* rbar, uint32_t& phase, int lane, uint64_t pol_r,
@@ -457,13 +458,13 @@ __device__ __forceinline__ bool k1_epilogue_tma(uint32_t trow, const RowparParam
     for (int i = 0; i < n_items; ++i) {
       const int ri = i / nch, c = i - ri * nch;
       const int r = rank < 0 ? ri : rank;
-      const int b = i % K1_EPI_NBUF;
+      const int b = i % NBUF;
       uint32_t v[64];
       __syncwarp();
       tmem_ld_32x32b_x32(trow + 64 * c, *reinterpret_cast<uint32_t(*)[32]>(v));
       tmem_ld_32x32b_x32(trow + 64 * c + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
       tmem_wait_ld();
-      if (lane == 0 && i >= K1_EPI_NBUF) bulk_wait_group_read1();  // the store from buffer b has read it
+      if (lane == 0 && i >= NBUF) bulk_wait_group_read<NBUF - 1>();  // the store from buffer b has read it
       __syncwarp();
       uint8_t* rowp = bufs + b * K1_EPI_BOX_BYTES + lane * 128;
 #pragma unroll
@@ -492,7 +493,7 @@ __device__ __forceinline__ bool k1_epilogue_tma(uint32_t trow, const RowparParam
     __syncwarp();
     return true;
   }
-  const int npre = min(K1_EPI_NBUF, n_items);
+  const int npre = min(NBUF, n_items);
   for (int i = 0; i < npre; ++i) {
     const int ri = i / nch, c = i - ri * nch;
     const int r = rank < 0 ? ri : rank;
@@ -505,7 +506,7 @@ __device__ __forceinline__ bool k1_epilogue_tma(uint32_t trow, const RowparParam
   for (int i = 0; i < n_items; ++i) {
     const int ri = i / nch, c = i - ri * nch;
     const int r = rank < 0 ? ri : rank;
-    const int b = i % K1_EPI_NBUF;
+    const int b = i % NBUF;
     uint32_t v[64];
     __syncwarp();
     tmem_ld_32x32b_x32(trow + 64 * c, *reinterpret_cast<uint32_t(*)[32]>(v));
@@ -543,7 +544,7 @@ __device__ __forceinline__ bool k1_epilogue_tma(uint32_t trow, const RowparParam
       if (row < prm.t_end) k1_put_partial(prm, r, row, slot, ss);
       ss = 0.f;
     }
-    const int nx = i + K1_EPI_NBUF;
+    const int nx = i + NBUF;
     if (nx < n_items) {
       if (lane == 0) {
         bulk_wait_group_read0();  // the store that read buffer b is done with it

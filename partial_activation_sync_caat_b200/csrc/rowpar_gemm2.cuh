@@ -34,14 +34,23 @@ namespace caat {
 constexpr int K2P_BM = 128;                     // rows per CTA (pair tile: 256)
 constexpr int K2P_BN = 256;                     // channels per pair tile (per CTA B half: 128)
 constexpr int K2P_BK = 64;
-constexpr int K2P_STAGES = 6;
 constexpr int K2P_A_BYTES = K2P_BM * K2P_BK * 2;        // 16 KiB
 constexpr int K2P_B_BYTES = (K2P_BN / 2) * K2P_BK * 2;  // 16 KiB
 constexpr int K2P_STAGE_BYTES = K2P_A_BYTES + K2P_B_BYTES;
-constexpr int K2P_SMEM_BYTES = 1024 + K2P_STAGES * K2P_STAGE_BYTES + K1_EPI_BYTES + 512;
+// Two shared-memory splits of the same size: 6 operand stages + 2 epilogue boxes per epilogue
+// warp (the default), or 5 stages + 4 boxes for workloads whose units are short in K (few k-blocks
+// per tile), where the epilogue's residual loads and h stores, not the operands, set the pace.
+constexpr int K2P_STAGES = 6;
+constexpr int K2P_STAGES_EPI = 5;
+constexpr int K2P_EPI_NBUF_EPI = 4;
+__host__ __device__ constexpr int k2p_smem_bytes(int stages, int nbuf) {
+  return 1024 + stages * K2P_STAGE_BYTES + 4 * nbuf * K1_EPI_BOX_BYTES + 512;
+}
+constexpr int K2P_SMEM_BYTES = k2p_smem_bytes(K2P_STAGES, K1_EPI_NBUF);
+static_assert(k2p_smem_bytes(K2P_STAGES_EPI, K2P_EPI_NBUF_EPI) <= K2P_SMEM_BYTES, "both splits fit the same size");
 constexpr uint64_t K2P_DRAIN_NS = 1000000;      // error path only: let copies in flight land
 
-template <bool kFused, int kMajor = 0>
+template <bool kFused, int kMajor = 0, int kStages = K2P_STAGES, int kEpiBuf = K1_EPI_NBUF>
 __global__ void __launch_bounds__(K1Threads<kFused>::value, 1)
     rowpar_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                             const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmH,
@@ -49,19 +58,19 @@ __global__ void __launch_bounds__(K1Threads<kFused>::value, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sA = smem;
-  uint8_t* sB = smem + K2P_STAGES * K2P_A_BYTES;
-  uint8_t* sEpi = smem + K2P_STAGES * K2P_STAGE_BYTES;  // [4 warps][K1_EPI_NBUF] boxes
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + K1_EPI_BYTES);
+  uint8_t* sB = smem + kStages * K2P_A_BYTES;
+  uint8_t* sEpi = smem + kStages * K2P_STAGE_BYTES;  // [4 warps][kEpiBuf] boxes
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + (4 * kEpiBuf * K1_EPI_BOX_BYTES));
   uint64_t* full = bars;                    // [STAGES]  used in the leader
-  uint64_t* empty = full + K2P_STAGES;      // [STAGES]  both CTAs (multicast commit)
-  uint64_t* tfull = empty + K2P_STAGES;     // [2]       both CTAs (multicast commit)
+  uint64_t* empty = full + kStages;      // [STAGES]  both CTAs (multicast commit)
+  uint64_t* tfull = empty + kStages;     // [2]       both CTAs (multicast commit)
   uint64_t* tempty = tfull + 2;             // [2]       leader: 4 local + 4 peer warps
   uint64_t* sfull = tempty + 2;             // [SCHED]   both CTAs (leader producer arrives)
   uint64_t* sempty = sfull + K1_SCHED;      // [SCHED]   leader: 5 local + 5 peer arrivals
   uint64_t* mma_done = sempty + K1_SCHED;   // [1]       leader
   uint64_t* sig = mma_done + 1;                   // [4] epilogue warps meet per tile
-  uint64_t* rbar = sig + 4;                        // [4 warps][K1_EPI_NBUF]
-  int* sched_unit = reinterpret_cast<int*>(rbar + 4 * K1_EPI_NBUF);  // [SCHED] both CTAs
+  uint64_t* rbar = sig + 4;                        // [4 warps][kEpiBuf]
+  int* sched_unit = reinterpret_cast<int*>(rbar + 4 * kEpiBuf);  // [SCHED] both CTAs
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sched_unit + K1_SCHED);
 
   const int warp = threadIdx.x >> 5;
@@ -70,7 +79,7 @@ __global__ void __launch_bounds__(K1Threads<kFused>::value, 1)
   const bool leader = cta == 0;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < K2P_STAGES; ++s) {
+    for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -84,7 +93,7 @@ __global__ void __launch_bounds__(K1Threads<kFused>::value, 1)
     }
     mbar_init(mma_done, 1);
     for (int b = 0; b < 4; ++b) mbar_init(&sig[b], K1Threads<kFused>::epi_warps);
-    for (int b = 0; b < 4 * K1_EPI_NBUF; ++b) mbar_init(&rbar[b], 1);
+    for (int b = 0; b < 4 * kEpiBuf; ++b) mbar_init(&rbar[b], 1);
     fence_mbar_init();
     tma_prefetch_desc(&tmX);
     tma_prefetch_desc(&tmW);
@@ -156,7 +165,7 @@ __global__ void __launch_bounds__(K1Threads<kFused>::value, 1)
               tma_load_3d_pair(sB + stage * K2P_B_BYTES, &tmW, fbar, kb * K2P_BK, wrow, r, pol_w);
             }
             issued = true;
-            if (++stage == K2P_STAGES) { stage = 0; phase ^= 1; }
+            if (++stage == kStages) { stage = 0; phase ^= 1; }
           }
         }
       }
@@ -196,7 +205,7 @@ __global__ void __launch_bounds__(K1Threads<kFused>::value, 1)
             umma_bf16_pair(dt, ad, bd, idesc, (j > 0 || kk > 0) ? 1u : 0u);
           }
           umma_commit_pair_mc(&empty[stage], 0x3);
-          if (++stage == K2P_STAGES) { stage = 0; phase ^= 1; }
+          if (++stage == kStages) { stage = 0; phase ^= 1; }
           if (++kb_in_rank == prm.kblk_per_rank) kb_in_rank = 0;
         }
         if (!ok) break;
@@ -212,8 +221,8 @@ __global__ void __launch_bounds__(K1Threads<kFused>::value, 1)
   } else {
     // ---------------------------------------------------------------- epilogue warps
     const int q = warp & 3;
-    uint8_t* my_bufs = sEpi + (warp - 2) * K1_EPI_NBUF * K1_EPI_BOX_BYTES;
-    uint64_t* my_rbar = rbar + (warp - 2) * K1_EPI_NBUF;
+    uint8_t* my_bufs = sEpi + (warp - 2) * kEpiBuf * K1_EPI_BOX_BYTES;
+    uint64_t* my_rbar = rbar + (warp - 2) * kEpiBuf;
     uint32_t rphase = 0;
     const uint64_t pol_r = policy_evict_first();
     // h is read back soon by the norm (fused, or the row-norm kernel beside this one), maybe
@@ -267,7 +276,7 @@ __global__ void __launch_bounds__(K1Threads<kFused>::value, 1)
                                  un.n)
                   : nullptr;
         if (merge && un.rank >= 0 && !k1_wait_sdone(prm, flag)) break;
-        if (!k1_epilogue_tma(trow, prm, &tmR, &tmH, row0, n0, un.rank, un.slot, my_bufs, my_rbar, rphase, lane,
+        if (!k1_epilogue_tma<kEpiBuf>(trow, prm, &tmR, &tmH, row0, n0, un.rank, un.slot, my_bufs, my_rbar, rphase, lane,
                              pol_r, pol_h, merge && un.rank >= 0))
           break;
         if (merge && un.rank < 0) k1_signal_sdone(flag);
