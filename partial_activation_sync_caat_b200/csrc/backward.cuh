@@ -193,6 +193,7 @@ __global__ void __launch_bounds__(KB_THREADS, 1) rownorm_bwd_kernel(const __grid
 // s * dh, so pass 3 only selects; as soon as pass 2 is done with a token's dout, the next
 // token's dout is requested into its slot (and its h after pass 3), so those loads overlap the
 // stores of dZt.
+template <int MAXP>  // P <= MAXP (8 or 16)
 __global__ void __launch_bounds__(KB_THREADS, 1) rownorm_bwd_smem_kernel(const __grid_constant__ BwdParams prm) {
   extern __shared__ __align__(16) uint8_t kb_smem[];
   __shared__ float red[2 * KB_MAXP][KB_THREADS / 32];
@@ -230,9 +231,12 @@ __global__ void __launch_bounds__(KB_THREADS, 1) rownorm_bwd_smem_kernel(const _
     const size_t toff = static_cast<size_t>(t) * H + c;
     const int64_t tn = t + gridDim.x;  // this CTA's next token
     asm volatile("cp.async.wait_group 0;" ::: "memory");  // this token's h and dout (own vectors)
-    for (int m = 0; m < P; ++m) {
+    // per rank m: value m = sum of h^2, value MAXP + m = sum of g h over this thread's channels
+    float sums[2 * MAXP];
+#pragma unroll
+    for (int m = 0; m < MAXP; ++m) {
       float a = 0.f, b = 0.f;
-      if (active) {
+      if (active && m < P) {
         float hf[8], df[8];
         unpack8(sh[m * nvec + v], hf);
         unpack8(sd[m * nvec + v], df);
@@ -242,14 +246,16 @@ __global__ void __launch_bounds__(KB_THREADS, 1) rownorm_bwd_smem_kernel(const _
           b = fmaf(df[e] * gam[e], hf[e], b);
         }
       }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        a += __shfl_xor_sync(0xFFFFFFFFu, a, off);
-        b += __shfl_xor_sync(0xFFFFFFFFu, b, off);
-      }
-      if (lane == 0) {
-        red[2 * m][warp] = a;
-        red[2 * m + 1][warp] = b;
+      sums[m] = a;
+      sums[MAXP + m] = b;
+    }
+    warp_sum_many<2 * MAXP>(sums, lane);
+    {
+      constexpr int kShift = (2 * MAXP == 32) ? 0 : (2 * MAXP == 16 ? 1 : 2);
+      const int idx = lane >> kShift;  // the value this lane holds the warp total of
+      if ((lane & ((1 << kShift) - 1)) == 0) {
+        const int m = idx % MAXP;
+        if (m < P) red[2 * m + (idx >= MAXP ? 1 : 0)][warp] = sums[0];
       }
     }
     __syncthreads();

@@ -101,7 +101,9 @@ caat_status device_info(DeviceInfo** out) {
                                caat::K3_SMEM_BYTES) != cudaSuccess ||
           cudaFuncSetAttribute(caat::decode_partials_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                caat::K4_SMEM_BYTES) != cudaSuccess ||
-          cudaFuncSetAttribute(caat::rownorm_bwd_smem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+          cudaFuncSetAttribute(caat::rownorm_bwd_smem_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(caat::KB_SMEM_MAX)) != cudaSuccess ||
+          cudaFuncSetAttribute(caat::rownorm_bwd_smem_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(caat::KB_SMEM_MAX)) != cudaSuccess ||
           cudaFuncSetAttribute(caat::rownorm_gather_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(caat::gather_smem_bytes(1024))) != cudaSuccess ||
@@ -180,6 +182,32 @@ int consumer_order_setting() {
     const char* e = std::getenv("CAAT_ORDER");
     const int o = (e && *e) ? std::atoi(e) : 0;
     return (o >= 0 && o <= 3) ? o : 0;
+  }();
+  return v;
+}
+// Largest k-blocks per rank for which the GEMM takes the epilogue-heavy shared-memory split
+// (tuning; CAAT_EPI_HEAVY_KBLK).
+int epi_heavy_kblk_setting() {
+  static int v = [] {
+    const char* e = std::getenv("CAAT_EPI_HEAVY_KBLK");
+    return (e && *e) ? std::atoi(e) : 12;
+  }();
+  return v;
+}
+// Smallest token count whose decode reduce runs one CTA per token (tuning; CAAT_DECODE_TOKEN_T).
+int decode_token_min_t() {
+  static int v = [] {
+    const char* e = std::getenv("CAAT_DECODE_TOKEN_T");
+    return (e && *e) ? std::max(1, std::atoi(e)) : 9;
+  }();
+  return v;
+}
+// Whether the decode streaming kernel splits its items evenly, cutting units (tuning;
+// CAAT_DECODE_STREAMK).
+bool decode_stream_k_setting() {
+  static bool v = [] {
+    const char* e = std::getenv("CAAT_DECODE_STREAMK");
+    return (e && *e) ? (*e == '1') : true;
   }();
   return v;
 }
@@ -371,7 +399,7 @@ RowparWs rowpar_ws_layout(int64_t T, int64_t H, int P, bool fused) {
 // Decode path (T <= CAAT_DECODE_MAX_T, P <= 16): the weight-streaming kernel splits the stream
 // of (unit, k-block) items evenly over its CTAs; a unit cut in two leaves two fp32 partials.
 bool decode_eligible(int64_t T, int P, int64_t H) {
-  return T >= 1 && T <= CAAT_DECODE_MAX_T && P <= caat::K4_MAXP && H <= 4 * caat::K4B_THREADS * caat::K4B_VEC;
+  return T >= 1 && T <= CAAT_DECODE_MAX_T && P <= caat::K4_MAXP && H <= caat::K4B_MAX_H;
 }
 
 // Decode workspace: [256 B | Zp fp32 [2 slots][P][T][H]].
@@ -589,7 +617,8 @@ caat_status launch_decode(const caat_rowpar_args* a, const std::vector<uint8_t>&
   prm.kblk = gp.kblk;
   // units cut between two streaming CTAs (their first and last k-block have different owners)
   if (units > int64_t(caat::K4_MAXP) * 64) return CAAT_ERR_UNSUPPORTED;
-  for (int64_t u = 0; u < units; ++u) {
+  gp.stream_k = decode_stream_k_setting() ? 1 : 0;
+  for (int64_t u = 0; gp.stream_k && u < units; ++u) {
     const int64_t first = u * gp.kblk;
     if (caat::k4_cta_of(first, items, grid) != caat::k4_cta_of(first + gp.kblk - 1, items, grid))
       prm.split_bits[u >> 5] |= 1u << (u & 31);
@@ -620,13 +649,19 @@ caat_status launch_decode(const caat_rowpar_args* a, const std::vector<uint8_t>&
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.gridDim = dim3(static_cast<unsigned>(P * T), 1, 1);
-  cfg.blockDim = dim3(caat::K4B_THREADS, 1, 1);
+  // few tokens: one CTA per (rank, token) row; more: one CTA per token (shared sum formed once)
+  const bool per_row = T < decode_token_min_t();
+  cfg.gridDim = dim3(static_cast<unsigned>(per_row ? P * T : T), 1, 1);
+  cfg.blockDim = dim3(per_row ? caat::K4B_THREADS : caat::K4T_THREADS, 1, 1);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, caat::decode_reduce_norm_kernel, prm) != cudaSuccess) return CAAT_ERR_CUDA;
+  const cudaError_t e =
+      per_row  ? cudaLaunchKernelEx(&cfg, caat::decode_reduce_norm_kernel<caat::K4B_THREADS, caat::K4B_VEC>, prm)
+      : P <= 8 ? cudaLaunchKernelEx(&cfg, caat::decode_reduce_token_kernel<8>, prm)
+               : cudaLaunchKernelEx(&cfg, caat::decode_reduce_token_kernel<16>, prm);
+  if (e != cudaSuccess) return CAAT_ERR_CUDA;
   rec.after_kernel(st);
   return CAAT_OK;
 }
@@ -799,7 +834,7 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
       cfg.attrs = attr;
       cfg.numAttrs = 1;
       // units short in K (few k-blocks per rank): the split with more epilogue buffers
-      const bool epi_heavy = !fused && major == 0 && prm.kblk_per_rank <= 12;
+      const bool epi_heavy = !fused && major == 0 && prm.kblk_per_rank <= epi_heavy_kblk_setting();
       const cudaError_t e =
           fused ? cudaLaunchKernelEx(&cfg, caat::rowpar_gemm_pair_kernel<true>, tmX, tmW, tmR, tmH, tmZ, prm)
           : epi_heavy
@@ -1128,7 +1163,12 @@ caat_status caat_rowpar_backward(const caat_rowpar_bwd_args* a) {
     if (mask[c]) bp.mask_bits[c >> 5] |= 1u << (c & 31);
   const size_t kb_smem = caat::bwd_smem_bytes(P, static_cast<int>(H));
   if (H <= 8 * caat::KB_THREADS && kb_smem <= caat::KB_SMEM_MAX)
-    caat::rownorm_bwd_smem_kernel<<<L.nb, caat::KB_THREADS, kb_smem, st>>>(bp);
+  {
+    if (P <= 8)
+      caat::rownorm_bwd_smem_kernel<8><<<L.nb, caat::KB_THREADS, kb_smem, st>>>(bp);
+    else
+      caat::rownorm_bwd_smem_kernel<16><<<L.nb, caat::KB_THREADS, kb_smem, st>>>(bp);
+  }
   else
     caat::rownorm_bwd_kernel<<<L.nb, caat::KB_THREADS, 0, st>>>(bp);
   if (cudaGetLastError() != cudaSuccess) return CAAT_ERR_CUDA;

@@ -41,8 +41,15 @@ constexpr int K4_THREADS = 192;
 constexpr int K4_SMEM_BYTES = 1024 + K4_RING_BYTES + 512;
 constexpr int K4_TMEM_COLS = 128;          // two accumulators of up to 64 columns
 constexpr int K4_MAXP = 16;                // ranks supported by the reduce kernel
+// The reduce kernels: 1024 threads, VEC 4-channel groups per thread, H <= 4 * 1024 * VEC = 8192.
+// Few tokens (T <= 8): one CTA per (rank, token) row; more tokens: one CTA per token, all ranks.
 constexpr int K4B_THREADS = 1024;
-constexpr int K4B_VEC = 2;                 // 4-channel groups per thread: H <= 4 * 1024 * 2 = 8192
+constexpr int K4B_VEC = 2;
+constexpr int K4B_MAX_H = 4 * K4B_THREADS * K4B_VEC;
+constexpr int K4T_THREADS = 512;            // the per-token kernel (registers for every rank's sums)
+constexpr int K4T_VEC = K4B_MAX_H / (4 * K4T_THREADS);
+// The reduce kernels' channel mask covers only the decode path's rows (a small parameter block).
+constexpr int K4_MASK_WORDS = K4B_MAX_H / 32;
 
 // Ring depth for a padded token count: stages of 16 KiB of W + Tpad x 128 B of X.
 __host__ __device__ constexpr int k4_stages(int Tpad) {
@@ -59,6 +66,7 @@ struct DecodeGemmParams {
   int last_k16;               // 16-wide steps in the last k-block of a rank
   int n_items;                // P * n_cb * kblk
   int stages;                 // ring depth
+  int stream_k;               // 1: split the items evenly (units may be cut); 0: whole units
   uint64_t timeout_ns;
 };
 
@@ -74,7 +82,7 @@ struct DecodeParams {
   float private_scale, eps;
   int permuted;               // 1: W's rows are channel-permuted (permuted.cuh): Zp columns are permuted
   int n_s;                    // shared channels (the permuted path's prefix length)
-  uint32_t mask_bits[K1_MASK_WORDS];
+  uint32_t mask_bits[K4_MASK_WORDS];         // bit c = channel c is shared (H <= K4B_MAX_H)
   uint32_t split_bits[K4_MAXP * 64 / 32];  // bit u: unit u = m * n_cb + cb has a second partial
 };
 
@@ -128,8 +136,12 @@ __global__ void __launch_bounds__(K4_THREADS, 1)
   const uint32_t tmem_base = *tmem_holder;
   const uint64_t tmo = prm.timeout_ns;
   const int64_t N = prm.n_items, G = gridDim.x;
-  const int item0 = static_cast<int>(static_cast<int64_t>(blockIdx.x) * N / G);
-  const int item1 = static_cast<int>((static_cast<int64_t>(blockIdx.x) + 1) * N / G);
+  // stream-K: an even share of the items; otherwise an even share of whole units
+  const int64_t U = N / prm.kblk;
+  const int item0 = prm.stream_k ? static_cast<int>(static_cast<int64_t>(blockIdx.x) * N / G)
+                                 : static_cast<int>(static_cast<int64_t>(blockIdx.x) * U / G) * prm.kblk;
+  const int item1 = prm.stream_k ? static_cast<int>((static_cast<int64_t>(blockIdx.x) + 1) * N / G)
+                                 : static_cast<int>((static_cast<int64_t>(blockIdx.x) + 1) * U / G) * prm.kblk;
   const int kblk = prm.kblk;
 
   if (warp == 0) {
@@ -242,9 +254,10 @@ __device__ __forceinline__ bool k4_split(const DecodeParams& prm, int m, int cb)
   return (prm.split_bits[u >> 5] >> (u & 31)) & 1u;
 }
 
-__global__ void __launch_bounds__(K4B_THREADS, 1)
+template <int THREADS, int VEC>
+__global__ void __launch_bounds__(THREADS, THREADS >= 1024 ? 1 : 2)
     decode_reduce_norm_kernel(const __grid_constant__ DecodeParams prm) {
-  __shared__ float red[K4B_THREADS / 32];
+  __shared__ float red[THREADS / 32];
   __shared__ float s_rstd;
   const int r = blockIdx.x % prm.P;
   const int t = blockIdx.x / prm.P;
@@ -255,17 +268,20 @@ __global__ void __launch_bounds__(K4B_THREADS, 1)
   const size_t zstride = static_cast<size_t>(prm.T) * prm.H;   // between ranks
   const size_t slot1 = static_cast<size_t>(prm.P) * zstride;    // between the two slots
   const float* zrow = prm.Zp + static_cast<size_t>(t) * prm.H;
-  __shared__ uint32_t s_mask[K1_MASK_WORDS];
-  __shared__ int s_pre[K1_MASK_WORDS + 1];
+  __shared__ uint32_t s_mask[K4_MASK_WORDS];
+  __shared__ int s_pre[K4_MASK_WORDS + 1];
   if (prm.permuted) mask_prefix(prm.mask_bits, (prm.H + 31) >> 5, s_mask, s_pre);
   asm volatile("griddepcontrol.wait;" ::: "memory");  // K4a's partials are complete and visible
 
-  static_assert(K4B_VEC == 2, "h of the two passes is held in hv0 / hv1");
-  uint2 hv0 = make_uint2(0u, 0u), hv1 = make_uint2(0u, 0u);
+  // the stored h of the thread's groups, in registers (selected by constant indices: the loop
+  // over groups itself is not unrolled, which keeps the 1024-thread shape within its registers)
+  uint2 hv[VEC];
+#pragma unroll
+  for (int j = 0; j < VEC; ++j) hv[j] = make_uint2(0u, 0u);
   float ss = 0.f;
 #pragma unroll 1
-  for (int k = 0; k < K4B_VEC; ++k) {
-    const int g = threadIdx.x + k * K4B_THREADS;
+  for (int k = 0; k < VEC; ++k) {
+    const int g = threadIdx.x + k * THREADS;
     if (g >= nq) continue;
     const int c = 4 * g;
     const uint32_t bits = (prm.mask_bits[c >> 5] >> (c & 31)) & 0xFu;  // 4 channels, 4-aligned
@@ -340,7 +356,9 @@ __global__ void __launch_bounds__(K4B_THREADS, 1)
       ss = fmaf(hi, hi, ss);
     }
     const uint2 hk = make_uint2(o[0], o[1]);
-    if (k == 0) hv0 = hk; else hv1 = hk;
+#pragma unroll
+    for (int j = 0; j < VEC; ++j)
+      if (j == k) hv[j] = hk;
     *reinterpret_cast<uint2*>(prm.Hout + rowoff + c) = hk;
   }
 #pragma unroll
@@ -349,17 +367,20 @@ __global__ void __launch_bounds__(K4B_THREADS, 1)
   __syncthreads();
   if (threadIdx.x == 0) {
     float v = 0.f;
-    for (int w = 0; w < K4B_THREADS / 32; ++w) v += red[w];
+    for (int w = 0; w < THREADS / 32; ++w) v += red[w];
     s_rstd = rsqrtf(v / static_cast<float>(prm.H) + prm.eps);
   }
   __syncthreads();
   const float rs = s_rstd;
 #pragma unroll
-  for (int k = 0; k < K4B_VEC; ++k) {
-    const int g = threadIdx.x + k * K4B_THREADS;
+  for (int k = 0; k < VEC; ++k) {
+    const int g = threadIdx.x + k * THREADS;
     if (g >= nq) continue;
     const uint2 gv = *reinterpret_cast<const uint2*>(prm.gamma + 4 * g);
-    const uint2 hk = k == 0 ? hv0 : hv1;
+    uint2 hk = hv[0];
+#pragma unroll
+    for (int j = 1; j < VEC; ++j)
+      if (j == k) hk = hv[j];
     const uint32_t w[2] = {hk.x, hk.y};
     const uint32_t gw[2] = {gv.x, gv.y};
     uint32_t o[2];
@@ -367,6 +388,147 @@ __global__ void __launch_bounds__(K4B_THREADS, 1)
     for (int e = 0; e < 2; ++e)
       o[e] = pack_bf16x2(bf16lo(w[e]) * rs * bf16lo(gw[e]), bf16hi(w[e]) * rs * bf16hi(gw[e]));
     *reinterpret_cast<uint2*>(prm.Out + rowoff + 4 * g) = make_uint2(o[0], o[1]);
+  }
+}
+
+// K4b' (T > 8): one CTA per token (512 threads), all ranks, 4 channels per thread and group.  For a
+// group, every rank's fp32 partial (a split unit's two slots added) and residual are loaded in one
+// round before anything is stored (the loads of later ranks cannot wait behind earlier ranks'
+// stores); the shared channels' cross-rank sum is formed once (ranks in order), each rank's h is
+// stored (shared: the sum; private: scale x the rank's own partial; plus the residual) and its sum
+// of squares accumulated.  The per-rank sums are reduced over the block (warp_sum_many), then
+// every rank's h of the group is read back in one round and out written.  The same arithmetic per
+// element as K4b.
+template <int MAXP>  // P <= MAXP
+__global__ void __launch_bounds__(K4T_THREADS, 1)
+    decode_reduce_token_kernel(const __grid_constant__ DecodeParams prm) {
+  __shared__ float red[MAXP][K4T_THREADS / 32];
+  __shared__ float s_rstd[MAXP];
+  __shared__ uint32_t s_mask[K4_MASK_WORDS];
+  __shared__ int s_pre[K4_MASK_WORDS + 1];
+  const int t = blockIdx.x;
+  const int P = prm.P;
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int nq = prm.H >> 2;
+  const size_t zstride = static_cast<size_t>(prm.T) * prm.H;    // between ranks
+  const size_t slot1 = static_cast<size_t>(P) * zstride;         // between the two slots
+  const size_t rstride = static_cast<size_t>(prm.T) * prm.H;     // between ranks of R, h, out
+  const float* zrow = prm.Zp + static_cast<size_t>(t) * prm.H;
+  const size_t trow = static_cast<size_t>(t) * prm.H;
+  if (prm.permuted) mask_prefix(prm.mask_bits, (prm.H + 31) >> 5, s_mask, s_pre);
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // K4a's partials are complete and visible
+
+  float ss[MAXP];
+#pragma unroll
+  for (int m = 0; m < MAXP; ++m) ss[m] = 0.f;
+#pragma unroll 1
+  for (int k = 0; k < K4T_VEC; ++k) {
+    const int g = threadIdx.x + k * K4T_THREADS;
+    if (g >= nq) continue;
+    const int c = 4 * g;
+    const uint32_t bits = (prm.mask_bits[c >> 5] >> (c & 31)) & 0xFu;
+    // every rank's partial and residual for these 4 channels, in one round of loads
+    float4 z[MAXP];
+    uint2 rv[MAXP];
+    if (!prm.permuted) {
+#pragma unroll
+      for (int m = 0; m < MAXP; ++m) {
+        z[m] = make_float4(0.f, 0.f, 0.f, 0.f);
+        rv[m] = make_uint2(0u, 0u);
+        if (m < P) {
+          z[m] = __ldcg(reinterpret_cast<const float4*>(zrow + m * zstride + c));
+          rv[m] = *reinterpret_cast<const uint2*>(prm.R + m * rstride + trow + c);
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < MAXP; ++m) {
+        if (m < P && k4_split(prm, m, c / K4_BM)) {
+          const float4 w = __ldcg(reinterpret_cast<const float4*>(zrow + slot1 + m * zstride + c));
+          z[m].x += w.x; z[m].y += w.y; z[m].z += w.z; z[m].w += w.w;
+        }
+      }
+    } else {
+      int col[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) col[e] = perm_pos(c + e, prm.n_s, s_mask, s_pre);
+#pragma unroll
+      for (int m = 0; m < MAXP; ++m) {
+        float zz[4] = {0.f, 0.f, 0.f, 0.f};
+        rv[m] = make_uint2(0u, 0u);
+        if (m < P) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            zz[e] = __ldcg(zrow + m * zstride + col[e]);
+            if (k4_split(prm, m, col[e] / K4_BM)) zz[e] += __ldcg(zrow + slot1 + m * zstride + col[e]);
+          }
+          rv[m] = *reinterpret_cast<const uint2*>(prm.R + m * rstride + trow + c);
+        }
+        z[m] = make_float4(zz[0], zz[1], zz[2], zz[3]);
+      }
+    }
+    // the shared sum, once for every rank (ranks in order)
+    float S[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int m = 0; m < MAXP; ++m) {
+      if (m < P) {
+        S[0] += z[m].x; S[1] += z[m].y; S[2] += z[m].z; S[3] += z[m].w;
+      }
+    }
+    // every rank's h for these channels
+#pragma unroll
+    for (int m = 0; m < MAXP; ++m) {
+      if (m >= P) break;
+      const float own[4] = {z[m].x, z[m].y, z[m].z, z[m].w};
+      const uint32_t rw[2] = {rv[m].x, rv[m].y};
+      uint32_t o[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float z0 = ((bits >> (2 * e)) & 1u) ? S[2 * e] : prm.private_scale * own[2 * e];
+        const float z1 = ((bits >> (2 * e + 1)) & 1u) ? S[2 * e + 1] : prm.private_scale * own[2 * e + 1];
+        o[e] = pack_bf16x2(z0 + bf16lo(rw[e]), z1 + bf16hi(rw[e]));
+        const float lo = bf16lo(o[e]), hi = bf16hi(o[e]);
+        ss[m] = fmaf(lo, lo, ss[m]);
+        ss[m] = fmaf(hi, hi, ss[m]);
+      }
+      *reinterpret_cast<uint2*>(prm.Hout + m * rstride + trow + c) = make_uint2(o[0], o[1]);
+    }
+  }
+  warp_sum_many<MAXP>(ss, lane);
+  {
+    constexpr int kShift = (MAXP == 32) ? 0 : (MAXP == 16 ? 1 : 2);
+    const int idx = lane >> kShift;  // the rank whose warp total this lane holds
+    if ((lane & ((1 << kShift) - 1)) == 0 && idx < P) red[idx][warp] = ss[0];
+  }
+  __syncthreads();
+  if (threadIdx.x < P) {
+    float v = 0.f;
+    for (int w = 0; w < K4T_THREADS / 32; ++w) v += red[threadIdx.x][w];
+    s_rstd[threadIdx.x] = rsqrtf(v / static_cast<float>(prm.H) + prm.eps);
+  }
+  __syncthreads();
+  // out = h / rms * gamma: every rank's stored h of a group read back in one round
+#pragma unroll 1
+  for (int k = 0; k < K4T_VEC; ++k) {
+    const int g = threadIdx.x + k * K4T_THREADS;
+    if (g >= nq) continue;
+    const uint2 gv = *reinterpret_cast<const uint2*>(prm.gamma + 4 * g);
+    const uint32_t gw[2] = {gv.x, gv.y};
+    uint2 hv[MAXP];
+#pragma unroll
+    for (int m = 0; m < MAXP; ++m)
+      hv[m] = (m < P) ? *reinterpret_cast<const uint2*>(prm.Hout + m * rstride + trow + 4 * g) : make_uint2(0u, 0u);
+#pragma unroll
+    for (int m = 0; m < MAXP; ++m) {
+      if (m >= P) break;
+      const float rs = s_rstd[m];
+      const uint32_t w[2] = {hv[m].x, hv[m].y};
+      uint32_t o[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e)
+        o[e] = pack_bf16x2(bf16lo(w[e]) * rs * bf16lo(gw[e]), bf16hi(w[e]) * rs * bf16hi(gw[e]));
+      *reinterpret_cast<uint2*>(prm.Out + m * rstride + trow + 4 * g) = make_uint2(o[0], o[1]);
+    }
   }
 }
 

@@ -287,6 +287,26 @@ __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w &
 __device__ __forceinline__ float bf16lo_p(uint32_t w) { return __uint_as_float(__byte_perm(w, 0u, 0x1044)); }
 __device__ __forceinline__ float bf16hi_p(uint32_t w) { return __uint_as_float(__byte_perm(w, 0u, 0x3244)); }
 
+// Sums each of NV (a power of two, <= 32) per-lane values over the warp with NV - 1 + log2(32/NV)
+// shuffles instead of 5 NV: at each step a lane keeps one half of its values and hands the other
+// half to its partner, which adds them.  Afterwards lane L holds in v[0] the warp total of value
+// index L >> log2(32/NV) (lanes L and L ^ 1 ... agree).
+template <int NV>
+__device__ __forceinline__ void warp_sum_many(float (&v)[NV], int lane) {
+#pragma unroll
+  for (int c = NV, d = 16; c > 1; c >>= 1, d >>= 1) {
+    const bool up = (lane & d) != 0;
+#pragma unroll
+    for (int i = 0; i < c / 2; ++i) {
+      const float send = up ? v[i] : v[i + c / 2];
+      const float keep = up ? v[i + c / 2] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, d);
+    }
+  }
+#pragma unroll
+  for (int d = 16 / NV; d > 0; d >>= 1) v[0] += __shfl_xor_sync(0xFFFFFFFFu, v[0], d);
+}
+
 // ------------------------------------------------------------------------------------------
 // Clusters and CTA pairs (tcgen05 cta_group::2)
 // ------------------------------------------------------------------------------------------
