@@ -536,7 +536,7 @@ def run_tp(args):
     from partial_activation_sync_caat_b200 import build as B
     from partial_activation_sync_caat_b200 import caat as C
     from partial_activation_sync_caat_b200 import inputs as I
-    from partial_activation_sync_caat_b200.tp import TPRowParallel, exchanged_bytes
+    from partial_activation_sync_caat_b200.tp import TPRowParallel, TPRowParallelP2P, exchanged_bytes, peer_exchange_bytes
 
     world, rank, local = rank_env()
     torch.cuda.set_device(local)
@@ -570,13 +570,21 @@ def run_tp(args):
     d = I.make_rowpar_inputs(T, K, H, P, seed=0, device="cuda")
     X, W, R = d["X"][rank].contiguous(), d["W"][rank].contiguous(), d["R"][rank].contiguous()
     del d["X"], d["W"], d["R"]
-    layer = TPRowParallel(H, p)
-    zs, h = layer.buffers(T, "cuda")
     out = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
     ws = C.alloc_workspace(256, "cuda")
+    if args.tp_peer:
+        # the exchange over peer memory (CUDA IPC buffers, the library's push / reduce / finish)
+        layer = TPRowParallelP2P(H, p, T)
+        h = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
 
-    def step():
-        layer.forward(X, W, R, d["gamma"], out, zs=zs, h=h, workspace=ws)
+        def step():
+            layer.forward(X, W, R, d["gamma"], out, h=h, workspace=ws)
+    else:
+        layer = TPRowParallel(H, p)
+        zs, h = layer.buffers(T, "cuda")
+
+        def step():
+            layer.forward(X, W, R, d["gamma"], out, zs=zs, h=h, workspace=ws)
 
     for _ in range(args.warmup):
         step()
@@ -592,6 +600,8 @@ def run_tp(args):
     ms = max_over_ranks(a.elapsed_time(b)) / args.steps
     status = C.caat_get_device_status()
     dist.barrier()
+    if args.tp_peer:
+        layer.close()
     dist.destroy_process_group()
     if rank != 0:
         return
@@ -603,9 +613,13 @@ def run_tp(args):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": f"fc2-7b over {P} devices: T={T} H={H} K={K} (K/P={K // P} per rank) p={p}",
                    "parallelism": f"tp{P}"},
-        "exchange": {"collective": "NCCL all-reduce (sum) of the shared channels' fp32 partials",
-                     "bytes_per_rank": exchanged_bytes(T, H, p), "full_all_reduce_bytes": 4 * T * H},
-        "gpu_launches": 2 * args.steps, "device_status": status}))
+        "exchange": ({"collective": "none: partials pushed to their owners' buffers by the GEMM epilogue "
+                                    "(peer memory), owners' reduce writes every rank's gather buffer",
+                      "bytes_sent_per_rank": peer_exchange_bytes(T, H, p, P), "full_all_reduce_bytes": 4 * T * H}
+                     if args.tp_peer else
+                     {"collective": "NCCL all-reduce (sum) of the shared channels' fp32 partials",
+                      "bytes_per_rank": exchanged_bytes(T, H, p), "full_all_reduce_bytes": 4 * T * H}),
+        "gpu_launches": (3 if args.tp_peer else 2) * args.steps, "device_status": status}))
 
 
 def run_caat(args):
@@ -910,6 +924,8 @@ def main():
     ap.add_argument("--tp", action="store_true",
                     help="the layer over real devices: one tensor-parallel rank per GPU (P = --gpus), NCCL "
                          "all-reduce of the shared channels")
+    ap.add_argument("--tp-peer", action="store_true",
+                    help="with --tp: exchange over peer memory (library kernels) instead of NCCL")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-workloads", action="store_true",
                     help="skip the per-workload records of the other configurations (fc2-7b default run)")

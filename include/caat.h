@@ -371,6 +371,47 @@ CAAT_API caat_status caat_rowpar_tp_local(const caat_tp_args* args);
 CAAT_API caat_status caat_rowpar_tp_finish(const caat_tp_args* args);
 
 /*
+ * The same layer with the exchange done by the library over peer memory (NVLink), no
+ * collective library involved (App. A.2 Eq. 22; §3; §4: fp32 sum of the shared channels; App. D:
+ * only the n_s shared channels cross devices).  Owner q of the world ranks owns the shared
+ * columns [q w, (q + 1) w), w = n_s / world.  Per call, in this order on every rank:
+ *   1. caat_rowpar_tp_local_push: the local GEMM (as caat_rowpar_tp_local) whose epilogue
+ *      stores this rank's fp32 partial of every shared column straight into its owner's receive
+ *      buffer (recv[q][rank][t][c - q w]); the launch's last CTA then raises
+ *      flags[q][0 * world + rank] = epoch on every rank q.  args->zs is not used.
+ *   2. caat_rowpar_tp_reduce: waits (bounded) until flags[rank][0 * world + r] = epoch for every
+ *      r, sums the world partials of its columns in rank order (fp32), writes the sum into
+ *      gather[g][t][rank w + j] of every rank g, and raises flags[g][1 * world + rank] = epoch.
+ *   3. caat_rowpar_tp_finish_wait: waits until flags[rank][1 * world + q] = epoch for every q,
+ *      then finishes as caat_rowpar_tp_finish with zs = gather[rank].
+ * A rank's own entries are its local buffers; the others are the peers' buffers mapped into
+ * this process (CUDA IPC), all on GPUs with peer access.  The caller allocates, per rank:
+ * recv [world][T][w] fp32, gather [T][n_s] fp32, flags [2][world] uint32 zeroed once, and
+ * reuses them across calls with an epoch that grows by one per call (0 is never used).  The
+ * three calls of one rank go on one stream in order; then no buffer is overwritten while it is
+ * still read: a rank's next push follows its finish, which waited for every owner's reduce, and
+ * an owner's next reduce waits for every rank's next push.  A wait that runs out (a rank that
+ * never arrives) sets
+ * the device status word (caat_get_device_status: CAAT_ERR_TIMEOUT) and the kernel returns;
+ * after an error nothing is signalled, so the other ranks' waits run out too.
+ * Requirements: world = 1..8, rank < world, n_s = floor(H p) a multiple of 32 world, the
+ * caat_rowpar_tp_local requirements, all pointers 16-byte aligned.
+ */
+#define CAAT_TP_MAX_WORLD 8
+typedef struct caat_tp_peers {
+  int32_t world;
+  int32_t rank;
+  uint32_t epoch;
+  float* recv[CAAT_TP_MAX_WORLD];
+  float* gather[CAAT_TP_MAX_WORLD];
+  uint32_t* flags[CAAT_TP_MAX_WORLD];
+} caat_tp_peers;
+
+CAAT_API caat_status caat_rowpar_tp_local_push(const caat_tp_args* args, const caat_tp_peers* peers);
+CAAT_API caat_status caat_rowpar_tp_reduce(const caat_tp_args* args, const caat_tp_peers* peers);
+CAAT_API caat_status caat_rowpar_tp_finish_wait(const caat_tp_args* args, const caat_tp_peers* peers);
+
+/*
  * caat_permute_weights - reorders the output channels (rows) of W for a sync set: with
  * perm(i) = the i-th shared channel for i < n_s and the (i - n_s)-th private channel
  * otherwise (both ascending), W_out[m, i, :] = W[m, perm(i), :] for every rank m.  The

@@ -50,8 +50,10 @@ EXPORTS = [
     "caat_timing_destroy", "caat_timing_reset", "caat_timing_read", "caat_status_string",
     "caat_version", "caat_permute_weights", "caat_speedup_model", "caat_rowpar_backward",
     "caat_plan_create", "caat_plan_execute", "caat_plan_destroy", "caat_rowpar_tp_local",
-    "caat_rowpar_tp_finish",
+    "caat_rowpar_tp_finish", "caat_rowpar_tp_local_push", "caat_rowpar_tp_reduce", "caat_rowpar_tp_finish_wait",
 ]
+
+CAAT_TP_MAX_WORLD = 8
 
 
 class CaatError(RuntimeError):
@@ -92,6 +94,14 @@ class TpArgs(ctypes.Structure):
         ("timing", ctypes.c_void_p), ("T", ctypes.c_int64), ("K_r", ctypes.c_int64), ("H", ctypes.c_int64),
         ("p", ctypes.c_double), ("eps", ctypes.c_float), ("private_scale", ctypes.c_float),
         ("flags", ctypes.c_uint32),
+    ]
+
+
+class TpPeers(ctypes.Structure):
+    _fields_ = [
+        ("world", ctypes.c_int32), ("rank", ctypes.c_int32), ("epoch", ctypes.c_uint32),
+        ("recv", ctypes.c_void_p * CAAT_TP_MAX_WORLD), ("gather", ctypes.c_void_p * CAAT_TP_MAX_WORLD),
+        ("flags", ctypes.c_void_p * CAAT_TP_MAX_WORLD),
     ]
 
 
@@ -144,6 +154,9 @@ def lib() -> ctypes.CDLL:
     L.caat_rowpar_tp_local.argtypes = [ctypes.POINTER(TpArgs)]
     L.caat_rowpar_tp_local.restype = ctypes.c_int
     L.caat_rowpar_tp_finish.argtypes = [ctypes.POINTER(TpArgs)]
+    for name in ("caat_rowpar_tp_local_push", "caat_rowpar_tp_reduce", "caat_rowpar_tp_finish_wait"):
+        getattr(L, name).argtypes = [ctypes.POINTER(TpArgs), ctypes.POINTER(TpPeers)]
+        getattr(L, name).restype = ctypes.c_int
     L.caat_rowpar_tp_finish.restype = ctypes.c_int
     L.caat_rowpar_backward.restype = ctypes.c_int
     L.caat_rowpar_backward.argtypes = [ctypes.POINTER(BwdArgs)]
@@ -407,6 +420,67 @@ def caat_rowpar_tp_finish(zs, residual, h, gamma, p: float, out, *, eps: float =
     a.h = _bf16_dev(h, "h")
     a.out = _bf16_dev(out, "out")
     _check(lib().caat_rowpar_tp_finish(ctypes.byref(a)), "caat_rowpar_tp_finish")
+    return out
+
+
+def tp_peers(world: int, rank: int, epoch: int, recv, gather, flags) -> TpPeers:
+    """Descriptor of the peer-memory exchange for one rank and call: recv[q], gather[q], flags[q]
+    are rank q's buffers (CUDA tensors, or device addresses as ints, valid in this process):
+    recv [world, T, n_s / world] fp32, gather [T, n_s] fp32, flags [2, world] int32 zeroed once."""
+    world = int(world)
+    if not 1 <= world <= CAAT_TP_MAX_WORLD:
+        raise ValueError(f"world must be 1..{CAAT_TP_MAX_WORLD}")
+    pe = TpPeers()
+    pe.world, pe.rank, pe.epoch = world, int(rank), int(epoch)
+
+    def addr(x):
+        return int(x) if isinstance(x, int) else _ptr(x)
+    for q in range(world):
+        pe.recv[q] = addr(recv[q])
+        pe.gather[q] = addr(gather[q])
+        pe.flags[q] = addr(flags[q])
+    return pe
+
+
+def caat_rowpar_tp_local_push(X, W, residual, p: float, h, peers: TpPeers, *, workspace=None,
+                              private_scale: float = 1.0, stream=None, timing=None):
+    """Local step of the peer-memory exchange: as caat_rowpar_tp_local, with this rank's fp32
+    partials of the shared channels stored into their owners' receive buffers (peers.recv)."""
+    T, K_r = int(X.shape[0]), int(X.shape[1])
+    H = int(W.shape[0])
+    if workspace is None:
+        workspace = alloc_workspace(256, X.device)
+    a = _tp_args(T, K_r, H, p, 1e-5, private_scale, stream, timing)
+    a.X = _bf16_dev(X, "X")
+    a.W = _bf16_dev(W, "W")
+    a.residual = _bf16_dev(residual, "residual")
+    a.h = _bf16_dev(h, "h")
+    a.workspace = _ptr(workspace)
+    a.ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().caat_rowpar_tp_local_push(ctypes.byref(a), ctypes.byref(peers)), "caat_rowpar_tp_local_push")
+    return h
+
+
+def caat_rowpar_tp_reduce(T: int, H: int, p: float, peers: TpPeers, *, workspace, stream=None, timing=None):
+    """Owner step of the peer-memory exchange: sums this rank's slice of the shared channels over
+    the ranks and writes it into every rank's gather buffer.  workspace: >= 256 bytes, device."""
+    a = _tp_args(T, 0, H, p, 1e-5, 1.0, stream, timing)
+    a.workspace = _ptr(workspace)
+    a.ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().caat_rowpar_tp_reduce(ctypes.byref(a), ctypes.byref(peers)), "caat_rowpar_tp_reduce")
+
+
+def caat_rowpar_tp_finish_wait(residual, h, gamma, p: float, out, peers: TpPeers, *, eps: float = 1e-5, stream=None,
+                               timing=None):
+    """Finishing step of the peer-memory exchange: waits for every owner's slice, then as
+    caat_rowpar_tp_finish with zs = this rank's gather buffer."""
+    T, H = int(h.shape[0]), int(h.shape[1])
+    a = _tp_args(T, 0, H, p, eps, 1.0, stream, timing)
+    a.residual = _bf16_dev(residual, "residual")
+    a.gamma = _bf16_dev(gamma, "gamma")
+    a.h = _bf16_dev(h, "h")
+    a.out = _bf16_dev(out, "out")
+    _check(lib().caat_rowpar_tp_finish_wait(ctypes.byref(a), ctypes.byref(peers)), "caat_rowpar_tp_finish_wait")
     return out
 
 

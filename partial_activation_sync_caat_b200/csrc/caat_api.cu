@@ -672,6 +672,7 @@ caat_status launch_decode(const caat_rowpar_args* a, const std::vector<uint8_t>&
 struct TpSplit {
   float* zs;
   int64_t n_s;
+  const caat_tp_peers* peers;  // non-null: push the partials to their owners (peer memory)
 };
 
 caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>& mask, const DeviceInfo* dev,
@@ -786,8 +787,20 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
   prm.sdone = merge ? reinterpret_cast<unsigned int*>(wsb + wl.sdone) : nullptr;
   const size_t zero_bytes = merge ? wl.sdone + wl.sdone_bytes : (consumer ? wl.consumer_total : wl.zeroed);
 
-  prm.zs_mode = split ? 1 : 0;
+  prm.zs_mode = split ? (split->peers ? 2 : 1) : 0;
   prm.zs_ns = split ? static_cast<int>(split->n_s) : 0;
+  if (split && split->peers) {
+    const caat_tp_peers* pe = split->peers;
+    for (int q = 0; q < pe->world; ++q) {
+      prm.tp_recv[q] = pe->recv[q];
+      prm.tp_flags[q] = pe->flags[q];
+    }
+    prm.tp_done = counter + 8;  // zeroed with the counters at launch
+    prm.tp_world = pe->world;
+    prm.tp_rank = pe->rank;
+    prm.tp_w = static_cast<int>(split->n_s / pe->world);
+    prm.tp_epoch = pe->epoch;
+  }
   if (split && (!pair || fused || permuted || gemm_only)) return CAAT_ERR_UNSUPPORTED;
   CUtensorMap tmX, tmW, tmR, tmH, tmZ;
   // K-major operands: boxes of 64 K x (128 rows); MN-major ones: 64 MN x 64 K rows, two per half
@@ -804,7 +817,7 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
   if (s != CAAT_OK) return s;
   // the split output's fp32 shared-channel partials: 32-row x 32-column boxes
   tmZ = tmH;
-  if (split && split->n_s > 0) {
+  if (split && split->n_s > 0 && !split->peers) {
     s = make_map_3d_f32(&tmZ, split->zs, static_cast<uint64_t>(split->n_s), T, 1, 32, 32);
     if (s != CAAT_OK) return s;
   }
@@ -1479,42 +1492,166 @@ caat_status caat_rowpar_tp_local(const caat_tp_args* a) {
   r.flags = CAAT_FLAG_FORCE_GEMM_PATH;
   static thread_local std::vector<uint8_t> zero_mask;
   zero_mask.assign(static_cast<size_t>(a->H), 0);
-  const TpSplit split{a->zs, ns};
+  const TpSplit split{a->zs, ns, nullptr};
   return launch_rowpar(&r, zero_mask, dev, static_cast<unsigned int*>(a->workspace), nullptr, &split);
 }
 
-caat_status caat_rowpar_tp_finish(const caat_tp_args* a) {
-  int64_t ns = 0;
-  caat_status s = validate_tp(a, &ns, false);
-  if (s != CAAT_OK) return s;
-  if (a->T == 0) return CAAT_OK;
-  if (!a->residual || !a->gamma || !a->h || !a->out || (ns > 0 && !a->zs)) return CAAT_ERR_INVALID_ARG;
+}  // extern "C"
+
+namespace {
+
+// The peer-memory exchange's descriptor: world, rank, epoch and the per-rank buffers.
+caat_status validate_peers(const caat_tp_peers* pe, int64_t ns) {
+  if (!pe) return CAAT_ERR_INVALID_ARG;
+  if (pe->world < 1 || pe->world > CAAT_TP_MAX_WORLD || pe->rank < 0 || pe->rank >= pe->world || pe->epoch == 0)
+    return CAAT_ERR_INVALID_ARG;
+  if (ns % (32 * int64_t(pe->world)) != 0) return CAAT_ERR_UNSUPPORTED;
+  for (int q = 0; q < pe->world; ++q) {
+    if (!pe->recv[q] || !pe->gather[q] || !pe->flags[q]) return CAAT_ERR_INVALID_ARG;
+    if (!aligned16(pe->recv[q]) || !aligned16(pe->gather[q]) || (reinterpret_cast<uintptr_t>(pe->flags[q]) & 3u))
+      return CAAT_ERR_UNSUPPORTED;
+  }
+  return CAAT_OK;
+}
+
+// The finishing kernel over zs, optionally after waiting for `wait_n` flags to reach `epoch`.
+caat_status tp_finish_launch(const caat_tp_args* a, int64_t ns, const float* z, const unsigned int* wait_flags,
+                             int wait_n, uint32_t epoch) {
+  if (!a->residual || !a->gamma || !a->h || !a->out || (ns > 0 && !z)) return CAAT_ERR_INVALID_ARG;
   if (!aligned16(a->residual) || !aligned16(a->gamma) || !aligned16(a->h) || !aligned16(a->out) ||
-      (ns > 0 && !aligned16(a->zs)))
+      (ns > 0 && !aligned16(z)))
     return CAAT_ERR_UNSUPPORTED;
   DeviceInfo* dev = nullptr;
-  s = device_info(&dev);
+  caat_status s = device_info(&dev);
   if (s != CAAT_OK) return s;
   Recorder rec;
   rec.begin(a->timing, a->stream);
   const int64_t warps = caat::KT_FIN_THREADS / 32;
   const int64_t nb = std::max<int64_t>(1, std::min<int64_t>((a->T + warps - 1) / warps, int64_t(dev->sm_count) * 4));
-  const float* z = a->zs;
   const __nv_bfloat16* R = reinterpret_cast<const __nv_bfloat16*>(a->residual);
   __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(a->h);
   __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(a->out);
   const __nv_bfloat16* g = reinterpret_cast<const __nv_bfloat16*>(a->gamma);
   const int Hi = static_cast<int>(a->H), nsi = static_cast<int>(ns);
   cudaStream_t st = a->stream;
+  const uint64_t tmo = timeout_ns();
   if (a->H <= 1024)
-    caat::tp_finish_kernel<4><<<nb, caat::KT_FIN_THREADS, 0, st>>>(z, R, h, o, g, a->T, Hi, nsi, a->eps);
+    caat::tp_finish_kernel<4><<<nb, caat::KT_FIN_THREADS, 0, st>>>(z, R, h, o, g, a->T, Hi, nsi, a->eps, wait_flags,
+                                                                   wait_n, epoch, tmo);
   else if (a->H <= 2048)
-    caat::tp_finish_kernel<8><<<nb, caat::KT_FIN_THREADS, 0, st>>>(z, R, h, o, g, a->T, Hi, nsi, a->eps);
+    caat::tp_finish_kernel<8><<<nb, caat::KT_FIN_THREADS, 0, st>>>(z, R, h, o, g, a->T, Hi, nsi, a->eps, wait_flags,
+                                                                   wait_n, epoch, tmo);
   else
-    caat::tp_finish_kernel<16><<<nb, caat::KT_FIN_THREADS, 0, st>>>(z, R, h, o, g, a->T, Hi, nsi, a->eps);
+    caat::tp_finish_kernel<16><<<nb, caat::KT_FIN_THREADS, 0, st>>>(z, R, h, o, g, a->T, Hi, nsi, a->eps,
+                                                                    wait_flags, wait_n, epoch, tmo);
   if (cudaGetLastError() != cudaSuccess) return CAAT_ERR_CUDA;
   rec.after_kernel(st);
   return CAAT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+caat_status caat_rowpar_tp_finish(const caat_tp_args* a) {
+  int64_t ns = 0;
+  caat_status s = validate_tp(a, &ns, false);
+  if (s != CAAT_OK) return s;
+  if (a->T == 0) return CAAT_OK;
+  return tp_finish_launch(a, ns, a->zs, nullptr, 0, 0);
+}
+
+caat_status caat_rowpar_tp_local_push(const caat_tp_args* a, const caat_tp_peers* pe) {
+  int64_t ns = 0;
+  caat_status s = validate_tp(a, &ns, true);
+  if (s != CAAT_OK) return s;
+  s = validate_peers(pe, ns);
+  if (s != CAAT_OK) return s;
+  if (a->T == 0) return CAAT_OK;
+  if (!a->X || !a->W || !a->residual || !a->h) return CAAT_ERR_INVALID_ARG;
+  if (!aligned16(a->X) || !aligned16(a->W) || !aligned16(a->residual) || !aligned16(a->h))
+    return CAAT_ERR_UNSUPPORTED;
+  if (!a->workspace || a->ws_bytes < kCounterBytes || (reinterpret_cast<uintptr_t>(a->workspace) & 255u))
+    return CAAT_ERR_WORKSPACE;
+  DeviceInfo* dev = nullptr;
+  s = device_info(&dev);
+  if (s != CAAT_OK) return s;
+  if (dev->max_pairs <= 0) return CAAT_ERR_UNSUPPORTED;
+  caat_rowpar_args r;
+  std::memset(&r, 0, sizeof(r));
+  r.X = a->X;
+  r.W = a->W;
+  r.residual = a->residual;
+  r.gamma = a->residual;  // unused by the split mode
+  r.out = a->h;
+  r.h_out = a->h;
+  r.workspace = a->workspace;
+  r.ws_bytes = kCounterBytes;
+  r.stream = a->stream;
+  r.timing = a->timing;
+  r.T = a->T;
+  r.K = a->K_r;
+  r.H = a->H;
+  r.p = 0.0;
+  r.eps = a->eps;
+  r.private_scale = a->private_scale;
+  r.P = 1;
+  r.flags = CAAT_FLAG_FORCE_GEMM_PATH;
+  static thread_local std::vector<uint8_t> zero_mask;
+  zero_mask.assign(static_cast<size_t>(a->H), 0);
+  // no shared channels: nothing crosses devices, and the other two steps do not wait
+  const TpSplit split{nullptr, ns, ns > 0 ? pe : nullptr};
+  return launch_rowpar(&r, zero_mask, dev, static_cast<unsigned int*>(a->workspace), nullptr, &split);
+}
+
+caat_status caat_rowpar_tp_reduce(const caat_tp_args* a, const caat_tp_peers* pe) {
+  int64_t ns = 0;
+  caat_status s = validate_tp(a, &ns, false);
+  if (s != CAAT_OK) return s;
+  s = validate_peers(pe, ns);
+  if (s != CAAT_OK) return s;
+  if (a->T == 0 || ns == 0) return CAAT_OK;
+  if (!a->workspace || a->ws_bytes < kCounterBytes || (reinterpret_cast<uintptr_t>(a->workspace) & 255u))
+    return CAAT_ERR_WORKSPACE;
+  DeviceInfo* dev = nullptr;
+  s = device_info(&dev);
+  if (s != CAAT_OK) return s;
+  caat::TpReduceParams rp{};
+  rp.recv = pe->recv[pe->rank];
+  for (int q = 0; q < pe->world; ++q) {
+    rp.gather[q] = pe->gather[q];
+    rp.flags[q] = pe->flags[q];
+  }
+  rp.done = static_cast<unsigned int*>(a->workspace);
+  rp.T = a->T;
+  rp.w = static_cast<int>(ns / pe->world);
+  rp.n_s = static_cast<int>(ns);
+  rp.world = pe->world;
+  rp.rank = pe->rank;
+  rp.epoch = pe->epoch;
+  rp.timeout_ns = timeout_ns();
+  const int64_t n4 = a->T * (rp.w / 4);
+  const int64_t nb =
+      std::max<int64_t>(1, std::min<int64_t>((n4 + caat::KT_RED_THREADS - 1) / caat::KT_RED_THREADS,
+                                             int64_t(dev->sm_count) * 4));
+  Recorder rec;
+  rec.begin(a->timing, a->stream);
+  if (cudaMemsetAsync(a->workspace, 0, 4, a->stream) != cudaSuccess) return CAAT_ERR_CUDA;
+  caat::tp_reduce_kernel<<<static_cast<unsigned>(nb), caat::KT_RED_THREADS, 0, a->stream>>>(rp);
+  if (cudaGetLastError() != cudaSuccess) return CAAT_ERR_CUDA;
+  rec.after_kernel(a->stream);
+  return CAAT_OK;
+}
+
+caat_status caat_rowpar_tp_finish_wait(const caat_tp_args* a, const caat_tp_peers* pe) {
+  int64_t ns = 0;
+  caat_status s = validate_tp(a, &ns, false);
+  if (s != CAAT_OK) return s;
+  s = validate_peers(pe, ns);
+  if (s != CAAT_OK) return s;
+  if (a->T == 0) return CAAT_OK;
+  if (ns == 0) return tp_finish_launch(a, 0, nullptr, nullptr, 0, 0);
+  return tp_finish_launch(a, ns, pe->gather[pe->rank], pe->flags[pe->rank] + pe->world, pe->world, pe->epoch);
 }
 
 }  // extern "C"

@@ -18,6 +18,7 @@
 #pragma once
 
 #include "ptx.cuh"
+#include "tp.cuh"
 
 namespace caat {
 
@@ -60,8 +61,17 @@ struct RowparParams {
   int merge_mixed;             // 1: mixed blocks use the TMA epilogue (see k1_epilogue_tma)
   int no_residual;             // 1: store Z (no residual add) -- channel-permuted path, see rownorm.cuh
   int zs_mode;                 // 1: split output of one rank of a multi-device layer (tp.cuh):
-                               // channels c < zs_ns go to Zs as the fp32 partial, the others to h
+                               // channels c < zs_ns go to Zs as the fp32 partial, the others to h;
+                               // 2: the same, the partials pushed to their owners' receive buffers
   int zs_ns;                   // shared channels (zs_mode)
+  // zs_mode 2 (peer-memory exchange, tp.cuh): owner q's receive buffer [world][T][tp_w] as this
+  // process maps it, every rank's flag array [2][world], the launch's done-CTA counter (zero at
+  // launch), and this call's epoch
+  float* tp_recv[TP_MAX_WORLD];
+  unsigned int* tp_flags[TP_MAX_WORLD];
+  unsigned int* tp_done;
+  int tp_world, tp_rank, tp_w;
+  uint32_t tp_epoch;
   int T, H, Kp, P;             // T: token rows of the tensors (the row stride of rank blocks)
   int t_begin, t_end;          // token rows this launch processes: [t_begin, t_end)
   int n_mblk;                  // row blocks of the kernel's tile height over [t_begin, t_end)
@@ -598,7 +608,24 @@ __device__ __forceinline__ bool k1_epilogue_split(uint32_t trow, const RowparPar
     tmem_ld_32x32b_x32(trow + 64 * c, *reinterpret_cast<uint32_t(*)[32]>(v));
     tmem_ld_32x32b_x32(trow + 64 * c + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
     tmem_wait_ld();
-    if (has_shared) {
+    if (has_shared && prm.zs_mode == 2) {
+      // each 32-column half goes to the owner of its columns: 8 16-byte stores per row
+      const int row = row0 + lane;
+      for (int hf = 0; hf < 2; ++hf) {
+        const int cc = col + 32 * hf;
+        if (cc >= prm.zs_ns) break;  // warp-uniform
+        const int q = cc / prm.tp_w;
+        const int j = cc - q * prm.tp_w;
+        if (row < prm.t_end) {
+          float4* dst = reinterpret_cast<float4*>(
+              prm.tp_recv[q] + (static_cast<size_t>(prm.tp_rank) * prm.T + row) * prm.tp_w + j);
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            dst[k] = make_float4(__uint_as_float(v[32 * hf + 4 * k]), __uint_as_float(v[32 * hf + 4 * k + 1]),
+                                 __uint_as_float(v[32 * hf + 4 * k + 2]), __uint_as_float(v[32 * hf + 4 * k + 3]));
+        }
+      }
+    } else if (has_shared) {
       // fp32 boxes of 32 rows x 32 columns (128-byte rows, 128-byte swizzle) in buffer 1
       for (int hf = 0; hf < 2; ++hf) {
         if (col + 32 * hf >= prm.zs_ns) break;  // warp-uniform

@@ -297,6 +297,7 @@ __global__ void __launch_bounds__(K1Threads<kFused>::value, 1)
       ++local;
     }
     if (pend_m128 >= 0) k1_publish_counts(prm, pend_m128, pend_rank);
+    if (prm.zs_mode == 2) fence_sc_sys();  // this warp's pushes to other GPUs, before the signal
   }
 
   tc_fence_before();
@@ -304,6 +305,9 @@ __global__ void __launch_bounds__(K1Threads<kFused>::value, 1)
   cluster_sync();  // neither CTA leaves while the other may still touch its shared memory
   tc_fence_after();
   if (warp == 1) tmem_dealloc_pair(tmem_base, K1_TMEM_COLS);
+  // peer-memory exchange: the launch's last CTA tells every owner that this rank's partials are in
+  if (prm.zs_mode == 2 && threadIdx.x == 0)
+    tp_signal_done(prm.tp_done, gridDim.x, prm.tp_flags, prm.tp_world, 0, prm.tp_rank, prm.tp_epoch);
 }
 
 }  // namespace caat

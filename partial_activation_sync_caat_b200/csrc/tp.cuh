@@ -1,6 +1,22 @@
-// tp.cuh - the finishing kernel of the layer split over real devices, one tensor-parallel rank
-// per GPU ("Tensor-Parallelism with Partially Synchronized Activations", App. A.2 Eq. 22; §3:
-// only the first floor(h p) channels are exchanged; §4 Eq. 9: residual add, then the norm).
+// tp.cuh - the layer split over real devices, one tensor-parallel rank per GPU ("Tensor-
+// Parallelism with Partially Synchronized Activations", App. A.2 Eq. 22; §3: only the first
+// floor(h p) channels are exchanged; §4: their sum accumulated in fp32; §4 Eq. 9: residual add,
+// then the norm).
+//
+// Two ways to exchange the shared channels' partials:
+//   * through the caller's collective (an all-reduce of zs [T, n_s]), then tp_finish_kernel;
+//   * over peer memory, with no library collective: the local GEMM's epilogue pushes each
+//     rank's fp32 partial of the shared channels straight into the receive buffer of the rank
+//     that owns those columns (owner q owns columns [q w, (q + 1) w), w = n_s / world), the
+//     owner sums the world partials of its slice in rank order and writes the sum into every
+//     rank's gather buffer (tp_reduce_kernel), and each rank finishes from its gather buffer
+//     (tp_finish_kernel after a wait).  The exchange is a reduce-scatter fused into the GEMM
+//     epilogue plus an all-gather: (world - 1) / world of T n_s fp32 values sent per rank in
+//     each half, as a ring all-reduce of the same buffer.  Completion is signalled with
+//     per-call epochs in each rank's flag array [2][world] (phase 0: partials pushed by rank
+//     r; phase 1: slice reduced by owner q): the last CTA of a launch to finish raises them
+//     (release, system scope) after every CTA's stores are fenced at system scope; waiters
+//     poll them (acquire, system scope) with a bounded wait.
 //
 // The local step (the CTA-pair GEMM kernel in its split-output mode, rowpar_common.cuh) leaves
 // this rank's fp32 partial of the shared channels in zs [T, n_s] and the finished private
@@ -16,12 +32,102 @@
 namespace caat {
 
 constexpr int KT_FIN_THREADS = 256;
+constexpr int TP_MAX_WORLD = 8;
+constexpr int KT_RED_THREADS = 256;
 
+// Bounded wait until flags[0..n) all reach `epoch`.  Returns false (and raises the device status
+// word as a timeout tagged `site`) if they do not within timeout_ns, or if another waiter
+// already raised it.
+__device__ __forceinline__ bool tp_wait_flags(const unsigned int* flags, int n, uint32_t epoch, uint64_t timeout_ns,
+                                              int site) {
+  const uint64_t t0 = globaltimer_ns();
+  for (int i = 0; i < n; ++i) {
+    for (uint32_t k = 1;; ++k) {
+      if (static_cast<int32_t>(ld_acquire_sys_u32(flags + i) - epoch) >= 0) break;
+      if ((k & 63u) == 0u) {
+        if (status_poll() != 0) return false;
+        if (globaltimer_ns() - t0 > timeout_ns) {
+          status_raise(4, site);
+          return false;
+        }
+      }
+    }
+  }
+  return true;
+}
+
+// One thread per CTA, after the CTA's stores (to this and other GPUs) are complete and fenced:
+// count the CTA as done; the last of `total` raises flags[q][phase * world + rank] = epoch on
+// every rank q.  Nothing is raised once the device status word is set (an error: the waiters
+// time out instead of reading incomplete data).
+__device__ __forceinline__ void tp_signal_done(unsigned int* done, uint32_t total, unsigned int* const* flags,
+                                               int world, int phase, int rank, uint32_t epoch) {
+  fence_sc_sys();
+  const uint32_t old = atom_add_acq_rel_gpu_u32(done, 1u);
+  if (old != total - 1u || status_poll() != 0) return;
+  fence_sc_sys();
+  for (int q = 0; q < world; ++q) st_release_sys_u32(flags[q] + phase * world + rank, epoch);
+}
+
+// The owner's step of the peer-memory exchange.
+struct TpReduceParams {
+  const float* recv;                   // this rank's receive buffer [world][T][w]
+  float* gather[TP_MAX_WORLD];         // every rank's gather buffer [T][n_s]
+  unsigned int* flags[TP_MAX_WORLD];   // every rank's flag array [2][world]
+  unsigned int* done;                  // CTAs of this launch done, zero at launch
+  int64_t T;
+  int w, n_s, world, rank;
+  uint32_t epoch;
+  uint64_t timeout_ns;
+};
+
+// Waits until every rank has pushed its partials of this rank's slice, sums the world partials
+// per element in rank order (fp32), and stores the sum into columns [rank w, (rank + 1) w) of
+// every rank's gather buffer; then signals phase 1.  16-byte accesses (w % 4 == 0).
+__global__ void __launch_bounds__(KT_RED_THREADS)
+    tp_reduce_kernel(const __grid_constant__ TpReduceParams prm) {
+  __shared__ int s_ok;
+  if (threadIdx.x == 0)
+    s_ok = tp_wait_flags(prm.flags[prm.rank], prm.world, prm.epoch, prm.timeout_ns, 81) ? 1 : 0;
+  __syncthreads();
+  if (!s_ok) return;
+  const int w4 = prm.w >> 2;
+  const int64_t n4 = prm.T * w4;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * KT_RED_THREADS;
+  const int64_t slab = prm.T * prm.w;  // between the partials of two ranks
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * KT_RED_THREADS + threadIdx.x; i < n4; i += stride) {
+    const int64_t t = i / w4;
+    const int j = static_cast<int>(i - t * w4) * 4;
+    const float* src = prm.recv + t * prm.w + j;
+    float4 s = __ldcg(reinterpret_cast<const float4*>(src));
+    for (int r = 1; r < prm.world; ++r) {
+      const float4 z = __ldcg(reinterpret_cast<const float4*>(src + r * slab));
+      s.x += z.x;
+      s.y += z.y;
+      s.z += z.z;
+      s.w += z.w;
+    }
+    const int64_t off = t * prm.n_s + static_cast<int64_t>(prm.rank) * prm.w + j;
+    for (int g = 0; g < prm.world; ++g) *reinterpret_cast<float4*>(prm.gather[g] + off) = s;
+  }
+  fence_sc_sys();
+  __syncthreads();
+  if (threadIdx.x == 0) tp_signal_done(prm.done, gridDim.x, prm.flags, prm.world, 1, prm.rank, prm.epoch);
+}
+
+// wait_flags (optional): the peer-memory exchange's phase-1 flags of this rank [world]; the
+// kernel first waits (bounded) until they all reach `epoch`.
 template <int VPL>
 __global__ void __launch_bounds__(KT_FIN_THREADS, 2)
-    tp_finish_kernel(const float* __restrict__ zs, const __nv_bfloat16* __restrict__ R, __nv_bfloat16* h,
-                     __nv_bfloat16* out, const __nv_bfloat16* __restrict__ gamma, int64_t T, int H, int n_s,
-                     float eps) {
+    tp_finish_kernel(const float* zs, const __nv_bfloat16* __restrict__ R, __nv_bfloat16* h, __nv_bfloat16* out,
+                     const __nv_bfloat16* __restrict__ gamma, int64_t T, int H, int n_s, float eps,
+                     const unsigned int* wait_flags, int wait_n, uint32_t epoch, uint64_t timeout_ns) {
+  if (wait_flags != nullptr) {
+    __shared__ int s_ok;
+    if (threadIdx.x == 0) s_ok = tp_wait_flags(wait_flags, wait_n, epoch, timeout_ns, 82) ? 1 : 0;
+    __syncthreads();
+    if (!s_ok) return;
+  }
   const int lane = threadIdx.x & 31;
   const int64_t warp_global = (static_cast<int64_t>(blockIdx.x) * KT_FIN_THREADS + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * KT_FIN_THREADS) >> 5;
@@ -41,7 +147,7 @@ __global__ void __launch_bounds__(KT_FIN_THREADS, 2)
         if (8 * idx + 8 <= n_s) {
           // shared: the ranks' summed partial plus this rank's residual, rounded once
           const uint4 r = __ldg(rp + idx);
-          const float4 z0 = __ldg(zp + 2 * idx), z1 = __ldg(zp + 2 * idx + 1);
+          const float4 z0 = __ldcg(zp + 2 * idx), z1 = __ldcg(zp + 2 * idx + 1);
           x[u].x = pack_bf16x2(z0.x + bf16lo(r.x), z0.y + bf16hi(r.x));
           x[u].y = pack_bf16x2(z0.z + bf16lo(r.y), z0.w + bf16hi(r.y));
           x[u].z = pack_bf16x2(z1.x + bf16lo(r.z), z1.y + bf16hi(r.z));
