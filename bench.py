@@ -90,12 +90,13 @@ def load_peaks():
 
 
 def kernel_source_hash() -> str:
-    """sha256 over the sources of the forward GEMM and norm kernels: their headers and the
-    forward launch code of caat_api.cu (from launch_rowpar up to validate_rowpar)."""
+    """sha256 over the sources of the forward GEMM and norm kernels: their headers (with tp.cuh,
+    which the GEMM header includes) and the forward launch code of caat_api.cu (from
+    launch_rowpar up to validate_rowpar)."""
     import hashlib
     h = hashlib.sha256()
     d = os.path.join(ROOT, "partial_activation_sync_caat_b200", "csrc")
-    for f in ("ptx.cuh", "rowpar_common.cuh", "rowpar_gemm.cuh", "rowpar_gemm2.cuh", "rownorm.cuh"):
+    for f in ("ptx.cuh", "tp.cuh", "rowpar_common.cuh", "rowpar_gemm.cuh", "rowpar_gemm2.cuh", "rownorm.cuh"):
         h.update(f.encode())
         with open(os.path.join(d, f), "rb") as fh:
             h.update(fh.read())

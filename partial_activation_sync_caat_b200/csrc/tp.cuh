@@ -56,8 +56,8 @@ __device__ __forceinline__ bool tp_wait_flags(const unsigned int* flags, int n, 
   return true;
 }
 
-// One thread per CTA, after the CTA's stores (to this and other GPUs) are complete and fenced:
-// count the CTA as done; the last of `total` raises flags[q][phase * world + rank] = epoch on
+// One thread per CTA, after a CTA barrier that orders the CTA's stores (to this and other GPUs)
+// before it: fence at system scope and count the CTA as done; the last of `total` raises flags[q][phase * world + rank] = epoch on
 // every rank q.  Nothing is raised once the device status word is set (an error: the waiters
 // time out instead of reading incomplete data).
 __device__ __forceinline__ void tp_signal_done(unsigned int* done, uint32_t total, unsigned int* const* flags,
@@ -110,8 +110,7 @@ __global__ void __launch_bounds__(KT_RED_THREADS)
     const int64_t off = t * prm.n_s + static_cast<int64_t>(prm.rank) * prm.w + j;
     for (int g = 0; g < prm.world; ++g) *reinterpret_cast<float4*>(prm.gather[g] + off) = s;
   }
-  fence_sc_sys();
-  __syncthreads();
+  __syncthreads();  // the CTA's stores precede thread 0's system-scope fence in tp_signal_done
   if (threadIdx.x == 0) tp_signal_done(prm.done, gridDim.x, prm.flags, prm.world, 1, prm.rank, prm.epoch);
 }
 
