@@ -203,11 +203,13 @@ int decode_token_min_t() {
   return v;
 }
 // Whether the decode streaming kernel splits its items evenly, cutting units (tuning;
-// CAAT_DECODE_STREAMK).
-bool decode_stream_k_setting() {
-  static bool v = [] {
+// CAAT_DECODE_STREAMK: 1 always, 0 never; unset: with the per-row reduce (few tokens) only.
+// Measured on one box: T = 8 30.8 us with the split against 32.1 us with whole units; T = 64
+// 38.6 us against 37.1 us, the per-token reduce then paying for the split units' second slots).
+int decode_stream_k_setting() {
+  static int v = [] {
     const char* e = std::getenv("CAAT_DECODE_STREAMK");
-    return (e && *e) ? (*e == '1') : true;
+    return (e && *e) ? (*e == '1' ? 1 : 0) : -1;
   }();
   return v;
 }
@@ -617,7 +619,7 @@ caat_status launch_decode(const caat_rowpar_args* a, const std::vector<uint8_t>&
   prm.kblk = gp.kblk;
   // units cut between two streaming CTAs (their first and last k-block have different owners)
   if (units > int64_t(caat::K4_MAXP) * 64) return CAAT_ERR_UNSUPPORTED;
-  gp.stream_k = decode_stream_k_setting() ? 1 : 0;
+  gp.stream_k = decode_stream_k_setting() >= 0 ? decode_stream_k_setting() : (T < decode_token_min_t() ? 1 : 0);
   for (int64_t u = 0; gp.stream_k && u < units; ++u) {
     const int64_t first = u * gp.kblk;
     if (caat::k4_cta_of(first, items, grid) != caat::k4_cta_of(first + gp.kblk - 1, items, grid))
