@@ -119,12 +119,15 @@ class CudaPeerMemory:
         self.mapped.append(ptr)
         return int(ptr)
 
-    def close(self):
+    def close_mapped(self):
         for ptr in self.mapped:
             self.rt.cudaIpcCloseMemHandle(ptr)
+        self.mapped = []
+
+    def free_own(self):
         for ptr in self.own:
             self.rt.cudaFree(ptr)
-        self.own, self.mapped = [], []
+        self.own = []
 
 
 class LibraryPeerOps:
@@ -200,7 +203,14 @@ class TPRowParallelP2P:
         self.epoch = 0
 
     def close(self):
-        self.memory.close()
+        """Unmaps the other ranks' buffers, waits until every rank has done so, then frees this
+        rank's own (an exporter frees only after every importer has closed its mapping).  Call it
+        on every rank, after the last forward has completed."""
+        import torch.distributed as dist
+        self.memory.close_mapped()
+        if self.world > 1:
+            dist.barrier(group=self.group)
+        self.memory.free_own()
 
     def forward(self, X_r, W_r, R_r, gamma, out, *, h=None, workspace=None):
         """X_r [T, K_r], W_r [H, K_r], R_r [T, H], gamma [H] (bf16) -> out [T, H]; returns

@@ -46,11 +46,16 @@ class ShmMemory:
         self.mapped.append(shm)
         return shm
 
-    def close(self):
-        for shm in self.mapped + self.own:
+    def close_mapped(self):
+        for shm in self.mapped:
             shm.close()
+        self.mapped = []
+
+    def free_own(self):
         for shm in self.own:
+            shm.close()
             shm.unlink()
+        self.own = []
 
 
 def _wait(flags, phase, world, epoch, timeout=60.0):
@@ -135,11 +140,10 @@ def _worker(rank, world, port, p, out_q):
             ok, max_abs, _ = O.within_tolerance(out.float(), ref["out"][rank])
             h_err = float(np.max(np.abs(O._f64(h.float()) - ref["h"][rank])))
             res.append((ok, max_abs, h_err))
-        dist.barrier()  # every rank is done reading the others' buffers
         out_q[rank] = (res, layer.epoch, layer.n_s, peer_exchange_bytes(24, H, p, world))
+        layer.close()  # unmap, barrier, free
+        layer = None
     finally:
-        if layer is not None:
-            layer.close()
         dist.destroy_process_group()
 
 
