@@ -213,6 +213,16 @@ int decode_stream_k_setting() {
   }();
   return v;
 }
+// Streaming CTAs per SM on the decode path, each with half the ring (tuning; CAAT_DECODE_CTAS:
+// 1 or 2).  Two measured faster at T = 1 / 8 / 64 on one box: 30.9 / 30.8 / 37.0 us with one,
+// 28.8 / 28.9 / 34.7 us with two (more copies in flight against DRAM at once).
+int decode_ctas_per_sm_setting() {
+  static int v = [] {
+    const char* e = std::getenv("CAAT_DECODE_CTAS");
+    return (e && *e == '1') ? 1 : 2;
+  }();
+  return v;
+}
 bool order_env_set() {
   static bool v = [] {
     const char* e = std::getenv("CAAT_ORDER");
@@ -599,11 +609,14 @@ caat_status launch_decode(const caat_rowpar_args* a, const std::vector<uint8_t>&
   const int64_t items = units * gp.kblk;
   if (items > INT32_MAX / 2) return CAAT_ERR_UNSUPPORTED;
   gp.n_items = static_cast<int>(items);
-  gp.stages = caat::k4_stages(gp.Tpad);
+  const int per_sm = decode_ctas_per_sm_setting();
+  gp.ring_bytes = per_sm == 2 ? caat::K4_RING_BYTES_HALF : caat::K4_RING_BYTES;
+  gp.stages = caat::k4_stages(gp.Tpad, gp.ring_bytes);
   gp.timeout_ns = timeout_ns();
   // No more CTAs than units: every CTA then streams at least one unit's worth of items, so a
   // unit is cut at most once (two partials).
-  const int grid = static_cast<int>(std::min<int64_t>(dev->sm_count, units));
+  const int grid = static_cast<int>(std::min<int64_t>(int64_t(per_sm) * dev->sm_count, units));
+  const int k4_smem = 1024 + gp.ring_bytes + 512;
 
   static thread_local caat::DecodeParams prm;
   std::memset(&prm, 0, sizeof(prm));
@@ -642,7 +655,7 @@ caat_status launch_decode(const caat_rowpar_args* a, const std::vector<uint8_t>&
   Recorder own;
   Recorder& rec = outer ? *outer : own;
   if (!outer) rec.begin(a->timing, st);
-  caat::decode_partials_kernel<<<grid, caat::K4_THREADS, caat::K4_SMEM_BYTES, st>>>(tmW, tmX, gp);
+  caat::decode_partials_kernel<<<grid, caat::K4_THREADS, k4_smem, st>>>(tmW, tmX, gp);
   if (cudaGetLastError() != cudaSuccess) return CAAT_ERR_CUDA;
   rec.after_kernel(st);
   // The reduce kernel is a programmatic dependent of the partials kernel: its launch overlaps

@@ -51,10 +51,13 @@ constexpr int K4T_VEC = K4B_MAX_H / (4 * K4T_THREADS);
 // The reduce kernels' channel mask covers only the decode path's rows (a small parameter block).
 constexpr int K4_MASK_WORDS = K4B_MAX_H / 32;
 
+// A ring for two streaming CTAs per SM (shared memory of both, with their reservations, fits).
+constexpr int K4_RING_BYTES_HALF = 112640;
+
 // Ring depth for a padded token count: stages of 16 KiB of W + Tpad x 128 B of X.
-__host__ __device__ constexpr int k4_stages(int Tpad) {
-  return (K4_RING_BYTES / (K4_A_BYTES + Tpad * 128)) < K4_MAX_STAGES ? (K4_RING_BYTES / (K4_A_BYTES + Tpad * 128))
-                                                                       : K4_MAX_STAGES;
+__host__ __device__ constexpr int k4_stages(int Tpad, int ring_bytes = K4_RING_BYTES) {
+  return (ring_bytes / (K4_A_BYTES + Tpad * 128)) < K4_MAX_STAGES ? (ring_bytes / (K4_A_BYTES + Tpad * 128))
+                                                                    : K4_MAX_STAGES;
 }
 
 // The streaming kernel's parameters (no channel mask: a small parameter block).
@@ -67,6 +70,7 @@ struct DecodeGemmParams {
   int n_items;                // P * n_cb * kblk
   int stages;                 // ring depth
   int stream_k;               // 1: split the items evenly (units may be cut); 0: whole units
+  int ring_bytes;             // shared memory of the ring (the barriers follow it)
   uint64_t timeout_ns;
 };
 
@@ -100,7 +104,7 @@ __global__ void __launch_bounds__(K4_THREADS, 1)
   const uint32_t b_bytes = static_cast<uint32_t>(prm.Tpad) * K4_BK * 2;
   uint8_t* sA = smem;                               // [S] W tiles (16 KiB, 1024-aligned)
   uint8_t* sB = smem + S * K4_A_BYTES;              // [S] X tiles (Tpad x 128 B, 1024-aligned)
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + K4_RING_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + prm.ring_bytes);
   uint64_t* full = bars;                            // [K4_MAX_STAGES]
   uint64_t* empty = full + K4_MAX_STAGES;           // [K4_MAX_STAGES]
   uint64_t* tfull = empty + K4_MAX_STAGES;
