@@ -502,6 +502,10 @@ def sub_workloads(args, peaks, peak_src):
     names = ["fc2-1b", "mlp-7b", "attn-out-7b", "decode-1", "decode-8", "decode-64", "tiny"]
     for name in names:
         case = Case(name, seed=2000)
+        # one second idle first: each workload starts from a comparable power state instead of
+        # the sustained power cap the previous workload's clock soak left behind
+        torch.cuda.synchronize()
+        time.sleep(1.0)
         steps = 20
         ms_local, per_kernel, clocks = time_case(case, steps, 5, sample_clocks=True, soak_ms=150.0)
         ms = ms_local / steps
