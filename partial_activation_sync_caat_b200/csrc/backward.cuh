@@ -39,6 +39,7 @@ struct BwdParams {
   int P, H;
   int64_t T;
   float eps, private_scale;
+  int zk_regs;                 // 1 (P <= 8): bf16(s dh) kept in registers between passes 2 and 3
   uint32_t mask_bits[K1_MASK_WORDS];
 };
 
@@ -273,39 +274,81 @@ __global__ void __launch_bounds__(KB_THREADS, 1) rownorm_bwd_smem_kernel(const _
     float S[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) S[e] = 0.f;
-    if (active) {
-      // pass 2: dh per rank -> dR, the shared sum S, dgamma; the h slot gets bf16(s dh)
-      for (int m = 0; m < P; ++m) {
-        float hf[8], df[8], dh[8], zp[8];
-        unpack8(sh[m * nvec + v], hf);
-        unpack8(sd[m * nvec + v], df);
-        const float r = s_r[m], kk = s_k[m];
+    if (MAXP <= 8 && prm.zk_regs) {
+      // pass 2: dh per rank -> dR, the shared sum S, dgamma; bf16(s dh) kept in registers, so
+      // both of this token's slots are free before pass 3 and the next token's loads start now
+      uint4 zk[MAXP];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          dh[e] = r * df[e] * gam[e] - hf[e] * kk;
-          S[e] += dh[e];
-          dg[e] = fmaf(df[e], hf[e] * r, dg[e]);
-          zp[e] = prm.private_scale * dh[e];
+      for (int m = 0; m < MAXP; ++m) {
+        zk[m] = make_uint4(0u, 0u, 0u, 0u);
+        if (active && m < P) {
+          float hf[8], df[8], dh[8], zp[8];
+          unpack8(sh[m * nvec + v], hf);
+          unpack8(sd[m * nvec + v], df);
+          const float r = s_r[m], kk = s_k[m];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            dh[e] = r * df[e] * gam[e] - hf[e] * kk;
+            S[e] += dh[e];
+            dg[e] = fmaf(df[e], hf[e] * r, dg[e]);
+            zp[e] = prm.private_scale * dh[e];
+          }
+          if (prm.dR != nullptr) *reinterpret_cast<uint4*>(prm.dR + m * rstride + toff) = pack8(dh);
+          zk[m] = pack8(zp);
         }
-        if (prm.dR != nullptr) *reinterpret_cast<uint4*>(prm.dR + m * rstride + toff) = pack8(dh);
-        sh[m * nvec + v] = pack8(zp);
       }
-    }
-    if (tn < prm.T) stage(sd, prm.dout, tn);  // dout of this token is no longer needed
-    asm volatile("cp.async.commit_group;" ::: "memory");
-    if (active) {
+      if (tn < prm.T) {  // this thread's slots of this token are no longer read
+        stage(sd, prm.dout, tn);
+        stage(sh, prm.h, tn);
+      }
+      asm volatile("cp.async.commit_group;" ::: "memory");
       // pass 3: dZt per rank (shared channels: S, private: s dh)
-      for (int m = 0; m < P; ++m) {
-        float z[8];
-        unpack8(sh[m * nvec + v], z);
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-          if ((bits >> e) & 1u) z[e] = S[e];
-        *reinterpret_cast<uint4*>(prm.dZt + m * rstride + toff) = pack8(z);
+      for (int m = 0; m < MAXP; ++m) {
+        if (active && m < P) {
+          float z[8];
+          unpack8(zk[m], z);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            if ((bits >> e) & 1u) z[e] = S[e];
+          *reinterpret_cast<uint4*>(prm.dZt + m * rstride + toff) = pack8(z);
+        }
       }
+    } else {
+      if (active) {
+        // pass 2: dh per rank -> dR, the shared sum S, dgamma; the h slot gets bf16(s dh)
+        for (int m = 0; m < P; ++m) {
+          float hf[8], df[8], dh[8], zp[8];
+          unpack8(sh[m * nvec + v], hf);
+          unpack8(sd[m * nvec + v], df);
+          const float r = s_r[m], kk = s_k[m];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            dh[e] = r * df[e] * gam[e] - hf[e] * kk;
+            S[e] += dh[e];
+            dg[e] = fmaf(df[e], hf[e] * r, dg[e]);
+            zp[e] = prm.private_scale * dh[e];
+          }
+          if (prm.dR != nullptr) *reinterpret_cast<uint4*>(prm.dR + m * rstride + toff) = pack8(dh);
+          sh[m * nvec + v] = pack8(zp);
+        }
+      }
+      if (tn < prm.T) stage(sd, prm.dout, tn);  // dout of this token is no longer needed
+      asm volatile("cp.async.commit_group;" ::: "memory");
+      if (active) {
+        // pass 3: dZt per rank (shared channels: S, private: s dh)
+        for (int m = 0; m < P; ++m) {
+          float z[8];
+          unpack8(sh[m * nvec + v], z);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            if ((bits >> e) & 1u) z[e] = S[e];
+          *reinterpret_cast<uint4*>(prm.dZt + m * rstride + toff) = pack8(z);
+        }
+      }
+      if (tn < prm.T) stage(sh, prm.h, tn);  // the h slots were read back by this thread only
+      asm volatile("cp.async.commit_group;" ::: "memory");
     }
-    if (tn < prm.T) stage(sh, prm.h, tn);  // the h slots were read back by this thread only
-    asm volatile("cp.async.commit_group;" ::: "memory");
     __syncthreads();  // red / s_r / s_k are reused next token
   }
   asm volatile("cp.async.wait_group 0;" ::: "memory");

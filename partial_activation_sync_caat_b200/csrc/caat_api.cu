@@ -223,6 +223,15 @@ int decode_ctas_per_sm_setting() {
   }();
   return v;
 }
+// Norm backward: bf16(s dh) kept in registers between its passes 2 and 3, so that the next
+// token's loads start a pass earlier (tuning; CAAT_BWD_ZK: 1 on, 0 off).
+bool bwd_zk_regs_setting() {
+  static bool v = [] {
+    const char* e = std::getenv("CAAT_BWD_ZK");
+    return (e && *e) ? (*e == '1') : true;
+  }();
+  return v;
+}
 bool order_env_set() {
   static bool v = [] {
     const char* e = std::getenv("CAAT_ORDER");
@@ -1187,6 +1196,7 @@ caat_status caat_rowpar_backward(const caat_rowpar_bwd_args* a) {
   bp.T = T;
   bp.eps = a->eps;
   bp.private_scale = a->private_scale;
+  bp.zk_regs = bwd_zk_regs_setting() ? 1 : 0;
   for (int64_t c = 0; c < H; ++c)
     if (mask[c]) bp.mask_bits[c >> 5] |= 1u << (c & 31);
   const size_t kb_smem = caat::bwd_smem_bytes(P, static_cast<int>(H));
