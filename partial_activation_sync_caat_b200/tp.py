@@ -107,6 +107,7 @@ class CudaPeerMemory:
     def alloc(self, nbytes: int):
         ptr = self._ok(self.rt.cudaMalloc(int(nbytes)), "cudaMalloc")
         self._ok(self.rt.cudaMemset(ptr, 0, int(nbytes)), "cudaMemset")
+        self._ok(self.rt.cudaDeviceSynchronize(), "cudaDeviceSynchronize")  # zeroed before any peer maps it
         self.own.append(ptr)
         handle = self._ok(self.rt.cudaIpcGetMemHandle(ptr), "cudaIpcGetMemHandle")
         return bytes(handle.reserved), int(ptr)
