@@ -21,6 +21,7 @@ from __future__ import annotations
 
 import argparse
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -131,6 +132,20 @@ def alg_bytes_of(T, K, H, P, mlp=False):
     if mlp:   # K is the FFN size F: X [P,T,H], A [P,2F/P,H], Y [P,T,F/P] out and in, W2 [P,H,F/P], R, out
         return 2.0 * (P * T * H + 2 * K * H + 2 * T * K + K * H + 2 * P * T * H + H)
     return 2.0 * (T * K + H * K + 2 * P * T * H + H)
+
+
+def shared_sums_once(case) -> bool:
+    """Whether the forward stores the shared channels' cross-rank sums once (fp32) and its norm
+    kernel (rownorm_zs_kernel) adds each rank's residual: the library takes that path for a
+    contiguous sync set S = the first n_s channels with n_s % 8 == 0, H <= 4096, the CTA-pair
+    GEMM (T > 128), the separate norm after the GEMM and the full workspace (CAAT_ZS_SUM=0
+    turns it off).  Used to name the norm kernel and count its bytes."""
+    from partial_activation_sync_caat_b200 import caat as C
+    n_s = int(math.floor(case.H * case.p))
+    other = (C.CAAT_FLAG_SINGLE_CTA | C.CAAT_FLAG_FUSED_NORM | C.CAAT_FLAG_OVERLAP_NORM |
+             C.CAAT_FLAG_NORM_BESIDE_GEMM | C.CAAT_FLAG_W_PERMUTED | C.CAAT_FLAG_FORCE_DECODE_PATH)
+    return (os.environ.get("CAAT_ZS_SUM", "1") != "0" and not case.bwd and not case.rand and
+            not (case.flags & other) and 0 < n_s and n_s % 8 == 0 and case.H <= 4096 and case.T > 128)
 
 
 def alg_flops_of(T, K, H, mlp=False):
@@ -738,7 +753,10 @@ def run_caat(args):
     k1_ms = kernel_ms[kg] if len(kernel_ms) > kg else float("nan")
     k2_ms = kernel_ms[kg + 1] if len(kernel_ms) > kg + 1 else None
     k1_tflops = fc2_flops / k1_ms / 1e9
-    norm_bytes = 2.0 * P * T * H * 2
+    zs_once = shared_sums_once(case)
+    n_s = int(math.floor(H * p))
+    # the norm reads h (or, for the shared channels, the fp32 sums and the residual) and writes out
+    norm_bytes = 2.0 * P * T * H * 2 + (4.0 * T * n_s if zs_once else 0.0)
     alg_bytes = alg_bytes_of(T, K, H, P)
     if overlapped:
         t_g, t_n = recorded_traffic(args.workload, "gemm"), recorded_traffic(args.workload, "norm_overlapped")
@@ -750,7 +768,8 @@ def run_caat(args):
     else:
         traffic = recorded_traffic(args.workload, "gemm") if default_case else None
         kname = ("rowpar_gemm_pair_kernel (tcgen05 cta_group::2 GEMM + partial channel-reduce "
-                 "+ residual" + (")" if k2_ms else " + fused RMSNorm)"))
+                 + ("; residual on the private channels, the shared channels' sums stored once in fp32)"
+                    if zs_once else "+ residual" + (")" if k2_ms else " + fused RMSNorm)")))
         algo = "2*T*K*H flops per launch"
     result = {
         "metric": "TFLOP/s & tokens/s of partially-synced row-parallel FC2 (7B shape), % bf16 peak",
@@ -805,12 +824,17 @@ def run_caat(args):
         result["decode"] = {"us_per_call": round(ms_step * 1e3, 2), "hbm_gbs": round(alg_bytes / ms_step / 1e6, 1),
                             "frac_of_measured_hbm": round(alg_bytes / ms_step / 1e6 / peaks["hbm_gbs"], 3)}
     if k2_ms and not overlapped:
-        result["norm_kernel"] = {"kernel": "rownorm_reg_kernel" if H <= 4096 else "rownorm_kernel", "bound": "hbm",
+        result["norm_kernel"] = {"kernel": ("rownorm_zs_kernel" if zs_once else
+                                            "rownorm_reg_kernel" if H <= 4096 else "rownorm_kernel"),
+                                 "bound": "hbm",
                                  "achieved": round(norm_bytes / k2_ms / 1e6, 1),
                                  "traffic": recorded_traffic(args.workload, "norm") if default_case else None,
                                  "peak": peaks["hbm_gbs"], "unit": "GB/s",
                                  "frac": round(norm_bytes / k2_ms / 1e6 / peaks["hbm_gbs"], 3),
-                                 "launch_ms": round(k2_ms, 4), "algorithmic": "2*P*T*H*2 bytes (read h, write out)"}
+                                 "launch_ms": round(k2_ms, 4),
+                                 "algorithmic": ("4*T*n_s + 2*P*T*H*2 bytes (read the shared sums once, the residual "
+                                                 "of the shared and h of the private channels; write out)"
+                                                 if zs_once else "2*P*T*H*2 bytes (read h, write out)")}
     if args.flags:
         result["config"]["flags"] = hex(args.flags)
     if not mlp:

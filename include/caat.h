@@ -132,10 +132,13 @@ typedef enum caat_status {
  *             every path: the fused norm's row-block counters and per-row partial sums of
  *             squares (about 64 ceil(H/256) P T bytes), the completion flags that give
  *             column blocks mixing shared and private channels the TMA epilogue (T/8
- *             ceil(H/256) bytes), the decode path's fp32 partials (4 P T H bytes, T <= 64).
- *             The separate-norm GEMM path runs with 256 bytes (mixed column blocks then take
- *             the register epilogue); a smaller workspace than a call needs gives
- *             CAAT_ERR_WORKSPACE.
+ *             ceil(H/256) bytes), the decode path's fp32 partials (4 P T H bytes, T <= 64),
+ *             and the cross-rank sums of the shared channels stored once for all ranks
+ *             (4 T n_s bytes; H <= 4096, S the first n_s channels, n_s % 8 == 0; each rank's
+ *             residual is then added by the norm kernel).  The separate-norm GEMM path runs
+ *             with 256 bytes (mixed column blocks then take the register epilogue and every
+ *             shared tile stores h for all P ranks); a smaller workspace than a call needs
+ *             gives CAAT_ERR_WORKSPACE.
  * eps = 1e-5 and private_scale = 1 (use caat_rowpar_forward_ex for other values).
  * Returns CAAT_OK once the work is queued.
  */
@@ -198,11 +201,12 @@ CAAT_API caat_status caat_rowpar_forward_host(const caat_rowpar_args* args);
  * process exits.  It holds whatever workspace the path the call takes uses, when that fits:
  * the GEMM kernel's work-unit counter (always), the row-block counters and job list of the
  * norm that runs beside the GEMM (8 bytes per 128 tokens per rank), the completion flags of
- * column blocks that mix shared and private channels (T/8 ceil(H/256) bytes), the fused
- * norm's counters and partials, and the decode path's fp32 partials (4 P T H bytes).
+ * column blocks that mix shared and private channels (T/8 ceil(H/256) bytes), the shared
+ * channels' cross-rank sums (4 T n_s bytes), the fused norm's counters and partials, and the
+ * decode path's fp32 partials (4 P T H bytes).
  *   - A fused norm (CAAT_FLAG_FUSED_NORM) whose partials do not fit runs as the separate norm;
  *     a decode-sized call whose partials do not fit takes the GEMM path; the optional parts
- *     (job list, flags) are simply not used when they do not fit.  A call that still needs
+ *     (job list, flags, shared sums) are simply not used when they do not fit.  A call that still needs
  *     more than the array (a forced decode path that does not fit) returns
  *     CAAT_ERR_WORKSPACE and queues nothing.
  *   - Calls no cudaMalloc, cudaFree or other allocating routine.

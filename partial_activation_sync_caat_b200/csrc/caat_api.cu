@@ -232,6 +232,16 @@ bool bwd_zk_regs_setting() {
   }();
   return v;
 }
+// The shared units store their cross-rank sums once (fp32) and the norm kernel adds each rank's
+// residual, instead of every shared tile storing h for all P ranks (tuning; CAAT_ZS_SUM: 1 on,
+// 0 off).
+bool zs_sum_setting() {
+  static bool v = [] {
+    const char* e = std::getenv("CAAT_ZS_SUM");
+    return (e && *e) ? (*e == '1') : true;
+  }();
+  return v;
+}
 bool order_env_set() {
   static bool v = [] {
     const char* e = std::getenv("CAAT_ORDER");
@@ -417,6 +427,11 @@ RowparWs rowpar_ws_layout(int64_t T, int64_t H, int P, bool fused) {
   return L;
 }
 
+// The GEMM path's shared-sum mode: after the counters, Zs [T, n_s] fp32 (the cross-rank sums of
+// the shared channels, stored once by the shared units, read by the norm kernel for every rank).
+constexpr size_t kZsOffset = kCounterBytes;
+size_t zs_workspace(int64_t T, int64_t n_s) { return kZsOffset + align256(size_t(T) * size_t(n_s) * 4); }
+
 // Decode path (T <= CAAT_DECODE_MAX_T, P <= 16): the weight-streaming kernel splits the stream
 // of (unit, k-block) items evenly over its CTAs; a unit cut in two leaves two fp32 partials.
 bool decode_eligible(int64_t T, int P, int64_t H) {
@@ -441,6 +456,7 @@ size_t rowpar_workspace(int64_t T, int64_t K, int64_t H, int P) {
   (void)K;
   size_t n = std::max(rowpar_ws_layout(T, H, P, true).total, rowpar_ws_layout(T, H, P, false).total);
   if (decode_eligible(T, P, H)) n = std::max(n, decode_workspace(T, H, P));
+  if (H <= 4096) n = std::max(n, zs_workspace(T, H));  // the shared sums, up to every channel
   return n;
 }
 
@@ -759,6 +775,14 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
                         (a->flags & CAAT_FLAG_NORM_BESIDE_GEMM) && !(a->flags & CAAT_FLAG_OVERLAP_NORM) &&
                         a->ws_bytes >= wl.consumer_total;
   prm.publish = fused ? 1 : (consumer ? 2 : 0);
+  // Shared-sum mode: S the first n_s channels, rows of at most 4096 channels, room for Zs, h
+  // not stored over the residual (a mixed block's private tiles write whole h boxes, whose
+  // shared columns the norm kernel rewrites from Zs and the residual).
+  bool contiguous = true;
+  for (int64_t c = 0; c < H && contiguous; ++c) contiguous = (mask[c] != 0) == (c < n_s);
+  const bool zs3 = zs_sum_setting() && pair_possible && !split && !fused && !permuted && !gemm_only && !consumer &&
+                   !(a->flags & CAAT_FLAG_OVERLAP_NORM) && contiguous && n_s > 0 && n_s % 8 == 0 && H <= 4096 &&
+                   a->ws_bytes >= zs_workspace(T, n_s) && static_cast<const void*>(hdst) != a->residual;
   if (consumer) {
     prm.rb_count = reinterpret_cast<unsigned int*>(wsb + wl.rb_count);
     if (!(a->flags & (CAAT_FLAG_ORDER_ROWBLOCK | CAAT_FLAG_ORDER_GROUPED))) {
@@ -806,13 +830,13 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
   // their shared tiles, when the workspace holds the flags.
   bool any_mixed = false;
   for (int nb = 0; nb < nblk; ++nb) any_mixed |= prm.ncls[nb] == 2;
-  const bool merge = pair && !fused && any_mixed && a->ws_bytes >= wl.total;
+  const bool merge = pair && !fused && any_mixed && a->ws_bytes >= wl.total && !zs3;
   prm.merge_mixed = merge ? 1 : 0;
   prm.sdone = merge ? reinterpret_cast<unsigned int*>(wsb + wl.sdone) : nullptr;
   const size_t zero_bytes = merge ? wl.sdone + wl.sdone_bytes : (consumer ? wl.consumer_total : wl.zeroed);
 
-  prm.zs_mode = split ? (split->peers ? 2 : 1) : 0;
-  prm.zs_ns = split ? static_cast<int>(split->n_s) : 0;
+  prm.zs_mode = split ? (split->peers ? 2 : 1) : (zs3 ? 3 : 0);
+  prm.zs_ns = split ? static_cast<int>(split->n_s) : (zs3 ? n_s : 0);
   if (split && split->peers) {
     const caat_tp_peers* pe = split->peers;
     for (int q = 0; q < pe->world; ++q) {
@@ -841,6 +865,11 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
   if (s != CAAT_OK) return s;
   // the split output's fp32 shared-channel partials: 32-row x 32-column boxes
   tmZ = tmH;
+  float* zs_buf = zs3 ? reinterpret_cast<float*>(wsb + kZsOffset) : nullptr;
+  if (zs3) {
+    s = make_map_3d_f32(&tmZ, zs_buf, static_cast<uint64_t>(n_s), T, 1, 32, 32);
+    if (s != CAAT_OK) return s;
+  }
   if (split && split->n_s > 0 && !split->peers) {
     s = make_map_3d_f32(&tmZ, split->zs, static_cast<uint64_t>(split->n_s), T, 1, 32, 32);
     if (s != CAAT_OK) return s;
@@ -927,6 +956,21 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
     }
     const int64_t warps_per_block = caat::K2_THREADS / 32;
     const int64_t blocks = std::min<int64_t>((rows + warps_per_block - 1) / warps_per_block, max_blocks);
+    if (zs3) {
+      // every rank's row: shared channels from Zs (the token's cross-rank sum) plus its residual,
+      // private channels from h; then the norm (one warp per row, the row in registers)
+      // one CTA per token (its ranks on the CTA's warps), the token's sums staged once
+      const int64_t fb = std::min<int64_t>(T, int64_t(dev->sm_count) * 2);
+      const __nv_bfloat16* rr = reinterpret_cast<const __nv_bfloat16*>(a->residual);
+      const int Hi = static_cast<int>(H);
+      if (H <= 1024)
+        caat::rownorm_zs_kernel<4><<<fb, caat::KZ_THREADS, 0, ns>>>(zs_buf, rr, hdst, o, g, T, P, Hi, n_s, a->eps);
+      else if (H <= 2048)
+        caat::rownorm_zs_kernel<8><<<fb, caat::KZ_THREADS, 0, ns>>>(zs_buf, rr, hdst, o, g, T, P, Hi, n_s, a->eps);
+      else
+        caat::rownorm_zs_kernel<16><<<fb, caat::KZ_THREADS, 0, ns>>>(zs_buf, rr, hdst, o, g, T, P, Hi, n_s, a->eps);
+      return cudaGetLastError() == cudaSuccess ? CAAT_OK : CAAT_ERR_CUDA;
+    }
     if (H <= 4096) {
       // row held in registers: VPL 128-bit vectors per lane
       int64_t rb = std::min<int64_t>((rows + warps_per_block - 1) / warps_per_block, int64_t(dev->sm_count) * 2);
@@ -1562,13 +1606,13 @@ caat_status tp_finish_launch(const caat_tp_args* a, int64_t ns, const float* z, 
   const uint64_t tmo = timeout_ns();
   if (a->H <= 1024)
     caat::tp_finish_kernel<4><<<nb, caat::KT_FIN_THREADS, 0, st>>>(z, R, h, o, g, a->T, Hi, nsi, a->eps, wait_flags,
-                                                                   wait_n, epoch, tmo);
+                                                                   wait_n, epoch, tmo, a->T, 1);
   else if (a->H <= 2048)
     caat::tp_finish_kernel<8><<<nb, caat::KT_FIN_THREADS, 0, st>>>(z, R, h, o, g, a->T, Hi, nsi, a->eps, wait_flags,
-                                                                   wait_n, epoch, tmo);
+                                                                   wait_n, epoch, tmo, a->T, 1);
   else
     caat::tp_finish_kernel<16><<<nb, caat::KT_FIN_THREADS, 0, st>>>(z, R, h, o, g, a->T, Hi, nsi, a->eps,
-                                                                    wait_flags, wait_n, epoch, tmo);
+                                                                    wait_flags, wait_n, epoch, tmo, a->T, 1);
   if (cudaGetLastError() != cudaSuccess) return CAAT_ERR_CUDA;
   rec.after_kernel(st);
   return CAAT_OK;

@@ -62,7 +62,10 @@ struct RowparParams {
   int no_residual;             // 1: store Z (no residual add) -- channel-permuted path, see rownorm.cuh
   int zs_mode;                 // 1: split output of one rank of a multi-device layer (tp.cuh):
                                // channels c < zs_ns go to Zs as the fp32 partial, the others to h;
-                               // 2: the same, the partials pushed to their owners' receive buffers
+                               // 2: the same, the partials pushed to their owners' receive buffers;
+                               // 3: one device, P ranks: a shared unit stores its accumulator (the
+                               // cross-rank sum) as fp32 to Zs [T, zs_ns] once, the norm kernel
+                               // adds the residual; private units store h as usual
   int zs_ns;                   // shared channels (zs_mode)
   // zs_mode 2 (peer-memory exchange, tp.cuh): owner q's receive buffer [world][T][tp_w] as this
   // process maps it, every rank's flag array [2][world], the launch's done-CTA counter (zero at
@@ -578,6 +581,43 @@ __device__ __forceinline__ bool k1_epilogue_tma(uint32_t trow, const RowparParam
   }
   __syncwarp();
   return true;
+}
+
+// Shared unit in zs_mode 3: the accumulator of the columns below zs_ns (the cross-rank sum of
+// Eq. 22, exact fp32) is stored to Zs [T, zs_ns] by 32 x 32 fp32 boxes (128-byte rows,
+// 128-byte swizzle, clipped at zs_ns and T by the tensor map) through the warp's second box.
+// Nothing else: the residual add and the store of h for every rank move to the norm kernel,
+// which reads Zs once per rank row.
+__device__ __forceinline__ void k1_epilogue_zs(uint32_t trow, const RowparParams& prm, const void* tmZ, int row0,
+                                               int n0, uint8_t* bufs, int lane, uint64_t pol) {
+  const int nch = min(4, (prm.H - n0 + 63) / 64);
+  for (int c = 0; c < nch; ++c) {
+    const int col = n0 + 64 * c;
+    if (col >= prm.zs_ns) break;  // warp-uniform
+    uint32_t v[64];
+    __syncwarp();
+    tmem_ld_32x32b_x32(trow + 64 * c, *reinterpret_cast<uint32_t(*)[32]>(v));
+    tmem_ld_32x32b_x32(trow + 64 * c + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+    tmem_wait_ld();
+    for (int hf = 0; hf < 2; ++hf) {
+      if (col + 32 * hf >= prm.zs_ns) break;  // warp-uniform
+      if (lane == 0) bulk_wait_group_read0();
+      __syncwarp();
+      uint8_t* rowp = bufs + K1_EPI_BOX_BYTES + lane * 128;
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        *reinterpret_cast<uint4*>(rowp + ((j ^ (lane & 7)) << 4)) =
+            make_uint4(v[32 * hf + 4 * j], v[32 * hf + 4 * j + 1], v[32 * hf + 4 * j + 2], v[32 * hf + 4 * j + 3]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_3d(tmZ, bufs + K1_EPI_BOX_BYTES, col + 32 * hf, row0, 0, pol);
+        bulk_commit_group();
+      }
+    }
+  }
+  if (lane == 0) bulk_wait_group_read0();
+  __syncwarp();
 }
 
 // Epilogue of one tile of the split-output mode (one tensor-parallel rank per device, every

@@ -99,7 +99,7 @@ __global__ void __launch_bounds__(K1Threads<kFused>::value, 1)
     tma_prefetch_desc(&tmW);
     tma_prefetch_desc(&tmR);
     tma_prefetch_desc(&tmH);
-    if (prm.zs_mode) tma_prefetch_desc(&tmZ);
+    if (prm.zs_mode == 1 || prm.zs_mode == 3) tma_prefetch_desc(&tmZ);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_holder, K1_TMEM_COLS);
@@ -263,7 +263,15 @@ __global__ void __launch_bounds__(K1Threads<kFused>::value, 1)
       const int n0 = un.n * K2P_BN;
       const bool mixed = prm.ncls[un.n] == 2;
       const bool merge = mixed && !kFused && prm.merge_mixed;
-      if (prm.zs_mode) {
+      if (prm.zs_mode == 3) {
+        const int row0 = prm.t_begin + un.m * (2 * K2P_BM) + static_cast<int>(cta) * K2P_BM + q * 32;
+        if (un.rank < 0) {
+          k1_epilogue_zs(trow, prm, &tmZ, row0, n0, my_bufs, lane, pol_h);
+        } else if (!k1_epilogue_tma<kEpiBuf>(trow, prm, &tmR, &tmH, row0, n0, un.rank, un.slot, my_bufs, my_rbar,
+                                             rphase, lane, pol_r, pol_h, false)) {
+          break;  // private: full h boxes (a mixed block's shared columns are rewritten from Zs)
+        }
+      } else if (prm.zs_mode) {
         const int row0 = prm.t_begin + un.m * (2 * K2P_BM) + static_cast<int>(cta) * K2P_BM + q * 32;
         if (!k1_epilogue_split(trow, prm, &tmR, &tmH, &tmZ, row0, n0, un.rank, my_bufs, my_rbar, rphase, lane,
                                pol_r, pol_h))

@@ -115,12 +115,16 @@ __global__ void __launch_bounds__(KT_RED_THREADS)
 }
 
 // wait_flags (optional): the peer-memory exchange's phase-1 flags of this rank [world]; the
-// kernel first waits (bounded) until they all reach `epoch`.
+// kernel first waits (bounded) until they all reach `epoch`.  The T rows are `ranks` x `tokens`
+// ([ranks, tokens, H]; ranks = 1 for one device's rank), and the row of token tk of any rank takes
+// its shared sums from zs row tk: the single-device layer's P ranks add their own residual to the
+// same cross-rank sum.
 template <int VPL>
 __global__ void __launch_bounds__(KT_FIN_THREADS, 2)
-    tp_finish_kernel(const float* zs, const __nv_bfloat16* __restrict__ R, __nv_bfloat16* h, __nv_bfloat16* out,
+    tp_finish_kernel(const float* __restrict__ zs, const __nv_bfloat16* __restrict__ R, __nv_bfloat16* h, __nv_bfloat16* out,
                      const __nv_bfloat16* __restrict__ gamma, int64_t T, int H, int n_s, float eps,
-                     const unsigned int* wait_flags, int wait_n, uint32_t epoch, uint64_t timeout_ns) {
+                     const unsigned int* wait_flags, int wait_n, uint32_t epoch, uint64_t timeout_ns,
+                     int64_t tokens, int ranks) {
   if (wait_flags != nullptr) {
     __shared__ int s_ok;
     if (threadIdx.x == 0) s_ok = tp_wait_flags(wait_flags, wait_n, epoch, timeout_ns, 82) ? 1 : 0;
@@ -133,10 +137,14 @@ __global__ void __launch_bounds__(KT_FIN_THREADS, 2)
   const int nvec = H >> 3;
   const float inv_h = 1.0f / static_cast<float>(H);
   const uint4* g4 = reinterpret_cast<const uint4*>(gamma);
-  for (int64_t t = warp_global; t < T; t += nwarps) {
+  for (int64_t i = warp_global; i < T; i += nwarps) {
+    // row i: token tk = i / ranks of rank m = i % ranks, so the ranks of a token are neighbouring
+    // warps and read its shared sums (zs row tk) while they are in cache
+    const int64_t tk = i / ranks;
+    const int64_t t = (i - tk * ranks) * tokens + tk;  // the row in [ranks, tokens, H]
     uint4* hp = reinterpret_cast<uint4*>(h + t * H);
     const uint4* rp = reinterpret_cast<const uint4*>(R + t * H);
-    const float4* zp = reinterpret_cast<const float4*>(zs + t * n_s);
+    const float4* zp = reinterpret_cast<const float4*>(zs + tk * n_s);
     uint4 x[VPL];
 #pragma unroll
     for (int u = 0; u < VPL; ++u) {
@@ -151,10 +159,17 @@ __global__ void __launch_bounds__(KT_FIN_THREADS, 2)
           x[u].y = pack_bf16x2(z0.z + bf16lo(r.y), z0.w + bf16hi(r.y));
           x[u].z = pack_bf16x2(z1.x + bf16lo(r.z), z1.y + bf16hi(r.z));
           x[u].w = pack_bf16x2(z1.z + bf16lo(r.w), z1.w + bf16hi(r.w));
-          hp[idx] = x[u];
         } else {
           x[u] = hp[idx];  // private channels, finished by the local step
         }
+      }
+    }
+    // (no store in the loop above, so that its loads can all be in flight together)
+    if (h != out) {  // h and out the same buffer: out below overwrites it
+#pragma unroll
+      for (int u = 0; u < VPL; ++u) {
+        const int idx = 32 * u + lane;
+        if (idx < nvec && 8 * idx + 8 <= n_s) hp[idx] = x[u];
       }
     }
     float ss = 0.f;
@@ -186,6 +201,109 @@ __global__ void __launch_bounds__(KT_FIN_THREADS, 2)
         op[idx] = make_uint4(o[0], o[1], o[2], o[3]);
       }
     }
+  }
+}
+
+// The norm of the single-device layer's shared-sum mode: one CTA (8 warps) per token, the ranks
+// of that token on its warps.  The token's shared sums (zs row, n_s fp32) are copied once into
+// shared memory (cp.async, double-buffered across the CTA's tokens) and read from there by every
+// rank's warp: rank m's row gets h[c] = bf16(zs[c] + R_m[c]) for c < n_s and its private h[c]
+// (stored by the GEMM) otherwise, then the RMSNorm (fp32 sum of squares of the bf16 row, one
+// warp, the row in registers) and out = h / sqrt(sum / H + eps) * gamma.  h is stored for the
+// shared channels only when it is not the out buffer.  Same arithmetic as tp_finish_kernel.
+constexpr int KZ_THREADS = 256;
+constexpr int KZ_MAX_NS = 4096;
+
+template <int VPL>
+__global__ void __launch_bounds__(KZ_THREADS, 2)
+    rownorm_zs_kernel(const float* __restrict__ zs, const __nv_bfloat16* __restrict__ R, __nv_bfloat16* h,
+                      __nv_bfloat16* out, const __nv_bfloat16* __restrict__ gamma, int64_t tokens, int P, int H,
+                      int n_s, float eps) {
+  __shared__ __align__(16) float s_z[2][KZ_MAX_NS];
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int nvec = H >> 3;
+  const int nz4 = n_s >> 2;  // float4 of a zs row
+  const float inv_h = 1.0f / static_cast<float>(H);
+  const uint4* g4 = reinterpret_cast<const uint4*>(gamma);
+  auto fetch = [&](int64_t tk, int b) {
+    const float4* src = reinterpret_cast<const float4*>(zs + tk * n_s);
+    float4* dst = reinterpret_cast<float4*>(s_z[b]);
+    for (int j = threadIdx.x; j < nz4; j += KZ_THREADS)
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst + j)), "l"(src + j) : "memory");
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  int64_t tk = blockIdx.x;
+  if (tk < tokens) fetch(tk, 0);
+  for (int k = 0; tk < tokens; tk += gridDim.x, ++k) {
+    const int b = k & 1;
+    const bool more = tk + gridDim.x < tokens;
+    if (more) fetch(tk + gridDim.x, b ^ 1);  // the other buffer was released at the last barrier
+    if (more) asm volatile("cp.async.wait_group 1;" ::: "memory");
+    else asm volatile("cp.async.wait_group 0;" ::: "memory");
+    __syncthreads();  // every thread's part of this token's zs row has landed
+    const float4* z4 = reinterpret_cast<const float4*>(s_z[b]);
+    for (int m = warp; m < P; m += KZ_THREADS / 32) {
+      const int64_t row = static_cast<int64_t>(m) * tokens + tk;
+      uint4* hp = reinterpret_cast<uint4*>(h + row * H);
+      const uint4* rp = reinterpret_cast<const uint4*>(R + row * H);
+      uint4 x[VPL];
+#pragma unroll
+      for (int u = 0; u < VPL; ++u) {
+        const int idx = 32 * u + lane;
+        x[u] = make_uint4(0, 0, 0, 0);
+        if (idx < nvec) x[u] = (8 * idx + 8 <= n_s) ? __ldg(rp + idx) : hp[idx];  // residual / private h
+      }
+#pragma unroll
+      for (int u = 0; u < VPL; ++u) {
+        const int idx = 32 * u + lane;
+        if (idx < nvec && 8 * idx + 8 <= n_s) {
+          const uint4 r = x[u];
+          const float4 z0 = z4[2 * idx], z1 = z4[2 * idx + 1];
+          x[u].x = pack_bf16x2(z0.x + bf16lo(r.x), z0.y + bf16hi(r.x));
+          x[u].y = pack_bf16x2(z0.z + bf16lo(r.y), z0.w + bf16hi(r.y));
+          x[u].z = pack_bf16x2(z1.x + bf16lo(r.z), z1.y + bf16hi(r.z));
+          x[u].w = pack_bf16x2(z1.z + bf16lo(r.w), z1.w + bf16hi(r.w));
+        }
+      }
+      if (h != out) {
+#pragma unroll
+        for (int u = 0; u < VPL; ++u) {
+          const int idx = 32 * u + lane;
+          if (idx < nvec && 8 * idx + 8 <= n_s) hp[idx] = x[u];
+        }
+      }
+      float ss = 0.f;
+#pragma unroll
+      for (int u = 0; u < VPL; ++u) {
+        const uint32_t w[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float a = bf16lo(w[e]), c = bf16hi(w[e]);
+          ss = fmaf(a, a, ss);
+          ss = fmaf(c, c, ss);
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, off);
+      const float rstd = rsqrtf(ss * inv_h + eps);
+      uint4* op = reinterpret_cast<uint4*>(out + row * H);
+#pragma unroll
+      for (int u = 0; u < VPL; ++u) {
+        const int idx = 32 * u + lane;
+        if (idx < nvec) {
+          const uint4 g = __ldg(g4 + idx);
+          const uint32_t w[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
+          const uint32_t gw[4] = {g.x, g.y, g.z, g.w};
+          uint32_t o[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            o[e] = pack_bf16x2(bf16lo_p(w[e]) * rstd * bf16lo(gw[e]), bf16hi_p(w[e]) * rstd * bf16hi(gw[e]));
+          op[idx] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+      }
+    }
+    __syncthreads();  // every warp is done with this token's buffer before it is refilled
   }
 }
 

@@ -251,3 +251,33 @@ def test_mixed_block_tma_merge_matches_register_epilogue(p, random_idx):
                          return_all=True)
     assert_h_close(res[0][1], r["h"], "h merged")
     assert_out_close(res[0][0], r["out"], "out merged")
+
+
+# ------------------------------------------------------------------ shared sums stored once
+@pytest.mark.parametrize("T,H,p,with_h", [(600, 1024, 0.5, True), (300, 776, 1.0, True),
+                                          (600, 1280, 0.375, True), (600, 1280, 0.375, False),
+                                          (129, 512, 0.25, True)])
+def test_shared_sums_once_match_per_rank_stores(T, H, p, with_h):
+    """S the first n_s channels with n_s % 8 == 0: with the full workspace the GEMM stores the
+    shared channels' cross-rank sums once (fp32) and the norm kernel adds each rank's residual;
+    with the 256-byte minimum every shared tile stores h for all P ranks.  h has the same bits
+    either way (one fp32 sum plus the residual, one rounding); both match the oracle.  Covers
+    tile-aligned and mixed shared boundaries (480 of 1280), p = 1, a ragged last row block and
+    h written in place into out."""
+    K, P = 1024, 4
+    d = I.make_rowpar_inputs(T, K, H, P, seed=31, x_std=1.0, w_std=0.05, r_std=1.0, gamma="uniform")
+    g = to_dev(d)
+    ref = O.rowpar_forward(d["X"], d["W"], d["R"], d["gamma"], P, p, return_all=True)
+    res = []
+    for ws_bytes in (C.caat_workspace_size(T, K, H, P, C.CAAT_VARIANT_ROWPAR), 256):
+        ws = C.alloc_workspace(ws_bytes)
+        out = torch.empty_like(g["R"])
+        hb = torch.empty_like(g["R"]) if with_h else None
+        C.caat_rowpar_forward(g["X"], g["W"], g["R"], g["gamma"], None, P, p, out, h_out=hb, workspace=ws)
+        torch.cuda.synchronize()
+        assert C.caat_get_device_status() == 0
+        res.append((out.cpu(), hb.cpu() if with_h else None))
+        assert_out_close(res[-1][0], ref["out"], f"out ws={ws_bytes}")
+    if with_h:
+        assert torch.equal(res[0][1], res[1][1])
+        assert_h_close(res[0][1], ref["h"], "h shared sums")
