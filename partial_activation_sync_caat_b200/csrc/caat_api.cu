@@ -957,12 +957,11 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
     const int64_t warps_per_block = caat::K2_THREADS / 32;
     const int64_t blocks = std::min<int64_t>((rows + warps_per_block - 1) / warps_per_block, max_blocks);
     if (zs3) {
-      // every rank's row: shared channels from Zs (the token's cross-rank sum) plus its residual,
-      // private channels from h; then the norm (one warp per row, the row in registers)
-      // one CTA per token (its ranks on the CTA's warps), the token's sums staged once
-      const int64_t fb = std::min<int64_t>(T, int64_t(dev->sm_count) * 2);
+      // one CTA per token (its ranks on the CTA's warps), the token's sums staged once.  A
+      // plain launch: as a programmatic dependent of the GEMM the step took 62 us longer.
       const __nv_bfloat16* rr = reinterpret_cast<const __nv_bfloat16*>(a->residual);
       const int Hi = static_cast<int>(H);
+      const int64_t fb = std::min<int64_t>(T, int64_t(dev->sm_count) * 2);
       if (H <= 1024)
         caat::rownorm_zs_kernel<4><<<fb, caat::KZ_THREADS, 0, ns>>>(zs_buf, rr, hdst, o, g, T, P, Hi, n_s, a->eps);
       else if (H <= 2048)

@@ -206,11 +206,14 @@ __global__ void __launch_bounds__(KT_FIN_THREADS, 2)
 
 // The norm of the single-device layer's shared-sum mode: one CTA (8 warps) per token, the ranks
 // of that token on its warps.  The token's shared sums (zs row, n_s fp32) are copied once into
-// shared memory (cp.async, double-buffered across the CTA's tokens) and read from there by every
+// shared memory (cp.async, a ring of three rows across the CTA's tokens, so that one barrier per
+// token both publishes a row and frees the one refilled next) and read from there by every
 // rank's warp: rank m's row gets h[c] = bf16(zs[c] + R_m[c]) for c < n_s and its private h[c]
 // (stored by the GEMM) otherwise, then the RMSNorm (fp32 sum of squares of the bf16 row, one
 // warp, the row in registers) and out = h / sqrt(sum / H + eps) * gamma.  h is stored for the
 // shared channels only when it is not the out buffer.  Same arithmetic as tp_finish_kernel.
+//   * Tokens are taken from the last one down: the GEMM stores its last rank's private tiles
+//     last, so some of those rows may still be in L2.
 constexpr int KZ_THREADS = 256;
 constexpr int KZ_MAX_NS = 4096;
 
@@ -219,7 +222,7 @@ __global__ void __launch_bounds__(KZ_THREADS, 2)
     rownorm_zs_kernel(const float* __restrict__ zs, const __nv_bfloat16* __restrict__ R, __nv_bfloat16* h,
                       __nv_bfloat16* out, const __nv_bfloat16* __restrict__ gamma, int64_t tokens, int P, int H,
                       int n_s, float eps) {
-  __shared__ __align__(16) float s_z[2][KZ_MAX_NS];
+  __shared__ __align__(16) float s_z[3][KZ_MAX_NS];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int nvec = H >> 3;
@@ -229,16 +232,18 @@ __global__ void __launch_bounds__(KZ_THREADS, 2)
   auto fetch = [&](int64_t tk, int b) {
     const float4* src = reinterpret_cast<const float4*>(zs + tk * n_s);
     float4* dst = reinterpret_cast<float4*>(s_z[b]);
-    for (int j = threadIdx.x; j < nz4; j += KZ_THREADS)
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst + j)), "l"(src + j) : "memory");
+    for (int q = threadIdx.x; q < nz4; q += KZ_THREADS)
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst + q)), "l"(src + q) : "memory");
     asm volatile("cp.async.commit_group;" ::: "memory");
   };
-  int64_t tk = blockIdx.x;
-  if (tk < tokens) fetch(tk, 0);
-  for (int k = 0; tk < tokens; tk += gridDim.x, ++k) {
-    const int b = k & 1;
-    const bool more = tk + gridDim.x < tokens;
-    if (more) fetch(tk + gridDim.x, b ^ 1);  // the other buffer was released at the last barrier
+  int64_t j = blockIdx.x;  // the CTA's k-th token is tokens - 1 - (blockIdx.x + k gridDim.x)
+  if (j < tokens) fetch(tokens - 1 - j, 0);
+  for (int k = 0; j < tokens; j += gridDim.x, ++k) {
+    const int64_t tk = tokens - 1 - j;
+    const int b = k % 3;
+    const bool more = j + gridDim.x < tokens;
+    // the row refilled here held token k - 2, which every warp finished before the last barrier
+    if (more) fetch(tk - gridDim.x, b == 2 ? 0 : b + 1);
     if (more) asm volatile("cp.async.wait_group 1;" ::: "memory");
     else asm volatile("cp.async.wait_group 0;" ::: "memory");
     __syncthreads();  // every thread's part of this token's zs row has landed
@@ -303,7 +308,6 @@ __global__ void __launch_bounds__(KZ_THREADS, 2)
         }
       }
     }
-    __syncthreads();  // every warp is done with this token's buffer before it is refilled
   }
 }
 
