@@ -242,6 +242,15 @@ bool zs_sum_setting() {
   }();
   return v;
 }
+// Shared-sum mode: pairs of pure shared column blocks run as one 256 x 512 unit (tuning;
+// CAAT_WIDE: 1 wherever the mode allows, 0 never; unset: with private units and K >= 8192).
+int wide_setting() {
+  static int v = [] {
+    const char* e = std::getenv("CAAT_WIDE");
+    return (e && *e) ? (*e == '1' ? 1 : 0) : -1;
+  }();
+  return v;
+}
 bool order_env_set() {
   static bool v = [] {
     const char* e = std::getenv("CAAT_ORDER");
@@ -818,6 +827,20 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
   for (int64_t c = 0; c < H; ++c)
     if ((*tmask)[c]) prm.mask_bits[c >> 5] |= 1u << (c & 31);
   prm.nslots = prm.nS + prm.nPriv;
+  // Shared-sum mode in unit order 0: adjacent pure shared blocks two by two as 256 x 512 units
+  // (the MMA of both halves reads one X stage: a quarter fewer operand bytes per FLOP).  The
+  // first blocks of a contiguous S are pure except perhaps the last.  Only with private units
+  // (short: they fill the last round behind the long wide ones) and K >= 8192 (a wide unit's
+  // epilogue no longer overlaps the next wide unit's mainloop, so the mainloop must be long).
+  // Measured on one box: fc2-7b 0.766 -> 0.748 ms; p = 1 (no private units) 0.743 -> 0.751;
+  // K = 4096 0.501 -> 0.507.
+  prm.wide = 0;
+  const bool wide_auto = prm.nPriv > 0 && a->K >= 8192;
+  if (zs3 && prm.order == 0 && (wide_setting() == 1 || (wide_setting() < 0 && wide_auto))) {
+    int pure = 0;
+    while (pure < prm.nS && prm.slist[pure] == pure && prm.ncls[pure] == 1) ++pure;
+    prm.wide = pure / 2;
+  }
   // The CTA-pair kernel (256-token tiles) for all but the smallest token counts.
   const bool pair = pair_possible;
   const int major = ((a->flags & kFlagAMn) ? 1 : 0) | ((a->flags & kFlagBMn) ? 2 : 0);
@@ -880,7 +903,7 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
     prm.t_begin = static_cast<int>(t0);
     prm.t_end = static_cast<int>(t0 + tc);
     prm.n_mblk = static_cast<int>((tc + bm - 1) / bm);
-    const int64_t units = int64_t(prm.n_mblk) * (prm.nS + int64_t(P) * prm.nPriv);
+    const int64_t units = int64_t(prm.n_mblk) * (prm.nS - prm.wide + int64_t(P) * prm.nPriv);
     prm.n_units = static_cast<int>(units);
     if (cudaMemsetAsync(counter, 0, zero_bytes, st) != cudaSuccess) return CAAT_ERR_CUDA;
     if (pair) {

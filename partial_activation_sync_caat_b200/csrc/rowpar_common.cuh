@@ -81,6 +81,8 @@ struct RowparParams {
   int kblk_per_rank;           // ceil(Kp / 64)
   int last_k16;                // 16-wide K steps in the last k-block of a rank (1..4)
   int nS, nPriv;               // n-blocks that have a shared unit / private units
+  int wide;                    // unit order 0, shared-sum mode: the first 2 * wide shared blocks
+                               // (pure, adjacent) run as `wide` 256 x 512 units per row block
   int n_units;
   int fuse_norm;               // 1: normalizer warps produce `Out`; 0: h only
   int publish;                 // 1 (fused norm): count each tile into its (128-row block, rank)
@@ -110,10 +112,12 @@ struct RowparParams {
 struct K1Unit {
   int m, n, rank;   // rank < 0: shared unit
   int slot;         // partial slot of this unit's contribution to each row
+  int wide;         // 1: shared unit of the column blocks n and n + 1 (a 256 x 512 tile)
 };
 
 __device__ __forceinline__ K1Unit k1_decode(int u, const RowparParams& prm) {
   K1Unit un;
+  un.wide = 0;
   if (prm.order == 3) {
     // Staggered: step s holds the shared units of row block s (if s < n_mblk), then the
     // private units of row block s - D (rank-major, n fastest).  Row blocks complete at an even
@@ -206,10 +210,13 @@ __device__ __forceinline__ K1Unit k1_decode(int u, const RowparParams& prm) {
     }
     return un;
   }
-  const int n_shared_units = prm.n_mblk * prm.nS;
+  const int nSu = prm.nS - prm.wide;  // shared units per row block (a wide unit takes two blocks)
+  const int n_shared_units = prm.n_mblk * nSu;
   if (u < n_shared_units) {
-    un.m = u / prm.nS;
-    un.slot = u - un.m * prm.nS;
+    un.m = u / nSu;
+    const int v = u - un.m * nSu;
+    un.wide = v < prm.wide ? 1 : 0;
+    un.slot = un.wide ? 2 * v : v + prm.wide;
     un.n = prm.slist[un.slot];
     un.rank = -1;
   } else {
@@ -585,12 +592,13 @@ __device__ __forceinline__ bool k1_epilogue_tma(uint32_t trow, const RowparParam
 
 // Shared unit in zs_mode 3: the accumulator of the columns below zs_ns (the cross-rank sum of
 // Eq. 22, exact fp32) is stored to Zs [T, zs_ns] by 32 x 32 fp32 boxes (128-byte rows,
-// 128-byte swizzle, clipped at zs_ns and T by the tensor map) through the warp's second box.
-// Nothing else: the residual add and the store of h for every rank move to the norm kernel,
-// which reads Zs once per rank row.
+// 128-byte swizzle, clipped at zs_ns and T by the tensor map) through the warp's first two
+// boxes in turn.  Nothing else: the residual add and the store of h for every rank move to the
+// norm kernel, which reads Zs once per token.
 __device__ __forceinline__ void k1_epilogue_zs(uint32_t trow, const RowparParams& prm, const void* tmZ, int row0,
                                                int n0, uint8_t* bufs, int lane, uint64_t pol) {
   const int nch = min(4, (prm.H - n0 + 63) / 64);
+  int nb = 0;  // boxes stored so far; box nb goes through buffer nb % 2
   for (int c = 0; c < nch; ++c) {
     const int col = n0 + 64 * c;
     if (col >= prm.zs_ns) break;  // warp-uniform
@@ -601,9 +609,10 @@ __device__ __forceinline__ void k1_epilogue_zs(uint32_t trow, const RowparParams
     tmem_wait_ld();
     for (int hf = 0; hf < 2; ++hf) {
       if (col + 32 * hf >= prm.zs_ns) break;  // warp-uniform
-      if (lane == 0) bulk_wait_group_read0();
+      uint8_t* box = bufs + (nb & 1) * K1_EPI_BOX_BYTES;
+      if (lane == 0 && nb >= 2) bulk_wait_group_read1();  // the store two boxes back has read this buffer
       __syncwarp();
-      uint8_t* rowp = bufs + K1_EPI_BOX_BYTES + lane * 128;
+      uint8_t* rowp = box + lane * 128;
 #pragma unroll
       for (int j = 0; j < 8; ++j)
         *reinterpret_cast<uint4*>(rowp + ((j ^ (lane & 7)) << 4)) =
@@ -611,9 +620,10 @@ __device__ __forceinline__ void k1_epilogue_zs(uint32_t trow, const RowparParams
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
-        tma_store_3d(tmZ, bufs + K1_EPI_BOX_BYTES, col + 32 * hf, row0, 0, pol);
+        tma_store_3d(tmZ, box, col + 32 * hf, row0, 0, pol);
         bulk_commit_group();
       }
+      ++nb;
     }
   }
   if (lane == 0) bulk_wait_group_read0();

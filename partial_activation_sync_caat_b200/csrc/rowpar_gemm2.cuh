@@ -145,6 +145,29 @@ __global__ void __launch_bounds__(K1Threads<kFused>::value, 1)
         const int r1 = un.rank < 0 ? prm.P : un.rank + 1;
         const int xrow = prm.t_begin + un.m * (2 * K2P_BM) + static_cast<int>(cta) * K2P_BM;
         const int wrow = un.n * K2P_BN + static_cast<int>(cta) * (K2P_BN / 2);
+        if constexpr (kMajor == 0) {
+          if (un.wide) {
+            // 256 x 512: per k-block one stage with X and the first block's W half, one with
+            // the second block's W half only
+            for (int r = r0; r < r1 && ok; ++r) {
+              for (int kb = 0; kb < prm.kblk_per_rank; ++kb) {
+                if (!mbar_wait(&empty[stage], phase ^ 1, tmo, 23)) { ok = false; break; }
+                uint32_t fbar = mapa_shared(smem_u32(&full[stage]), 0);
+                if (leader) mbar_arrive_expect_tx(&full[stage], 2 * K2P_STAGE_BYTES);
+                tma_load_3d_pair(sA + stage * K2P_A_BYTES, &tmX, fbar, kb * K2P_BK, xrow, r, pol_x);
+                tma_load_3d_pair(sB + stage * K2P_B_BYTES, &tmW, fbar, kb * K2P_BK, wrow, r, pol_w);
+                issued = true;
+                if (++stage == kStages) { stage = 0; phase ^= 1; }
+                if (!mbar_wait(&empty[stage], phase ^ 1, tmo, 23)) { ok = false; break; }
+                fbar = mapa_shared(smem_u32(&full[stage]), 0);
+                if (leader) mbar_arrive_expect_tx(&full[stage], 2 * K2P_B_BYTES);
+                tma_load_3d_pair(sB + stage * K2P_B_BYTES, &tmW, fbar, kb * K2P_BK, wrow + K2P_BN, r, pol_w);
+                if (++stage == kStages) { stage = 0; phase ^= 1; }
+              }
+            }
+            continue;
+          }
+        }
         for (int r = r0; r < r1 && ok; ++r) {
           for (int kb = 0; kb < prm.kblk_per_rank; ++kb) {
             if (!mbar_wait(&empty[stage], phase ^ 1, tmo, 23)) { ok = false; break; }
@@ -187,6 +210,49 @@ __global__ void __launch_bounds__(K1Threads<kFused>::value, 1)
         mbar_arrive(&sempty[slot]);
         if (u >= prm.n_units) break;
         const K1Unit un = k1_decode(u, prm);
+        if constexpr (kMajor == 0) {
+          if (un.wide) {
+            // both accumulators: the first block's columns in buffer local & 1, the second's in
+            // the other (the buffers of tiles local and local + 1)
+            const int b0 = local & 1;
+            const uint32_t ph0 = (local >> 1) & 1, ph1 = ((local + 1) >> 1) & 1;
+            if (!mbar_wait_cluster(&tempty[b0], ph0 ^ 1, tmo, 25)) { ok = false; break; }
+            if (!mbar_wait_cluster(&tempty[b0 ^ 1], ph1 ^ 1, tmo, 25)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t dt0 = tmem_base + static_cast<uint32_t>(b0 * K2P_BN);
+            const uint32_t dt1 = tmem_base + static_cast<uint32_t>((b0 ^ 1) * K2P_BN);
+            const int nkb = prm.P * prm.kblk_per_rank;
+            int kb_in_rank = 0;
+            for (int j = 0; j < nkb; ++j) {
+              const int sa = stage;  // X and the first block's W half
+              if (!mbar_wait(&full[stage], phase, tmo, 26)) { ok = false; break; }
+              if (++stage == kStages) { stage = 0; phase ^= 1; }
+              const int sb = stage;  // the second block's W half
+              if (!mbar_wait(&full[stage], phase, tmo, 26)) { ok = false; break; }
+              if (++stage == kStages) { stage = 0; phase ^= 1; }
+              const int nk16 = (kb_in_rank == prm.kblk_per_rank - 1) ? prm.last_k16 : (K2P_BK / 16);
+              const uint32_t a_addr = smem_u32(sA + sa * K2P_A_BYTES);
+              const uint32_t b0_addr = smem_u32(sB + sa * K2P_B_BYTES);
+              const uint32_t b1_addr = smem_u32(sB + sb * K2P_B_BYTES);
+              for (int kk = 0; kk < nk16; ++kk)
+                umma_bf16_pair(dt0, sw128_kmajor_desc(a_addr + kk * 32), sw128_kmajor_desc(b0_addr + kk * 32), idesc,
+                               (j > 0 || kk > 0) ? 1u : 0u);
+              for (int kk = 0; kk < nk16; ++kk)
+                umma_bf16_pair(dt1, sw128_kmajor_desc(a_addr + kk * 32), sw128_kmajor_desc(b1_addr + kk * 32), idesc,
+                               (j > 0 || kk > 0) ? 1u : 0u);
+              umma_commit_pair_mc(&empty[sa], 0x3);
+              umma_commit_pair_mc(&empty[sb], 0x3);
+              if (++kb_in_rank == prm.kblk_per_rank) kb_in_rank = 0;
+            }
+            if (!ok) break;
+            if (!(prm.flags & K1_FLAG_TEST_STALL)) {
+              umma_commit_pair_mc(&tfull[b0], 0x3);
+              umma_commit_pair_mc(&tfull[b0 ^ 1], 0x3);
+            }
+            local += 2;
+            continue;
+          }
+        }
         const int buf = local & 1;
         const uint32_t bph = (local >> 1) & 1;
         if (!mbar_wait_cluster(&tempty[buf], bph ^ 1, tmo, 25)) { ok = false; break; }
@@ -248,6 +314,26 @@ __global__ void __launch_bounds__(K1Threads<kFused>::value, 1)
       u = __shfl_sync(0xFFFFFFFFu, u, 0);
       if (!ok || u >= prm.n_units) break;
       const K1Unit un = k1_decode(u, prm);
+      if (un.wide) {
+        // shared-sum mode, 256 x 512: the two column blocks' accumulators in turn, each released
+        // as soon as it is stored (the next unit's first block may start in it)
+        const int row0 = prm.t_begin + un.m * (2 * K2P_BM) + static_cast<int>(cta) * K2P_BM + q * 32;
+        for (int hh = 0; hh < 2 && ok; ++hh) {
+          const int bh = (local + hh) & 1;
+          if (lane == 0) ok = mbar_wait(&tfull[bh], ((local + hh) >> 1) & 1, tmo, 29) ? 1 : 0;
+          ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t trow = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(bh * K2P_BN);
+          k1_epilogue_zs(trow, prm, &tmZ, row0, (un.n + hh) * K2P_BN, my_bufs, lane, pol_h);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(tempty_leader[bh]);
+        }
+        if (!ok) break;
+        local += 2;
+        continue;
+      }
       const int buf = local & 1;
       const uint32_t bph = (local >> 1) & 1;
       if (lane == 0) ok = mbar_wait(&tfull[buf], bph, tmo, 29) ? 1 : 0;

@@ -1,6 +1,9 @@
 """GPU parity of the row-parallel layer (tcgen05 GEMM + partial channel-reduce epilogue +
 RMSNorm kernels, called through the C ABI) against the float64 oracle."""
 import math
+import os
+import subprocess
+import sys
 
 import numpy as np
 import pytest
@@ -256,14 +259,17 @@ def test_mixed_block_tma_merge_matches_register_epilogue(p, random_idx):
 # ------------------------------------------------------------------ shared sums stored once
 @pytest.mark.parametrize("T,H,p,with_h", [(600, 1024, 0.5, True), (300, 776, 1.0, True),
                                           (600, 1280, 0.375, True), (600, 1280, 0.375, False),
-                                          (129, 512, 0.25, True)])
+                                          (129, 512, 0.25, True), (520, 2048, 0.625, True),
+                                          (520, 2048, 0.625, False)])
 def test_shared_sums_once_match_per_rank_stores(T, H, p, with_h):
     """S the first n_s channels with n_s % 8 == 0: with the full workspace the GEMM stores the
     shared channels' cross-rank sums once (fp32) and the norm kernel adds each rank's residual;
     with the 256-byte minimum every shared tile stores h for all P ranks.  h has the same bits
     either way (one fp32 sum plus the residual, one rounding); both match the oracle.  Covers
     tile-aligned and mixed shared boundaries (480 of 1280), p = 1, a ragged last row block and
-    h written in place into out."""
+    h written in place into out.  Pairs of whole shared column blocks run as 256 x 512 units:
+    1024 x 0.5 has one, 776 x 1.0 two (the second ending in an 8-channel block), 2048 x 0.625
+    two and one ordinary shared unit."""
     K, P = 1024, 4
     d = I.make_rowpar_inputs(T, K, H, P, seed=31, x_std=1.0, w_std=0.05, r_std=1.0, gamma="uniform")
     g = to_dev(d)
@@ -281,3 +287,35 @@ def test_shared_sums_once_match_per_rank_stores(T, H, p, with_h):
     if with_h:
         assert torch.equal(res[0][1], res[1][1])
         assert_h_close(res[0][1], ref["h"], "h shared sums")
+
+
+def test_shared_sums_wide_units_long_k():
+    """K = 8192 with private channels: the default takes the 256 x 512 shared units (two whole
+    shared column blocks per unit) for S = the first 512 of 1024 channels.  Same h bits as the
+    per-rank-store path; both match the oracle."""
+    T, K, H, P, p = 520, 8192, 1024, 4, 0.5
+    d = I.make_rowpar_inputs(T, K, H, P, seed=32, x_std=1.0, w_std=0.02, r_std=1.0, gamma="uniform")
+    g = to_dev(d)
+    ref = O.rowpar_forward(d["X"], d["W"], d["R"], d["gamma"], P, p, return_all=True)
+    hs = []
+    for ws_bytes in (C.caat_workspace_size(T, K, H, P, C.CAAT_VARIANT_ROWPAR), 256):
+        ws = C.alloc_workspace(ws_bytes)
+        out, hb = torch.empty_like(g["R"]), torch.empty_like(g["R"])
+        C.caat_rowpar_forward(g["X"], g["W"], g["R"], g["gamma"], None, P, p, out, h_out=hb, workspace=ws)
+        torch.cuda.synchronize()
+        assert C.caat_get_device_status() == 0
+        assert_out_close(out.cpu(), ref["out"], f"out ws={ws_bytes}")
+        hs.append(hb.cpu())
+    assert torch.equal(hs[0], hs[1])
+    assert_h_close(hs[0], ref["h"], "h wide")
+
+
+@pytest.mark.skipif(os.environ.get("CAAT_WIDE") is not None, reason="already the child run")
+def test_shared_sums_with_wide_units_forced():
+    """The shared-sum cases above with 256 x 512 units wherever two whole shared blocks pair up
+    (CAAT_WIDE=1, read once per process: a child pytest), also at p = 1 and short K."""
+    env = dict(os.environ, CAAT_WIDE="1")
+    r = subprocess.run([sys.executable, "-m", "pytest", __file__, "-q", "-m", "gpu", "-p", "no:cacheprovider",
+                        "-k", "shared_sums_once or p_sweep_ragged or single_rank"],
+                       env=env, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
