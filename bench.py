@@ -406,7 +406,7 @@ class Case:
         return n_intervals + (1 if overlapped else 0)
 
 
-def time_case(case, steps, warmup, world=1, sample_clocks=False, local=0, soak_ms=500.0):
+def time_case(case, steps, warmup, world=1, sample_clocks=False, local=0, soak_ms=500.0, warmup_ms=0.0):
     """Times exactly `steps` steps after `warmup` untimed ones: CUDA events on the launching
     stream, synchronize (and a barrier across ranks) on both sides; the per-kernel split comes
     from `steps` more calls with the library's event recorder, after the timed region.  Workloads whose bytes fit
@@ -414,15 +414,22 @@ def time_case(case, steps, warmup, world=1, sample_clocks=False, local=0, soak_m
     would leave dirty lines whose write-back the next step would pay for); each step is then
     timed alone, and is one replay of a CUDA graph holding the one library call (the same
     kernels), so that the host's submission after the flush does not leave the GPU idle inside
-    the timed interval.  Returns (ms_local over all steps, per-call kernel intervals, clocks)."""
+    the timed interval.  `warmup_ms` > 0: after the `warmup` steps, more untimed steps until that
+    much wall time has passed (a part coming out of idle ramps its clocks over some milliseconds).
+    Returns (ms_local over all steps, per-call kernel intervals, clocks)."""
     import torch
     import torch.distributed as dist
     from partial_activation_sync_caat_b200 import caat as C
     stream = torch.cuda.current_stream()
     timing = C.Timing(capacity=steps + 8)
+    t_w = time.perf_counter()
     for _ in range(warmup):
         case.step()
     torch.cuda.synchronize()
+    while (time.perf_counter() - t_w) * 1e3 < warmup_ms:
+        for _ in range(4):
+            case.step()
+        torch.cuda.synchronize()
     if C.caat_get_device_status() != 0:
         raise SystemExit(f"device status set during warm-up of {case.name}")
     flush_buf = torch.ones(3 * L2_BYTES // 4, dtype=torch.float32, device="cuda") if case.flush else None
@@ -522,7 +529,8 @@ def sub_workloads(args, peaks, peak_src):
         torch.cuda.synchronize()
         time.sleep(1.0)
         steps = 20
-        ms_local, per_kernel, clocks = time_case(case, steps, 5, sample_clocks=True, soak_ms=150.0)
+        # 5 warm-up steps, and at least 50 ms of them: the part is coming out of that idle second
+        ms_local, per_kernel, clocks = time_case(case, steps, 5, sample_clocks=True, soak_ms=150.0, warmup_ms=50.0)
         ms = ms_local / steps
         km = kernel_means(per_kernel)
         tflops = case.flops / ms / 1e9
