@@ -16,6 +16,11 @@
 //     TMEM-empty barrier.
 //   * Dynamic scheduling: the leader's producer draws a unit from the global counter and
 //     writes it into both CTAs' broadcast ring.
+//   * Wide shared units (zs_mode 3, forward only): two adjacent whole shared column blocks as one
+//     256 x 512 unit.  Per k-block one ring stage holds X and the first block's W half, the
+//     next only the second block's W half; the MMA issuer runs both N = 256 halves on the same
+//     X stage, into the two TMEM buffers, so the unit counts as two tiles for the buffers'
+//     phases.  The epilogue stores each half's fp32 sums and releases its buffer in turn.
 // The RMSNorm is fused (rowpar_common.cuh): warps 6-9 of each CTA normalize completed row
 // blocks.
 // kMajor (GEMM-only use by the backward): bit 0 = A stored MN-major ([K][M], M contiguous),
