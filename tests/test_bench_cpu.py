@@ -85,3 +85,31 @@ def test_clock_record_from_nvml_samples():
     c = s.stop()
     assert c["sm_mhz"] == 1500 and c["samples"] == 3 and c["reasons"] == ["sw_power_cap"]
     assert c["power_w_max"] == 800.0
+
+
+def test_shared_sum_norm_rule(monkeypatch):
+    """The bench names the norm kernel (and counts its Zs read) from the library's rule for the
+    shared-sum path: a contiguous S with n_s % 8 == 0 and n_s > 0, H <= 4096, T > 128, the plain
+    forward (no fused / overlapped / beside-the-GEMM norm, no permuted W), CAAT_ZS_SUM not 0."""
+    from types import SimpleNamespace
+    from partial_activation_sync_caat_b200 import caat as C
+    monkeypatch.delenv("CAAT_ZS_SUM", raising=False)
+
+    def case(**kw):
+        base = dict(H=4096, p=0.5, T=8192, bwd=False, rand=False, flags=0)
+        base.update(kw)
+        return SimpleNamespace(**base)
+
+    assert bench.shared_sums_once(case())
+    assert bench.shared_sums_once(case(p=1.0))
+    assert not bench.shared_sums_once(case(p=0.0))            # no shared channels
+    assert not bench.shared_sums_once(case(H=776, p=0.5))     # n_s = 388, not a multiple of 8
+    assert not bench.shared_sums_once(case(H=8192))           # rows wider than 4096
+    assert not bench.shared_sums_once(case(T=128))            # one-CTA kernel
+    assert not bench.shared_sums_once(case(rand=True))        # a sync list (permuted W)
+    assert not bench.shared_sums_once(case(bwd=True))
+    for f in (C.CAAT_FLAG_FUSED_NORM, C.CAAT_FLAG_OVERLAP_NORM, C.CAAT_FLAG_NORM_BESIDE_GEMM,
+              C.CAAT_FLAG_SINGLE_CTA, C.CAAT_FLAG_W_PERMUTED, C.CAAT_FLAG_FORCE_DECODE_PATH):
+        assert not bench.shared_sums_once(case(flags=f))
+    monkeypatch.setenv("CAAT_ZS_SUM", "0")
+    assert not bench.shared_sums_once(case())
