@@ -10,7 +10,10 @@
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
+#include <functional>
 #include <mutex>
+#include <queue>
+#include <unordered_map>
 #include <new>
 #include <vector>
 
@@ -250,6 +253,46 @@ int wide_setting() {
     return (e && *e) ? (*e == '1' ? 1 : 0) : -1;
   }();
   return v;
+}
+// How many pairs of whole shared column blocks per row block to run as 256 x 512 units when
+// there are no private units (every shared block pure): the dynamic scheduler's makespan,
+// simulated on `pairs` CTA pairs for wide units first (each worth 1.84 ordinary units, as
+// measured at fc2-7b p = 1), then the ordinary shared units; the count with the shortest
+// makespan (the fewer wide units on a tie).  Cached per shape.
+int wide_count_by_schedule(int n_mblk, int nS, int pure_pairs, int pairs) {
+  static std::mutex mu;
+  static std::unordered_map<uint64_t, int> memo;
+  const uint64_t key = (uint64_t(n_mblk) << 40) ^ (uint64_t(nS) << 24) ^ (uint64_t(pure_pairs) << 12) ^ uint64_t(pairs);
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    auto it = memo.find(key);
+    if (it != memo.end()) return it->second;
+  }
+  constexpr double kWideCost = 1.84;
+  double best = 0.0;
+  int best_w = 0;
+  for (int w = 0; w <= pure_pairs; ++w) {
+    std::priority_queue<double, std::vector<double>, std::greater<double>> free_at;
+    for (int q = 0; q < std::max(pairs, 1); ++q) free_at.push(0.0);
+    double end = 0.0;
+    auto run = [&](int count, double cost) {
+      for (int i = 0; i < count; ++i) {
+        const double t = free_at.top() + cost;
+        free_at.pop();
+        free_at.push(t);
+        end = std::max(end, t);
+      }
+    };
+    run(n_mblk * w, kWideCost);
+    run(n_mblk * (nS - 2 * w), 1.0);
+    if (w == 0 || end < best - 1e-9) {
+      best = end;
+      best_w = w;
+    }
+  }
+  std::lock_guard<std::mutex> lk(mu);
+  memo[key] = best_w;
+  return best_w;
 }
 bool order_env_set() {
   static bool v = [] {
@@ -835,11 +878,15 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
   // Measured on one box: fc2-7b 0.766 -> 0.748 ms; p = 1 (no private units) 0.743 -> 0.751;
   // K = 4096 0.501 -> 0.507.
   prm.wide = 0;
-  const bool wide_auto = prm.nPriv > 0 && a->K >= 8192;
-  if (zs3 && prm.order == 0 && (wide_setting() == 1 || (wide_setting() < 0 && wide_auto))) {
+  if (zs3 && prm.order == 0 && wide_setting() != 0 && (wide_setting() == 1 || a->K >= 8192)) {
     int pure = 0;
     while (pure < prm.nS && prm.slist[pure] == pure && prm.ncls[pure] == 1) ++pure;
     prm.wide = pure / 2;
+    // without private units the short ordinary shared units fill the last round: take the
+    // number of wide units with the shortest simulated schedule
+    if (wide_setting() < 0 && prm.nPriv == 0)
+      prm.wide = wide_count_by_schedule(static_cast<int>((T + 2 * caat::K2P_BM - 1) / (2 * caat::K2P_BM)), prm.nS,
+                                        pure / 2, dev->max_pairs);
   }
   // The CTA-pair kernel (256-token tiles) for all but the smallest token counts.
   const bool pair = pair_possible;

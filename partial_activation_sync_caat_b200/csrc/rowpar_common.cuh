@@ -210,13 +210,22 @@ __device__ __forceinline__ K1Unit k1_decode(int u, const RowparParams& prm) {
     }
     return un;
   }
-  const int nSu = prm.nS - prm.wide;  // shared units per row block (a wide unit takes two blocks)
+  // shared units: every row block's wide units first (two blocks each), then the remaining
+  // ordinary shared units of every row block (short ones last), then the private units
+  const int nSu = prm.nS - prm.wide;   // shared units per row block
+  const int nSo = nSu - prm.wide;      // ordinary ones among them
+  const int n_wide_units = prm.n_mblk * prm.wide;
   const int n_shared_units = prm.n_mblk * nSu;
-  if (u < n_shared_units) {
-    un.m = u / nSu;
-    const int v = u - un.m * nSu;
-    un.wide = v < prm.wide ? 1 : 0;
-    un.slot = un.wide ? 2 * v : v + prm.wide;
+  if (u < n_wide_units) {
+    un.m = u / prm.wide;
+    un.slot = 2 * (u - un.m * prm.wide);
+    un.wide = 1;
+    un.n = prm.slist[un.slot];
+    un.rank = -1;
+  } else if (u < n_shared_units) {
+    const int v = u - n_wide_units;
+    un.m = v / nSo;
+    un.slot = 2 * prm.wide + (v - un.m * nSo);
     un.n = prm.slist[un.slot];
     un.rank = -1;
   } else {
