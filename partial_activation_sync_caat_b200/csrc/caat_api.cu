@@ -246,7 +246,8 @@ bool zs_sum_setting() {
   return v;
 }
 // Shared-sum mode: pairs of pure shared column blocks run as one 256 x 512 unit (tuning;
-// CAAT_WIDE: 1 wherever the mode allows, 0 never; unset: with private units and K >= 8192).
+// CAAT_WIDE: 1 every pair, 0 never; unset: for K >= 8192, every pair when there are private
+// units, else the count a simulated schedule favours).
 int wide_setting() {
   static int v = [] {
     const char* e = std::getenv("CAAT_WIDE");
@@ -872,11 +873,12 @@ caat_status launch_rowpar(const caat_rowpar_args* a, const std::vector<uint8_t>&
   prm.nslots = prm.nS + prm.nPriv;
   // Shared-sum mode in unit order 0: adjacent pure shared blocks two by two as 256 x 512 units
   // (the MMA of both halves reads one X stage: a quarter fewer operand bytes per FLOP).  The
-  // first blocks of a contiguous S are pure except perhaps the last.  Only with private units
-  // (short: they fill the last round behind the long wide ones) and K >= 8192 (a wide unit's
-  // epilogue no longer overlaps the next wide unit's mainloop, so the mainloop must be long).
-  // Measured on one box: fc2-7b 0.766 -> 0.748 ms; p = 1 (no private units) 0.743 -> 0.751;
-  // K = 4096 0.501 -> 0.507.
+  // first blocks of a contiguous S are pure except perhaps the last.  Only for K >= 8192 (a
+  // wide unit's epilogue no longer overlaps the next wide unit's mainloop, so the mainloop must
+  // be long): measured on one box, fc2-7b 0.766 -> 0.748 ms, K = 4096 0.501 -> 0.507 ms.  The
+  // wide units run first and the short units after them fill the last round: the private
+  // units, or without any (p = 1) the ordinary shared units, with the wide count taken from a
+  // simulated schedule (fc2-7b p = 1: 0.736 -> 0.710 ms; all pairs wide: 0.751 ms).
   prm.wide = 0;
   if (zs3 && prm.order == 0 && wide_setting() != 0 && (wide_setting() == 1 || a->K >= 8192)) {
     int pure = 0;
