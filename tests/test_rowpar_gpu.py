@@ -319,3 +319,27 @@ def test_shared_sums_with_wide_units_forced():
                         "-k", "shared_sums_once or p_sweep_ragged or single_rank"],
                        env=env, capture_output=True, text=True, timeout=900)
     assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
+
+
+def test_shared_sums_all_shared_schedule_chosen_wide_units():
+    """p = 1 (no private channels) with K = 8192 and 24 row blocks of 4 shared column blocks: on
+    the 74 CTA pairs of a B200 the host's simulated schedule runs one of each row block's two
+    pairs of blocks as a 256 x 512 unit and the other two blocks as ordinary units after every
+    wide one.  h has the per-rank-store path's bits (the 256-byte workspace); out matches the
+    oracle on sampled rows."""
+    T, K, H, P, p = 6144, 8192, 1024, 4, 1.0
+    d = I.make_rowpar_inputs(T, K, H, P, seed=33, x_std=1.0, w_std=0.02, r_std=1.0, gamma="uniform")
+    g = to_dev(d)
+    outs, hs = [], []
+    for ws_bytes in (C.caat_workspace_size(T, K, H, P, C.CAAT_VARIANT_ROWPAR), 256):
+        ws = C.alloc_workspace(ws_bytes)
+        out, hb = torch.empty_like(g["R"]), torch.empty_like(g["R"])
+        C.caat_rowpar_forward(g["X"], g["W"], g["R"], g["gamma"], None, P, p, out, h_out=hb, workspace=ws)
+        torch.cuda.synchronize()
+        assert C.caat_get_device_status() == 0
+        outs.append(out.cpu())
+        hs.append(hb.cpu())
+    assert torch.equal(hs[0], hs[1])
+    rows = I.sample_rows(T, 48, seed=3)
+    ref = O.rowpar_rows(d["X"], d["W"], d["R"], d["gamma"], P, p, rows)
+    assert_out_close(outs[0][:, torch.as_tensor(rows), :], ref, "p=1 schedule-chosen wide units")
